@@ -1,0 +1,418 @@
+#!/usr/bin/env python
+"""Benchmark of the GlowQ corrected quantised linear layer on B200.
+
+A step is one pass of the whole hot path over one batch of synthetic tokens:
+the LLaMA-2-7B attention linears at decode T=1 -- the Q/K/V input-sharing
+group (R = X B^T once, y_i = X w_hat_i^T + R A_i^T for Q, K, V) followed by the
+solo o_proj (its own R inline), INT4 g128 weights, rank 64.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl glowq|reference]
+
+Prints one JSON line (rank 0).  `value` is whole-job tokens/s from CUDA events
+around exactly K steps (all ranks, max over ranks); weights are rotated over
+enough replicas that every step streams its weights from HBM (inputs larger
+than L2).  `e2e` is the same metric through the public API with the token
+activations copied from pinned host memory and the outputs copied back each
+step.  `--impl reference` times the CPU oracle (float64 C) on a bounded sample
+of the same workload.  Multi-GPU runs are independent replicas (the layer has
+no cross-GPU exchange): weak scaling, no data-path collective.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GlowQ linear tok/s (decode T=1, prefill T=2048); % of HBM / tensor roofline"
+WORKLOAD = "llama2_7b_attn_decode"
+R_RANK = 64
+D = 4096
+QKV_OUTS = [4096, 4096, 4096]
+O_OUTS = [4096]
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p.get("bf16_tflops_sustained", 0)) or None, "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def group_bytes(outs, d, r, T, with_factors=True):
+    """Algorithmic HBM bytes of one group call: INT4 codes + fp16 scales + u8 zeros,
+    A_i (fp16) and B (fp16, once per group), X and R in, Y out."""
+    O = sum(outs)
+    b = O * d // 2 + O * (d // 128) * 3 + T * d * 2 + T * O * 2
+    if with_factors and r:
+        b += O * r * 2 + r * d * 2 + 2 * T * r * 2
+    return b
+
+
+def group_flops(outs, d, r, T):
+    O = sum(outs)
+    return 2 * T * O * d + (2 * T * r * d + 2 * T * O * r if r else 0)
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        loaded = [r[0] for r in rows if r[2] > 200.0] or [r[0] for r in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+
+
+# ------------------------------------------------------------------ workload
+
+def build_replicas(n_rep, T, device, seed=0):
+    import torch
+    from rank_error_correction_b200 import glowq, synth
+    reps = []
+    for i in range(n_rep):
+        rep = {}
+        for name, outs, sub in (("qkv", QKV_OUTS, 0), ("o_proj", O_OUTS, 10)):
+            mods = []
+            for j, O in enumerate(outs):
+                W = synth.device_weights(O, D, seed, sub=1000 * i + sub + j, device=device)
+                q, s, z = glowq.pack_int4(W)
+                del W
+                mods.append(glowq.QModule(q, s, z))
+            As, B = synth.device_factors(outs, D, R_RANK, seed, sub=1000 * i + sub, device=device)
+            for m, A in zip(mods, As):
+                m.A = A
+            rep[name] = (mods, B)
+        reps.append(rep)
+    torch.cuda.synchronize()
+    return reps
+
+
+def make_io(T, device, seed=0):
+    import torch
+    from rank_error_correction_b200 import glowq, synth
+    X = torch.from_numpy(synth.activations(T, D, synth.ALPHA_QKV, seed=seed)).to(device)
+    X2 = torch.from_numpy(synth.activations(T, D, synth.ALPHA_QKV, seed=seed, sub=1)).to(device)
+    Yqkv = torch.empty((T, sum(QKV_OUTS)), dtype=torch.float16, device=device)
+    Yo = torch.empty((T, O_OUTS[0]), dtype=torch.float16, device=device)
+    R = torch.empty((T, R_RANK), dtype=torch.float16, device=device)
+    ws = glowq.alloc_workspace(T, R_RANK, device)
+    views, c = [], 0
+    for O in QKV_OUTS:
+        views.append(Yqkv[:, c:c + O])
+        c += O
+    return dict(X=X, X2=X2, Yqkv=Yqkv, views=views, Yo=Yo, R=R, ws=ws)
+
+
+def run_step(rep, io, stream=None):
+    from rank_error_correction_b200 import glowq
+    mods, B = rep["qkv"]
+    glowq.group_forward(mods, B, io["X"], Ys=io["views"], R_out=io["R"], workspace=io["ws"], stream=stream)
+    mo, Bo = rep["o_proj"]
+    glowq.solo_forward(mo[0], Bo, io["X2"], Y=io["Yo"], workspace=io["ws"], stream=stream)
+
+
+def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
+    """Graph-replayed timing of `steps` steps; also per-group-call event timing."""
+    import torch
+    reps = build_replicas(n_rep, T, device)
+    io = make_io(T, device)
+    stream = torch.cuda.Stream(device=device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, 3)):
+            run_step(reps[i % n_rep], io)
+    stream.synchronize()
+    # one graph holding all timed steps, with event-record nodes around each group call
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            rep = reps[i % n_rep]
+            evs[i][0].record()
+            mods, B = rep["qkv"]
+            from rank_error_correction_b200 import glowq
+            glowq.group_forward(mods, B, io["X"], Ys=io["views"], R_out=io["R"], workspace=io["ws"])
+            evs[i][1].record()
+            mo, Bo = rep["o_proj"]
+            glowq.solo_forward(mo[0], Bo, io["X2"], Y=io["Yo"], workspace=io["ws"])
+            evs[i][2].record()
+    # warm the graph once (untimed), then time one replay of exactly `steps` steps
+    g.replay()
+    stream.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(gpu_index) if want_clocks else None
+    if sampler:
+        sampler.__enter__()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record()
+        g.replay()
+        t1.record()
+    stream.synchronize()
+    if sampler:
+        sampler.__exit__()
+    total_ms = t0.elapsed_time(t1)
+    qkv_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(steps)]
+    o_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(steps)]
+    del g
+    return dict(total_ms=total_ms, qkv_ms=statistics.mean(qkv_ms), o_ms=statistics.mean(o_ms),
+                qkv_ms_median=statistics.median(qkv_ms), clocks=sampler.summary() if sampler else None,
+                reps=reps, io=io)
+
+
+def time_e2e(T, steps, device, reps, io):
+    """Public-API steps with host<->device copies of the step's activations/outputs."""
+    import torch
+    Xh = io["X"].cpu().pin_memory()
+    X2h = io["X2"].cpu().pin_memory()
+    Yh = torch.empty(io["Yqkv"].shape, dtype=torch.float16).pin_memory()
+    Yoh = torch.empty(io["Yo"].shape, dtype=torch.float16).pin_memory()
+    n = min(steps, 200)
+
+    def one(i):
+        io["X"].copy_(Xh, non_blocking=True)
+        io["X2"].copy_(X2h, non_blocking=True)
+        run_step(reps[i % len(reps)], io)
+        Yh.copy_(io["Yqkv"], non_blocking=True)
+        Yoh.copy_(io["Yo"], non_blocking=True)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(n):
+        one(i)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / n
+    h2d = Xh.numel() * 2 + X2h.numel() * 2
+    d2h = Yh.numel() * 2 + Yoh.numel() * 2
+    return ms, h2d, d2h, n
+
+
+# ------------------------------------------------------------ oracle timing
+
+def oracle_sample(T=1, rows_per_module=512, seed=0):
+    """Oracle forward (float64 C, one thread) over a row sample of every module of the step."""
+    import numpy as np
+    import oracle
+    from rank_error_correction_b200 import synth
+    rows_total = sum(QKV_OUTS) + sum(O_OUTS)
+    X = synth.bits(synth.activations(T, D, synth.ALPHA_QKV, seed=seed))
+    mods = []
+    for j, O in enumerate(QKV_OUTS + O_OUTS):
+        W = synth.weights(rows_per_module, D, seed=seed, stream_sub=900 + j)
+        q, s, z = oracle.quantize_int4(W)
+        A = (np.random.default_rng(j).standard_normal((rows_per_module, R_RANK)) * 0.005).astype(np.float16)
+        mods.append((q, s, z, synth.bits(A)))
+    B = synth.bits((np.random.default_rng(99).standard_normal((R_RANK, D)) * 0.01).astype(np.float16))
+    t0 = time.perf_counter()
+    # QKV: one shared R; o_proj: its own R
+    oracle.group_forward(mods[:3], B, X)
+    q, s, z, A = mods[3]
+    oracle.solo_forward(q, s, z, A, B, X)
+    dt = time.perf_counter() - t0
+    frac = (4 * rows_per_module) / rows_total
+    return dt, frac
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    T = 1
+    steps, warmup = args.steps, args.warmup
+    # size each step so the whole run stays within a few minutes
+    rows = 256
+    for _ in range(warmup):
+        oracle_sample(T, rows)
+    times = []
+    frac = None
+    for _ in range(steps):
+        dt, frac = oracle_sample(T, rows)
+        times.append(dt)
+    step_s = sum(times) / len(times) / frac          # scaled to the full step
+    value = T / step_s
+    line = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
+            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": f"{WORKLOAD} (QKV group + o_proj solo, d=4096, r=64, INT4 g128)",
+                       "tokens": T, "sample": f"{rows} rows per module of 16384; scaled by row fraction"},
+            "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{rows} of 4096 rows per module x 4 modules per step, {steps} steps"},
+            "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="glowq", choices=["glowq", "reference"])
+    ap.add_argument("--replicas", type=int, default=8)
+    ap.add_argument("--no-extra", action="store_true", help="skip the T=4/16 decode lines")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    from rank_error_correction_b200 import build, glowq
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if rank == 0 or not os.path.exists(glowq.LIB_PATH):
+        build.build()
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
+        pg = dist
+        dist.barrier()
+    glowq.lib()
+
+    hbm_peak, tf_peak, tf_sust, peak_src = _peaks()
+    T = 1
+    res = time_decode(T, args.steps, args.warmup, device, args.replicas, local, want_clocks=(rank == 0))
+    total_ms = res["total_ms"]
+    if pg is not None:
+        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = world * T * args.steps / (total_ms / 1e3)
+    qkv_bytes = group_bytes(QKV_OUTS, D, R_RANK, T)
+    achieved = qkv_bytes / (res["qkv_ms"] * 1e-3) / 1e9
+    launches_per_step = 3 + 3          # (rproj_partial, rproj_reduce, corrected_gemv) x 2 calls
+    e2e_ms, h2d, d2h, _ = time_e2e(T, args.steps, device, res["reps"], res["io"])
+
+    extra = []
+    if not args.no_extra:
+        for Tx in (4, 16):
+            r2 = time_decode(Tx, min(args.steps, 100), args.warmup, device, args.replicas, local, want_clocks=False)
+            b = group_bytes(QKV_OUTS, D, R_RANK, Tx)
+            extra.append({"tokens": Tx, "tok_s": Tx * min(args.steps, 100) / (r2["total_ms"] / 1e3),
+                          "ms_per_step": r2["total_ms"] / min(args.steps, 100),
+                          "qkv_group_us": r2["qkv_ms"] * 1e3, "o_proj_us": r2["o_ms"] * 1e3,
+                          "qkv_group_GBps": b / (r2["qkv_ms"] * 1e-3) / 1e9,
+                          "qkv_group_hbm_frac": b / (r2["qkv_ms"] * 1e-3) / 1e9 / hbm_peak})
+            del r2
+
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        times, frac = [], None
+        t_start = time.perf_counter()
+        while time.perf_counter() - t_start < 10.0 and len(times) < 20:
+            dt, frac = oracle_sample(1, 512)
+            times.append(dt)
+        step_s = statistics.mean(times) / frac
+        cpu = {"value": 1.0 / step_s, "unit": "tok/s", "cores": 1, "kind": "oracle",
+               "sample": f"T=1, 512 of 4096 rows of each of the 4 modules per sample, {len(times)} samples, "
+                         f"scaled by the row fraction ({frac:.4f})"}
+
+    if rank == 0:
+        traffic = None
+        tr_path = os.path.join(ROOT, "profiles", "traffic.json")
+        if os.path.exists(tr_path):
+            try:
+                traffic = json.load(open(tr_path)).get("corrected_gemv_kernel<1> qkv T=1")
+            except Exception:
+                traffic = None
+        line = {
+            "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp16 x int4 -> fp32 acc", "data": "synthetic",
+            "config": {"workload": "LLaMA-2-7B attention linears, decode T=1: Q/K/V group (3x4096x4096) + "
+                                   "o_proj solo (4096x4096), INT4 g128 asym, r=64 fp16 factors",
+                       "tokens": T, "replicas": args.replicas,
+                       "l2": f"inputs larger than L2: {args.replicas} weight replicas rotated "
+                             f"({args.replicas * 38.4:.0f} MB)", "graph": "one CUDA graph of all timed steps",
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "roofline": {"bound": "hbm", "kernel": "glowq_group_forward (Q/K/V, T=1)", "achieved": achieved,
+                         "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s", "frac": achieved / hbm_peak,
+                         "traffic": traffic, "algorithmic_bytes": qkv_bytes,
+                         "us_per_launch": res["qkv_ms"] * 1e3},
+            "o_proj_us": res["o_ms"] * 1e3,
+            "e2e": {"value": T / (e2e_ms * 1e-3) * world, "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": res["clocks"],
+            "cpu_baseline": cpu,
+            "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

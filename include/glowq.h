@@ -1,0 +1,195 @@
+/*
+ * glowq.h -- C ABI of libglowq, the B200 (sm_100a) GlowQ corrected quantised
+ * linear layer.
+ *
+ * What it computes (GlowQ: Group-Shared Low-Rank Approximation for Quantized
+ * LLMs; papernotes.org summary, key design 4, and the experimental set-up
+ * paragraph): for an input-sharing group of m modules (Q/K/V, or gate/up) with
+ * INT4 g128 weights W_i^(q), per-module left factors A_i and one shared right
+ * factor B,
+ *
+ *     R   = X B^T                      (once per group, in the anchor step)
+ *     y_i = X deq(W_i^(q))^T + R A_i^T (every module of the group)
+ *
+ * and solo modules (o_proj, down_proj) compute y = X deq(W)^T + (X B^T) A^T
+ * with their own B, nothing shared.  GlowQ-S (same key design) enables the
+ * correction only on the top-k units ranked by g_ner(u) = ||E_u||_F^2 /
+ * ||W_u||_F^2, falling back to layer order when the signal is weak.
+ *
+ * Conventions (all calls):
+ *   - Matrices are row-major.  X is token-major: T x d.  Outputs are T x O.
+ *   - fp16 values travel as their IEEE binary16 bit patterns (uint16_t).
+ *   - Device pointers are caller-owned device memory; the library never
+ *     allocates or frees them.  Host pointers are marked "host".
+ *   - Every call that takes `stream` (a cudaStream_t, NULL = legacy default
+ *     stream) is asynchronous on that stream: it validates its arguments on
+ *     the host, enqueues kernels and returns.  Errors found on the host are
+ *     returned before anything is enqueued.  A launch failure returns
+ *     GLOWQ_ERR_CUDA.  Faults detected inside kernels (a bounded wait that ran
+ *     out) are recorded in a per-device status word read by
+ *     glowq_get_device_status().
+ *   - Alignment: every device pointer 16-byte aligned; d % 128 == 0;
+ *     out_features % 16 == 0; ldY % 8 == 0 and ldY >= out_features;
+ *     r % 8 == 0 with 0 <= r <= 256 (r == 0 disables the correction).
+ *   - No exception crosses this boundary.
+ */
+#ifndef GLOWQ_H
+#define GLOWQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GLOWQ_API __attribute__((visibility("default")))
+#else
+#define GLOWQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum glowq_status {
+    GLOWQ_OK = 0,
+    GLOWQ_ERR_ARG = 1,          /* null pointer, negative size, bad enum    */
+    GLOWQ_ERR_SHAPE = 2,        /* size constraint violated (d % 128, ...)  */
+    GLOWQ_ERR_ALIGN = 3,        /* pointer or leading dimension misaligned  */
+    GLOWQ_ERR_CUDA = 4,         /* CUDA runtime error while enqueueing      */
+    GLOWQ_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out       */
+    GLOWQ_ERR_UNSUPPORTED = 6   /* valid request outside this build's scope */
+} glowq_status;
+
+#define GLOWQ_GROUP_SIZE 128    /* INT4 quantisation group along d          */
+#define GLOWQ_MAX_RANK 256      /* largest correction rank r                */
+#define GLOWQ_MAX_MODULES 8     /* largest input-sharing group (m)          */
+
+/*
+ * One quantised module of a group.  Device pointers:
+ *   qweight  [O][d/8]  uint32: code k of row o is nibble (k % 8) of word k/8,
+ *                      lowest nibble first (codes 0..15)
+ *   scales   [O][d/128] fp16 bits (s)
+ *   zeros    [O][d/128] uint8   (z, 0..15)
+ *            dequantised weight w_hat[o][k] = fp16_RN((q - z) * s)
+ *   A        [O][r]    fp16 bits, left factor; NULL disables this module's
+ *                      correction (a GlowQ-S unit that is not restored)
+ *   Y        output, T rows of ldY fp16 elements; columns [0, O) written
+ */
+typedef struct glowq_module {
+    const uint32_t* qweight;
+    const uint16_t* scales;
+    const uint8_t* zeros;
+    const uint16_t* A;
+    int64_t out_features;
+    uint16_t* Y;
+    int64_t ldY;
+} glowq_module;
+
+/*
+ * INT4 g128 asymmetric round-to-nearest quantisation and packing (set-up
+ * paragraph: INT4 weights, group size 128).  Per row o and group j, in IEEE
+ * fp32 round-to-nearest-even without fused multiply-add:
+ *   mn = min(min w, 0), mx = max(max w, 0)
+ *   s  = fp16_RN((mx - mn) / 15)   (s == 0 -> 1.0, s == inf -> 65504)
+ *   z  = clamp(rint(-mn / s), 0, 15)
+ *   q  = clamp(rint(w / s) + z, 0, 15)      (NaN weights -> code 0)
+ * W: device, O x d fp32.  Outputs: qweight [O][d/8], scales [O][d/128],
+ * zeros [O][d/128] (device, caller-allocated).  group_size must be 128.
+ */
+GLOWQ_API glowq_status glowq_pack_int4(const float* W, int64_t O, int64_t d, int32_t group_size,
+                             uint32_t* qweight, uint16_t* scales, uint8_t* zeros,
+                             void* stream);
+
+/*
+ * Dequantise to fp16: W_deq[o][k] = fp16_RN((q - z) * s), one rounding of the
+ * exact product.  W_deq: device, O x d fp16 bits.  Used to check the packed
+ * format; the forward kernels dequantise in registers / shared memory and
+ * never materialise W_deq.
+ */
+GLOWQ_API glowq_status glowq_dequant_int4(const uint32_t* qweight, const uint16_t* scales,
+                                const uint8_t* zeros, int64_t O, int64_t d,
+                                int32_t group_size, uint16_t* W_deq, void* stream);
+
+/*
+ * Bytes of device scratch the forward calls need for T tokens at rank r
+ * (split-K partial sums of R = X B^T for small T, and the solo call's R).
+ * The caller allocates it once and may reuse it across calls on one stream.
+ */
+GLOWQ_API size_t glowq_workspace_bytes(int64_t T, int32_t r);
+
+/*
+ * Input-sharing group forward (key design 4): R = X B^T is computed once and
+ * written to R_out; then every module i computes
+ *   Y_i = X w_hat_i^T + R A_i^T   (A_i == NULL: Y_i = X w_hat_i^T)
+ * in one launch over the stacked rows of all modules.
+ *   mods       host array of m module descriptors (mods[0] is the anchor)
+ *   m          1..GLOWQ_MAX_MODULES
+ *   d          shared input dimension
+ *   B          device, r x d fp16 bits, shared right factor (NULL iff r == 0)
+ *   r          correction rank, 0..256, multiple of 8
+ *   X          device, T x d fp16 bits
+ *   T          tokens (>= 0; T == 0 is a no-op)
+ *   R_out      device, T x r fp16 bits (the cached projection; NULL iff r == 0)
+ *   workspace  device scratch of at least glowq_workspace_bytes(T, r) bytes
+ * Small T (<= 16) runs the weight-streaming decode kernels; larger T runs the
+ * tcgen05 tensor-core kernels.  Accumulation is fp32; R and Y are rounded to
+ * fp16 (round-to-nearest-even).
+ */
+GLOWQ_API glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d,
+                                 const uint16_t* B, int32_t r, const uint16_t* X,
+                                 int64_t T, uint16_t* R_out, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * Solo module forward (key design 4, o_proj / down_proj): its own
+ * R = X B^T is computed inline into the workspace and consumed at once;
+ * Y = X w_hat^T + R A^T.  A NULL mod->A or r == 0 gives plain W4A16.
+ * Arguments as for glowq_group_forward.
+ */
+GLOWQ_API glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16_t* B,
+                                int32_t r, const uint16_t* X, int64_t T, void* workspace,
+                                size_t workspace_bytes, void* stream);
+
+/*
+ * GlowQ-S selective restore (key design 4; about half of the units restored
+ * in the pages' efficiency results).  Host-only.
+ *   err_fro2[u] = ||E_u||_F^2, w_fro2[u] = ||W_u||_F^2  (host, n_units)
+ *   layer_idx[u], kind[u]   tie-break / fallback keys  (host, n_units)
+ *   k                       units to restore, 0..n_units
+ * Ranking: descending g_ner = err/w; exact ties by ascending (layer, kind,
+ * unit index).  Weak-signal fallback: if any score is NaN, or all scores lie
+ * within a relative spread of 1e-6 of the largest, the ranking is the plain
+ * layer order.  Outputs (host): restore_mask[u] = 1 for the first k units of
+ * the ranking, order[0..n_units) = the ranking (may be NULL).
+ * *used_fallback (may be NULL) is set to 1 when the layer order was used.
+ */
+GLOWQ_API glowq_status glowq_select_restore(const double* err_fro2, const double* w_fro2,
+                                  const int32_t* layer_idx, const int32_t* kind,
+                                  int32_t n_units, int32_t k, uint8_t* restore_mask,
+                                  int32_t* order, int32_t* used_fallback);
+
+/*
+ * Per-row squared norms for g_ner: row_norms[2*o] = ||W[o] - w_hat[o]||^2 and
+ * row_norms[2*o+1] = ||W[o]||^2 (fp64, deterministic), from a module's fp32
+ * weight and its packed form.  Summing the rows of every module of a unit
+ * gives err_fro2 and w_fro2 for glowq_select_restore.
+ *   W          device, O x d fp32
+ *   row_norms  device, 2*O doubles (caller-allocated)
+ */
+GLOWQ_API glowq_status glowq_error_norms(const float* W, const uint32_t* qweight,
+                               const uint16_t* scales, const uint8_t* zeros,
+                               int64_t O, int64_t d, double* row_norms, void* stream);
+
+/* Reads and clears this device's status word (GLOWQ_OK or GLOWQ_ERR_TIMEOUT);
+   synchronises `stream` first. */
+GLOWQ_API glowq_status glowq_get_device_status(void* stream);
+
+/* Static description of a status code. */
+GLOWQ_API const char* glowq_status_string(glowq_status s);
+
+/* Library version, "major.minor.patch". */
+GLOWQ_API const char* glowq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GLOWQ_H */

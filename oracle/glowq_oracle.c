@@ -237,9 +237,10 @@ int ora_module_forward(const uint32_t* q, const uint16_t* s, const uint8_t* z,
                        double* Y)
 {
     if (O < 0 || d < 0 || T < 0 || gs <= 0 || d % gs != 0) return -1;
-    uint16_t* wh = (uint16_t*)malloc((size_t)(d > 0 ? d : 1) * sizeof(uint16_t));
     double* whd = (double*)malloc((size_t)(d > 0 ? d : 1) * sizeof(double));
-    if (!wh || !whd) { free(wh); free(whd); return -2; }
+    double* xd = (double*)malloc((size_t)(T * d > 0 ? T * d : 1) * sizeof(double));
+    if (!whd || !xd) { free(whd); free(xd); return -2; }
+    for (int64_t i = 0; i < T * d; ++i) xd[i] = ora_f16_to_f64(X[i]);
     int64_t ng = d / gs;
     for (int64_t o = 0; o < O; ++o) {
         for (int64_t k = 0; k < d; ++k) {
@@ -251,15 +252,15 @@ int ora_module_forward(const uint32_t* q, const uint16_t* s, const uint8_t* z,
         for (int64_t t = 0; t < T; ++t) {
             double acc = 0.0;
             for (int64_t k = 0; k < d; ++k)
-                acc += ora_f16_to_f64(X[t * d + k]) * whd[k];
+                acc += xd[t * d + k] * whd[k];
             if (A && r > 0 && R)
                 for (int32_t j = 0; j < r; ++j)
                     acc += R[t * r + j] * ora_f16_to_f64(A[o * r + j]);
             Y[t * O + o] = acc;
         }
     }
-    free(wh);
     free(whd);
+    free(xd);
     return 0;
 }
 

@@ -1,0 +1,202 @@
+// api.cu -- the extern "C" boundary of libglowq: argument validation, path
+// dispatch (decode kernels for T <= 16, tcgen05 kernels above) and launches.
+// Argument meaning, layouts and error behaviour are documented in glowq.h.
+#include <cstdio>
+#include <cstring>
+
+#include "common.cuh"
+#include "internal.cuh"
+
+namespace glowq {
+
+__device__ unsigned int g_device_status = 0;
+
+unsigned int* device_status_ptr() {
+    static unsigned int* cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+    if (dev < 64 && cached[dev]) return cached[dev];
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    if (dev < 64) cached[dev] = static_cast<unsigned int*>(p);
+    return static_cast<unsigned int*>(p);
+}
+
+
+static inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int device_sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+
+static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+static size_t workspace_partial_bytes(int64_t T, int32_t r) {
+    if (r <= 0 || T <= 0 || T > kDecodeMaxTokens) return 0;
+    return align_up(decode_partial_bytes(T, r), 256);
+}
+
+static size_t workspace_solo_R_bytes(int64_t T, int32_t r) {
+    if (r <= 0 || T <= 0) return 0;
+    return align_up((size_t)T * (size_t)r * 2, 256);
+}
+
+// Shared validation for the forward calls.
+static glowq_status validate_forward(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
+                                     const uint16_t* X, int64_t T) {
+    if (!mods || m < 1 || m > GLOWQ_MAX_MODULES || d <= 0 || T < 0 || r < 0) return GLOWQ_ERR_ARG;
+    if (d % GLOWQ_GROUP_SIZE != 0 || d > (int64_t)1 << 20) return GLOWQ_ERR_SHAPE;
+    if (r > GLOWQ_MAX_RANK || r % 8 != 0) return GLOWQ_ERR_SHAPE;
+    if (r > 0 && !B) return GLOWQ_ERR_ARG;
+    if (T > 0 && !X) return GLOWQ_ERR_ARG;
+    if ((B && !aligned16(B)) || (X && !aligned16(X))) return GLOWQ_ERR_ALIGN;
+    int64_t rows = 0;
+    for (int i = 0; i < m; ++i) {
+        const glowq_module& md = mods[i];
+        if (!md.qweight || !md.scales || !md.zeros || !md.Y) return GLOWQ_ERR_ARG;
+        if (md.out_features <= 0 || md.out_features % 16 != 0) return GLOWQ_ERR_SHAPE;
+        if (md.ldY < md.out_features || md.ldY % 8 != 0) return GLOWQ_ERR_ALIGN;
+        if (!aligned16(md.qweight) || !aligned16(md.Y) || (md.A && !aligned16(md.A))) return GLOWQ_ERR_ALIGN;
+        if ((reinterpret_cast<uintptr_t>(md.scales) & 1u) != 0) return GLOWQ_ERR_ALIGN;
+        rows += md.out_features;
+    }
+    if (rows > ((int64_t)1 << 30) || T > ((int64_t)1 << 30)) return GLOWQ_ERR_SHAPE;
+    return GLOWQ_OK;
+}
+
+static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
+                                 const uint16_t* X, int64_t T, uint16_t* R, void* workspace, size_t ws_bytes,
+                                 cudaStream_t st) {
+    if (T == 0) return GLOWQ_OK;
+    ModuleView hm[GLOWQ_MAX_MODULES];
+    bool any_A = false;
+    for (int i = 0; i < m; ++i) {
+        hm[i] = {mods[i].qweight, mods[i].scales, mods[i].zeros, (r > 0) ? mods[i].A : nullptr,
+                 mods[i].Y, mods[i].ldY, mods[i].out_features};
+        any_A = any_A || hm[i].A != nullptr;
+    }
+    const bool use_r = r > 0;
+    if (T <= kDecodeMaxTokens) {
+        if (use_r) {
+            float* partial = reinterpret_cast<float*>(workspace);
+            cudaError_t e = launch_rproj_decode(X, B, (int)T, (int)d, r, partial, R, st);
+            if (e != cudaSuccess) return GLOWQ_ERR_CUDA;
+        }
+        cudaError_t e = launch_gemv_decode(hm, m, (int)d, (int)T, use_r ? r : 0, X, R, use_r, device_sm_count(), st);
+        return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
+    }
+    (void)any_A;
+    (void)ws_bytes;
+    return prefill_group_forward(hm, m, (int)d, use_r ? B : nullptr, use_r ? r : 0, X, T, R,
+                                 device_sm_count(), st);
+}
+
+}  // namespace glowq
+
+using namespace glowq;
+
+extern "C" {
+
+const char* glowq_version(void) { return "0.1.0"; }
+
+const char* glowq_status_string(glowq_status s) {
+    switch (s) {
+        case GLOWQ_OK: return "ok";
+        case GLOWQ_ERR_ARG: return "invalid argument (null pointer or negative size)";
+        case GLOWQ_ERR_SHAPE: return "unsupported shape (d % 128, out_features % 16, r % 8, r <= 256)";
+        case GLOWQ_ERR_ALIGN: return "misaligned pointer or leading dimension";
+        case GLOWQ_ERR_CUDA: return "CUDA error while enqueueing work";
+        case GLOWQ_ERR_TIMEOUT: return "a device-side bounded wait ran out";
+        case GLOWQ_ERR_UNSUPPORTED: return "request outside this build's scope";
+    }
+    return "unknown status";
+}
+
+glowq_status glowq_pack_int4(const float* W, int64_t O, int64_t d, int32_t group_size, uint32_t* qweight,
+                             uint16_t* scales, uint8_t* zeros, void* stream) {
+    if (O < 0 || d < 0) return GLOWQ_ERR_ARG;
+    if (group_size != GLOWQ_GROUP_SIZE) return GLOWQ_ERR_UNSUPPORTED;
+    if (d % GLOWQ_GROUP_SIZE != 0) return GLOWQ_ERR_SHAPE;
+    if (O == 0 || d == 0) return GLOWQ_OK;
+    if (!W || !qweight || !scales || !zeros) return GLOWQ_ERR_ARG;
+    if (!aligned16(W) || (reinterpret_cast<uintptr_t>(qweight) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 1u))
+        return GLOWQ_ERR_ALIGN;
+    return launch_pack_int4(W, O, d, qweight, scales, zeros, (cudaStream_t)stream) == cudaSuccess ? GLOWQ_OK
+                                                                                                : GLOWQ_ERR_CUDA;
+}
+
+glowq_status glowq_dequant_int4(const uint32_t* qweight, const uint16_t* scales, const uint8_t* zeros, int64_t O,
+                                int64_t d, int32_t group_size, uint16_t* W_deq, void* stream) {
+    if (O < 0 || d < 0) return GLOWQ_ERR_ARG;
+    if (group_size != GLOWQ_GROUP_SIZE) return GLOWQ_ERR_UNSUPPORTED;
+    if (d % GLOWQ_GROUP_SIZE != 0) return GLOWQ_ERR_SHAPE;
+    if (O == 0 || d == 0) return GLOWQ_OK;
+    if (!qweight || !scales || !zeros || !W_deq) return GLOWQ_ERR_ARG;
+    if (!aligned16(W_deq) || (reinterpret_cast<uintptr_t>(qweight) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 1u))
+        return GLOWQ_ERR_ALIGN;
+    return launch_dequant_int4(qweight, scales, zeros, O, d, W_deq, (cudaStream_t)stream) == cudaSuccess
+               ? GLOWQ_OK
+               : GLOWQ_ERR_CUDA;
+}
+
+glowq_status glowq_error_norms(const float* W, const uint32_t* qweight, const uint16_t* scales,
+                               const uint8_t* zeros, int64_t O, int64_t d, double* row_norms, void* stream) {
+    if (O < 0 || d < 0) return GLOWQ_ERR_ARG;
+    if (d % GLOWQ_GROUP_SIZE != 0) return GLOWQ_ERR_SHAPE;
+    if (O == 0 || d == 0) return GLOWQ_OK;
+    if (!W || !qweight || !scales || !zeros || !row_norms) return GLOWQ_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(row_norms) & 7u) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
+        (reinterpret_cast<uintptr_t>(qweight) & 3u) || (reinterpret_cast<uintptr_t>(W) & 3u))
+        return GLOWQ_ERR_ALIGN;
+    return launch_error_norms(W, qweight, scales, zeros, O, d, row_norms, (cudaStream_t)stream) == cudaSuccess
+               ? GLOWQ_OK
+               : GLOWQ_ERR_CUDA;
+}
+
+size_t glowq_workspace_bytes(int64_t T, int32_t r) {
+    if (T < 0 || r < 0) return 0;
+    return workspace_partial_bytes(T, r) + workspace_solo_R_bytes(T, r);
+}
+
+glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
+                                 const uint16_t* X, int64_t T, uint16_t* R_out, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    glowq_status v = validate_forward(mods, m, d, B, r, X, T);
+    if (v != GLOWQ_OK) return v;
+    if (T == 0) return GLOWQ_OK;
+    if (r > 0) {
+        if (!R_out) return GLOWQ_ERR_ARG;
+        if (!aligned16(R_out)) return GLOWQ_ERR_ALIGN;
+        const size_t need = workspace_partial_bytes(T, r);
+        if (need > 0 && (!workspace || workspace_bytes < need)) return GLOWQ_ERR_ARG;
+        if (workspace && !aligned16(workspace)) return GLOWQ_ERR_ALIGN;
+    }
+    return forward_impl(mods, m, d, B, r, X, T, R_out, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r, const uint16_t* X,
+                                int64_t T, void* workspace, size_t workspace_bytes, void* stream) {
+    glowq_status v = validate_forward(mod, 1, d, B, r, X, T);
+    if (v != GLOWQ_OK) return v;
+    if (T == 0) return GLOWQ_OK;
+    uint16_t* R = nullptr;
+    if (r > 0) {
+        const size_t need = glowq_workspace_bytes(T, r);
+        if (!workspace || workspace_bytes < need) return GLOWQ_ERR_ARG;
+        if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
+        R = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(workspace) + workspace_partial_bytes(T, r));
+    }
+    return forward_impl(mod, 1, d, B, r, X, T, R, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+glowq_status glowq_get_device_status(void* stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GLOWQ_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return GLOWQ_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero)) != cudaSuccess) return GLOWQ_ERR_CUDA;
+    return (glowq_status)v;
+}
+
+}  // extern "C"

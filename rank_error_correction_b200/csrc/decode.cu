@@ -1,0 +1,751 @@
+// decode.cu -- small-T (T <= 16) path of the GlowQ corrected linear layer.
+//
+// GlowQ pages, papernotes.org summary, key design 4: one shared projection
+// R = X B^T per input-sharing group, then y_i = W_i^(q) X + A_i R for every
+// module; solo modules compute their own R inline.
+//
+// At T <= 16 the layer is a weight-streaming GEMV: every INT4 weight byte is
+// read once from HBM and meets at most 16 tokens, so the kernels are HBM-bound.
+// Design:
+//   * rproj_partial / rproj_reduce: R = X B^T split along d over up to 32 CTAs
+//     (fp32 partial sums in the caller's workspace, reduced in a fixed order so
+//     the result is deterministic), rounded to fp16.
+//   * corrected_gemv: one launch over the stacked rows of all modules of the
+//     group.  128-bit streaming loads of the packed weights (4 groups of 128
+//     in flight per warp, issued before anything else); nibbles unpacked in
+//     registers to the exact fp16 integers (q - z) (half2 bias trick); the
+//     multiply-accumulate runs on the tensor cores with register operands
+//     (mma.sync m16n8k16, fp32 accumulate) so the ALU cost per weight stays
+//     below two instructions; the group scale s is applied in fp32 to each
+//     128-group's dot product.  The k order inside an MMA is permuted
+//     identically on both operands (a permutation of the contraction index
+//     leaves the dot product unchanged) so that packed words map straight onto
+//     fragments.  Activations and scales/zeros sit in shared memory; d is
+//     split across a thread-block cluster whose partial sums meet in
+//     distributed shared memory; the rank-r correction A_i R is one more short
+//     MMA slab on the same fp32 accumulators, after a programmatic-dependent-
+//     launch wait on the R kernels, so the weight stream overlaps the
+//     projection.
+//   * Numerics: the products (q - z) x are exact; each group's sum is scaled
+//     by s in fp32, i.e. the effective weight is the exact (q - z) s rather
+//     than its fp16 rounding (a difference of at most 2^-12 relative per
+//     weight, far inside the parity bar).
+#include <cstdio>
+#include <cstdlib>
+
+#include "common.cuh"
+#include "internal.cuh"
+
+namespace glowq {
+
+
+constexpr int kRprojMaxChunks = 32;
+
+// ---------------------------------------------------------------------------
+// R = X B^T, split along d.  Block: ceil(r/16) warps, warp w owns B rows
+// 16w .. 16w+15; block kc owns a slice of d in steps of 32.
+// partial[kc][t][j] (fp32).
+// ---------------------------------------------------------------------------
+template <int NT>
+__global__ void __launch_bounds__(512) rproj_partial_kernel(const __half* __restrict__ X,
+                                                             const __half* __restrict__ B, int T, int d,
+                                                             int r, int chunks, float* __restrict__ partial) {
+    pdl_wait();                 // X may come from the previous kernel in the stream
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int j0 = warp * 16 + g, j1 = j0 + 8;
+    const int kc = blockIdx.x;
+    const int nsteps = d / 32;
+    const int s0 = (int)((int64_t)kc * nsteps / chunks), s1 = (int)((int64_t)(kc + 1) * nsteps / chunks);
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+    const uint4 zero4 = make_uint4(0, 0, 0, 0);
+    for (int st = s0; st < s1; ++st) {
+        const int k = st * 32 + 8 * t;
+        const uint4 blo = (j0 < r) ? ldg_128(B + (int64_t)j0 * d + k) : zero4;
+        const uint4 bhi = (j1 < r) ? ldg_128(B + (int64_t)j1 * d + k) : zero4;
+        uint4 xv[NT];
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int tok = n * 8 + g;
+            xv[n] = (tok < T) ? ldg_128(X + (int64_t)tok * d + k) : zero4;
+        }
+        const uint32_t a0[4] = {blo.x, bhi.x, blo.y, bhi.y};
+        const uint32_t a1[4] = {blo.z, bhi.z, blo.w, bhi.w};
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const uint32_t b0[2] = {xv[n].x, xv[n].y};
+            const uint32_t b1[2] = {xv[n].z, xv[n].w};
+            mma_16816(acc[n], a0, b0);
+            mma_16816(acc[n], a1, b1);
+        }
+    }
+    float* out = partial + (int64_t)kc * T * r;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int tk = n * 8 + 2 * t;
+        if (j0 < r) {
+            if (tk < T) out[(int64_t)tk * r + j0] = acc[n][0];
+            if (tk + 1 < T) out[(int64_t)(tk + 1) * r + j0] = acc[n][1];
+        }
+        if (j1 < r) {
+            if (tk < T) out[(int64_t)tk * r + j1] = acc[n][2];
+            if (tk + 1 < T) out[(int64_t)(tk + 1) * r + j1] = acc[n][3];
+        }
+    }
+}
+
+// R[t][j] = fp16_RN(sum_kc partial[kc][t][j]) in ascending kc.
+__global__ void __launch_bounds__(256) rproj_reduce_kernel(const float* __restrict__ partial, int chunks,
+                                                            int T, int r, __half* __restrict__ R) {
+    pdl_launch_dependents();    // let the GEMV start streaming weights now
+    pdl_wait();                 // partial sums complete
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= T * r) return;
+    float acc = 0.f;
+    for (int kc = 0; kc < chunks; ++kc) acc += partial[(int64_t)kc * T * r + i];
+    R[i] = __float2half_rn(acc);
+}
+
+// ---------------------------------------------------------------------------
+// Corrected GEMV over the stacked rows of a group.
+//
+// Work shape (chosen on the host from the occupancy calculator so that every
+// CTA is resident in one wave with ~16-24 warps per SM):
+//   * a CTA holds `rt` row tiles of 16 rows x `kw` in-CTA splits of its slice
+//     of d (rt * kw warps; warp w owns tile w % rt and split w / rt);
+//   * optionally a thread-block cluster of `kc` CTAs splits d further (then
+//     kw == 1); partial sums meet in distributed shared memory.
+//
+// Arithmetic of one 128-group (row o, tokens t, codes q, zero z, scale s):
+//   sum_k (q_k - z) s x_k = s * (D - (64 + z) * S),
+//   D = sum_k (64 + q_k) x_k  (tensor cores, fp32 accumulate),  S = sum_k x_k.
+// 64 + q is built in one LOP3 per half2 by placing the nibble in mantissa bits
+// 4..7 of the fp16 constant 64.0 (no subtraction per weight); the products are
+// exact and the offset costs ~3 of fp32's 24 bits.  S is computed once per CTA.
+//
+// Shared memory (dynamic), in this order:
+//   ring [warps][kStages][128] uint4 packed-weight stream (cp.async, lane-private;
+//                                    a stage holds two 128-groups)
+//   xs   [T+1][wpt_max] uint4        the CTA's activation slice (row T all zero,
+//                                    read by the lanes of padding tokens); each
+//                                    8-element word stored as the half2 pairs
+//                                    (x0,x4) (x1,x5) (x2,x6) (x3,x7) of the MMA B
+//                                    fragment, word index XOR-swizzled
+//   xsum [ncta_max][8*NT] f32        per-group activation sums S (0 for padding)
+//   sz   [warps][16][nsub_max+1] f32x2  (s, 64 + z) of the warp's rows and groups
+//   red  [nslots][NT*4][32] f32      partial sums sent to the finalising warp
+//   as   [fin_slots][16][r+8] f16    A rows of the tiles this CTA finalises
+// ---------------------------------------------------------------------------
+constexpr int kMaxWarps = 8;
+constexpr int kStages = 4;     // pipeline stages per warp, 2 groups of 128 (2 KB) each
+
+struct GemvModule {
+    const uint32_t* q;
+    const __half* s;
+    const uint8_t* z;
+    const __half* A;   // nullptr: correction off for this module
+    __half* Y;
+    int64_t ldY;
+    int O;
+    int tile_begin;    // first 16-row tile of this module in the stacked order
+};
+
+struct GemvArgs {
+    GemvModule mod[GLOWQ_MAX_MODULES];
+    int m;
+    int d;
+    int T;
+    int r;
+    int num_tiles;
+    int rt;            // row tiles per CTA
+    int kw;            // in-CTA splits of d
+    int kc;            // CTAs per cluster splitting d (kw == 1 when kc > 1)
+    int wait_dep;      // launched behind the R kernels: griddepcontrol.wait before R
+    const __half* X;   // T x d
+    const __half* R;   // T x r (read after the wait)
+};
+
+struct GemvLayout {    // byte offsets into dynamic shared memory
+    int xs, xsum, sz, red, as, total;
+    int wpt_max, ncta_max, nsub_max, fin_slots;
+};
+
+__host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+__host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, int kw, int kc, int nt) {
+    GemvLayout L;
+    const int warps = rt * kw;
+    const int ngroups = d / 128;
+    L.ncta_max = ceil_div(ngroups, kc);
+    L.nsub_max = ceil_div(L.ncta_max, kw);
+    L.wpt_max = L.ncta_max * 16;
+    L.fin_slots = (kc > 1) ? ceil_div(rt, kc) : rt;
+    const int nslots = (kc > 1) ? kc * L.fin_slots : (kw > 1 ? kw * rt : 0);
+    int off = warps * kStages * 128 * 16;
+    L.xs = off;
+    off += (T + 1) * L.wpt_max * 16;
+    L.xsum = off;
+    off += L.ncta_max * 8 * nt * 4;
+    off = (off + 15) / 16 * 16;
+    L.sz = off;
+    off += warps * 16 * (L.nsub_max + 1) * 8;
+    L.red = off;
+    off += nslots * nt * 4 * 32 * 4;
+    L.as = off;
+    off += (r > 0) ? L.fin_slots * 16 * (r + 8) * 2 : 0;
+    L.total = (off + 15) / 16 * 16;
+    return L;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t smem_addr, const void* gptr) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr), "l"(gptr) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Issue one pipeline stage: groups Ga and Ga+1 (the second only if < G1) of
+// rows g (qlo) and g+8 (qhi) into ring slot `slot` of this lane.
+__device__ __forceinline__ void issue_stage(uint32_t ring_base, const uint32_t* qlo, const uint32_t* qhi, int Ga,
+                                            int G1, int slot) {
+    const uint32_t sb = ring_base + (uint32_t)(slot * 128 * 16);
+    cp_async16(sb, qlo + Ga * 16);
+    cp_async16(sb + 32 * 16, qhi + Ga * 16);
+    if (Ga + 1 < G1) {
+        cp_async16(sb + 64 * 16, qlo + (Ga + 1) * 16);
+        cp_async16(sb + 96 * 16, qhi + (Ga + 1) * 16);
+    }
+}
+
+// D = A * B with a zero accumulator (starts an independent chain)
+__device__ __forceinline__ void mma_16816_zc(float c[4], const uint32_t a[4], const uint32_t b[2]) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "f"(0.0f));
+}
+
+// One packed word (8 codes, low nibble first) -> four half2 holding the exact
+// values 64 + q of codes (0,4), (1,5), (2,6), (3,7): each nibble lands in
+// mantissa bits 4..7 of 64.0 (0x5400).
+__device__ __forceinline__ void unpack_offset64(uint32_t w, uint32_t out[4]) {
+    out[0] = ((w << 4) & 0x00F000F0u) | 0x54005400u;
+    out[1] = (w & 0x00F000F0u) | 0x54005400u;
+    out[2] = ((w >> 4) & 0x00F000F0u) | 0x54005400u;
+    out[3] = ((w >> 8) & 0x00F000F0u) | 0x54005400u;
+}
+
+template <int NT>
+__global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const __grid_constant__ GemvArgs args) {
+    pdl_launch_dependents();
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int rt = args.rt, kw = args.kw, kc = args.kc;
+    const int warps = rt * kw;
+    const int d = args.d, T = args.T, r = args.r;
+    const int ngroups = d / 128;
+    const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, NT);
+    uint4* ring = reinterpret_cast<uint4*>(smem);
+    uint4* xs = reinterpret_cast<uint4*>(smem + L.xs);
+    float* xsum = reinterpret_cast<float*>(smem + L.xsum);
+    float2* szs = reinterpret_cast<float2*>(smem + L.sz);
+    float* red = reinterpret_cast<float*>(smem + L.red);
+    __half* as = reinterpret_cast<__half*>(smem + L.as);
+
+    const int crank = blockIdx.x % kc;          // rank in the cluster (cluster dims (kc,1,1))
+    const int block = blockIdx.x / kc;
+    const int C0 = (int)((int64_t)crank * ngroups / kc), C1 = (int)((int64_t)(crank + 1) * ngroups / kc);
+    const int ncta = C1 - C0;
+    const int wpt = ncta * 16;                  // 8-element words per token in the CTA's slice
+    const int tl = warp % rt, ks = warp / rt;   // tile within the CTA, split index
+    const int G0 = C0 + (int)((int64_t)ks * ncta / kw);
+    const int G1 = C0 + (int)((int64_t)(ks + 1) * ncta / kw);
+    const int tile = block * rt + tl;
+    const bool active = tile < args.num_tiles;
+    int mi = 0;
+    for (int i = 1; i < args.m; ++i)
+        if (tile >= args.mod[i].tile_begin) mi = i;
+    const GemvModule& M = args.mod[mi];
+    const int tile_row = (tile - M.tile_begin) * 16;
+    const int row_lo = tile_row + g, row_hi = row_lo + 8;
+    // the warp that finalises this tile: split 0 of the owner CTA of the cluster
+    const int owner = (kc > 1) ? tl % kc : 0;
+    const int fslot = (kc > 1) ? tl / kc : tl;
+    const bool finaliser = ks == 0 && owner == crank;
+    const bool has_corr = r > 0 && M.A != nullptr;
+
+    // 1) start the weight stream: one commit group per stage (two 128-groups)
+    const int64_t wpr = d / 8;
+    const uint32_t* qlo = M.q + (int64_t)row_lo * wpr + 4 * t;
+    const uint32_t* qhi = M.q + (int64_t)row_hi * wpr + 4 * t;
+    uint4* my_ring = ring + warp * kStages * 128;
+    const uint32_t ring_base = (uint32_t)__cvta_generic_to_shared(my_ring) + (uint32_t)lane * 16u;
+    const int nsub = G1 - G0;
+    const int npairs = (nsub + 1) / 2;
+#pragma unroll
+    for (int i = 0; i < kStages; ++i) {
+        if (active && i < npairs) issue_stage(ring_base, qlo, qhi, G0 + 2 * i, G1, i);
+        cp_async_commit();
+    }
+    // 1b) the finalising warp prefetches its tile's rows of A
+    if (active && has_corr && finaliser) {
+        const uint32_t a_base = (uint32_t)__cvta_generic_to_shared(as + fslot * 16 * (r + 8));
+        const int cpr = r / 8;   // 16-byte chunks per row
+        for (int c = lane; c < 16 * cpr; c += 32) {
+            const int rr = c / cpr, cc = c - rr * cpr;
+            cp_async16(a_base + (uint32_t)((rr * (r + 8) + cc * 8) * 2), M.A + (int64_t)(tile_row + rr) * r + cc * 8);
+        }
+    }
+    cp_async_commit();
+
+    // 2) this warp's (s, 64 + z): rows of its tile x groups [G0, G1); loads in
+    //    batches of 16 per lane, all issued before any is used
+    const int sz_stride = L.nsub_max + 1;
+    float2* my_sz = szs + warp * 16 * sz_stride;
+    if (active) {
+        const int items = 16 * nsub;
+        for (int base = lane; base < items; base += 16 * 32) {
+            unsigned short sv[16];
+            unsigned char zv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int i = base + j * 32;
+                if (i < items) {
+                    const int rr = i / nsub, gg = i - rr * nsub;
+                    const int64_t o = (int64_t)(tile_row + rr) * ngroups + G0 + gg;
+                    sv[j] = __half_as_ushort(M.s[o]);
+                    zv[j] = M.z[o];
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int i = base + j * 32;
+                if (i < items) {
+                    const int rr = i / nsub, gg = i - rr * nsub;
+                    my_sz[rr * sz_stride + gg] = make_float2(__half2float(__ushort_as_half(sv[j])), 64.0f + (float)zv[j]);
+                }
+            }
+        }
+    }
+    // 3) the CTA's activation slice, paired and swizzled (all loads of a batch first)
+    const int stride = warps * 32;
+    {
+        const int items = T * wpt;
+        for (int base = threadIdx.x; base < items; base += 4 * stride) {
+            uint4 v[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = base + j * stride;
+                if (i < items) {
+                    const int tok = i / wpt, wd = i - tok * wpt;
+                    v[j] = ldg_128(args.X + (int64_t)tok * d + (int64_t)C0 * 128 + wd * 8);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int i = base + j * stride;
+                if (i < items) {
+                    const int tok = i / wpt, wd = i - tok * wpt;
+                    uint4 p;
+                    p.x = pair_lo(v[j].x, v[j].z);   // (x0,x4)
+                    p.y = pair_hi(v[j].x, v[j].z);   // (x1,x5)
+                    p.z = pair_lo(v[j].y, v[j].w);   // (x2,x6)
+                    p.w = pair_hi(v[j].y, v[j].w);   // (x3,x7)
+                    // swizzle: XOR the two low bits of the word with (bit 3, token parity)
+                    xs[tok * wpt + (wd ^ (((wd >> 3) & 1) | ((tok & 1) << 1)))] = p;
+                }
+            }
+        }
+        for (int i = threadIdx.x; i < wpt; i += stride) xs[T * wpt + i] = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+    // 4) per-group activation sums S (fixed summation order; 0 for padding tokens)
+    for (int i = threadIdx.x; i < ncta * 8 * NT; i += stride) {
+        const int gc = i / (8 * NT), tok = i - gc * (8 * NT);
+        float acc_s = 0.f;
+        if (tok < T) {
+            const uint4* src = xs + tok * wpt + gc * 16;
+#pragma unroll 4
+            for (int wd = 0; wd < 16; ++wd) {
+                const uint4 v = src[wd];
+                const float2 f0 = __half22float2(u32_as_h2(v.x)), f1 = __half22float2(u32_as_h2(v.y));
+                const float2 f2 = __half22float2(u32_as_h2(v.z)), f3 = __half22float2(u32_as_h2(v.w));
+                acc_s += ((f0.x + f0.y) + (f1.x + f1.y)) + ((f2.x + f2.y) + (f3.x + f3.y));
+            }
+        }
+        xsum[gc * 8 * NT + tok] = acc_s;
+    }
+    __syncthreads();
+
+    // 5) main loop: two independent MMA chains per 128-group on (64 + q) x,
+    //    then s * (D - (64 + z) S) in fp32
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+    if (active) {
+        const float2* sz_lo = my_sz + g * sz_stride;
+        const float2* sz_hi = sz_lo + 8 * sz_stride;
+        // lanes of padding tokens read the zero row, so every read is unconditional
+        const uint4* xrow[NT];
+        const int xsw = ((t >> 1) & 1) | ((g & 1) << 1);   // swizzle term of this lane
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int tok = (n * 8 + g < T) ? n * 8 + g : T;
+            xrow[n] = xs + tok * wpt + (G0 - C0) * 16;
+        }
+        const float* xsum_w = xsum + (G0 - C0) * 8 * NT + 2 * t;
+        const uint4* rd = my_ring + lane;
+        for (int p0 = 0; p0 < npairs; p0 += kStages) {
+#pragma unroll
+            for (int i = 0; i < kStages; ++i) {
+                const int p = p0 + i;
+                if (p < npairs) {
+                    cp_async_wait<kStages - 1>();     // the oldest stage has landed
+                    uint4 w4[2][2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        w4[h][0] = rd[i * 128 + h * 64];
+                        w4[h][1] = rd[i * 128 + h * 64 + 32];
+                    }
+                    if (p + kStages < npairs) issue_stage(ring_base, qlo, qhi, G0 + 2 * (p + kStages), G1, i);
+                    cp_async_commit();
+                    const bool two = 2 * p + 1 < nsub;    // warp-uniform
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        if (h == 1 && !two) break;
+                        const int gl = 2 * p + h;          // group within the warp's split
+                        const uint32_t wl[4] = {w4[h][0].x, w4[h][0].y, w4[h][0].z, w4[h][0].w};
+                        const uint32_t wh[4] = {w4[h][1].x, w4[h][1].y, w4[h][1].z, w4[h][1].w};
+                        float ta[NT][4], tb[NT][4];
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            uint32_t pl[4], ph[4];
+                            unpack_offset64(wl[w], pl);   // 64 + codes (i, i+4) of row g
+                            unpack_offset64(wh[w], ph);   // row g + 8
+                            const uint32_t a0[4] = {pl[0], ph[0], pl[1], ph[1]};
+                            const uint32_t a1[4] = {pl[2], ph[2], pl[3], ph[3]};
+#pragma unroll
+                            for (int n = 0; n < NT; ++n) {
+                                const uint4 x = xrow[n][gl * 16 + ((4 * t + w) ^ xsw)];
+                                const uint32_t b0[2] = {x.x, x.y};   // (x0,x4) (x1,x5)
+                                const uint32_t b1[2] = {x.z, x.w};   // (x2,x6) (x3,x7)
+                                if (w == 0) {
+                                    mma_16816_zc(ta[n], a0, b0);
+                                    mma_16816_zc(tb[n], a1, b1);
+                                } else {
+                                    mma_16816(ta[n], a0, b0);
+                                    mma_16816(tb[n], a1, b1);
+                                }
+                            }
+                        }
+                        const float2 zl = sz_lo[gl], zh = sz_hi[gl];   // (s, 64 + z)
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            const float2 sx = *reinterpret_cast<const float2*>(xsum_w + gl * 8 * NT + n * 8);
+                            acc[n][0] = fmaf(zl.x, fmaf(-zl.y, sx.x, ta[n][0] + tb[n][0]), acc[n][0]);
+                            acc[n][1] = fmaf(zl.x, fmaf(-zl.y, sx.y, ta[n][1] + tb[n][1]), acc[n][1]);
+                            acc[n][2] = fmaf(zh.x, fmaf(-zh.y, sx.x, ta[n][2] + tb[n][2]), acc[n][2]);
+                            acc[n][3] = fmaf(zh.x, fmaf(-zh.y, sx.y, ta[n][3] + tb[n][3]), acc[n][3]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncwarp();   // A rows copied by other lanes of this warp are visible
+
+    // 6) the R kernels have finished once this returns
+    if (args.wait_dep) pdl_wait();
+
+    // 7) split-d reduction in a fixed order, into the finalising warp
+    if (kc > 1) {
+        // cluster: partials of tile tl go to rank tl % kc, slot [crank][tl / kc]
+        const int idx0 = (crank * L.fin_slots + fslot) * NT * 4 * 32 + lane;
+        if (owner != crank) {
+            const uint32_t local = (uint32_t)__cvta_generic_to_shared(red);
+            uint32_t remote;
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(owner));
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(remote + (uint32_t)(idx0 + (n * 4 + i) * 32) * 4u),
+                                 "f"(acc[n][i])
+                                 : "memory");
+        } else {
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) red[idx0 + (n * 4 + i) * 32] = acc[n][i];
+        }
+        asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+        if (!finaliser) return;
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float v = 0.f;
+                for (int c = 0; c < kc; ++c) v += red[((c * L.fin_slots + fslot) * NT * 4 + n * 4 + i) * 32 + lane];
+                acc[n][i] = v;
+            }
+    } else if (kw > 1) {
+        // in-CTA: partials of tile tl from split ks at slot [ks][tl]
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) red[((ks * rt + tl) * NT * 4 + n * 4 + i) * 32 + lane] = acc[n][i];
+        __syncthreads();
+        if (!finaliser) return;
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float v = 0.f;
+                for (int k2 = 0; k2 < kw; ++k2) v += red[((k2 * rt + tl) * NT * 4 + n * 4 + i) * 32 + lane];
+                acc[n][i] = v;
+            }
+    }
+    if (!active) return;
+
+    // 8) rank-r correction A_i R^T, accumulated into the same fp32 registers
+    if (has_corr) {
+        const __half* a_lo = as + (fslot * 16 + g) * (r + 8);
+        const __half* a_hi = a_lo + 8 * (r + 8);
+        for (int kb = 0; kb < r; kb += 16) {
+            const int k = kb + 4 * t;
+            const bool kval = k < r;   // r % 8 == 0: 4-element chunks are all-or-nothing
+            uint2 al = make_uint2(0, 0), ah = make_uint2(0, 0);
+            if (kval) {
+                al = *reinterpret_cast<const uint2*>(a_lo + k);
+                ah = *reinterpret_cast<const uint2*>(a_hi + k);
+            }
+            const uint32_t a[4] = {al.x, ah.x, al.y, ah.y};
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int tok = n * 8 + g;
+                uint2 rv = make_uint2(0, 0);
+                if (kval && tok < T) rv = __ldg(reinterpret_cast<const uint2*>(args.R + (int64_t)tok * r + k));
+                const uint32_t b[2] = {rv.x, rv.y};
+                mma_16816(acc[n], a, b);
+            }
+        }
+    }
+
+    // 9) fp16 outputs (round to nearest even)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int tk = n * 8 + 2 * t;
+        if (tk < T) {
+            M.Y[(int64_t)tk * M.ldY + row_lo] = __float2half_rn(acc[n][0]);
+            M.Y[(int64_t)tk * M.ldY + row_hi] = __float2half_rn(acc[n][2]);
+        }
+        if (tk + 1 < T) {
+            M.Y[(int64_t)(tk + 1) * M.ldY + row_lo] = __float2half_rn(acc[n][1]);
+            M.Y[(int64_t)(tk + 1) * M.ldY + row_hi] = __float2half_rn(acc[n][3]);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Host-side launchers (called from api.cu after validation).
+// ---------------------------------------------------------------------------
+static int rproj_chunks(int d) {
+    const int nsteps = d / 32;
+    return nsteps < kRprojMaxChunks ? nsteps : kRprojMaxChunks;
+}
+
+size_t decode_partial_bytes(int64_t T, int r) {
+    return (size_t)kRprojMaxChunks * (size_t)T * (size_t)r * sizeof(float);
+}
+
+static cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                             void** args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+// R = X B^T into R (fp16), via fp32 partials in `partial`.
+cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, float* partial,
+                                uint16_t* R, cudaStream_t st) {
+    const int chunks = rproj_chunks(d);
+    const int warps = (r + 15) / 16;
+    const __half* Xh = reinterpret_cast<const __half*>(X);
+    const __half* Bh = reinterpret_cast<const __half*>(B);
+    void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&chunks, (void*)&partial};
+    const void* fn = (T <= 8) ? (const void*)rproj_partial_kernel<1> : (const void*)rproj_partial_kernel<2>;
+    cudaError_t e = launch_ex(fn, dim3(chunks), dim3(warps * 32), 0, st, true, a1);
+    if (e != cudaSuccess) return e;
+    __half* Rh = reinterpret_cast<__half*>(R);
+    const float* pc = partial;
+    void* a2[] = {(void*)&pc, (void*)&chunks, (void*)&T, (void*)&r, (void*)&Rh};
+    const int n = T * r;
+    return launch_ex((const void*)rproj_reduce_kernel, dim3((n + 255) / 256), dim3(256), 0, st, true, a2);
+}
+
+
+// Resident CTAs of one variant and shape (cached: the occupancy query is not free).
+static int resident_ctas(const void* fn, int warps, int kc, size_t smem, int num_sms) {
+    struct Entry { const void* fn; int warps, kc; size_t smem; int n; };
+    static Entry cache[256];
+    static int used = 0;
+    for (int i = 0; i < used; ++i)
+        if (cache[i].fn == fn && cache[i].warps == warps && cache[i].kc == kc && cache[i].smem == smem)
+            return cache[i].n;
+    int n = 0;
+    if (kc == 1) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, warps * 32, smem) == cudaSuccess)
+            n = per_sm * num_sms;
+    } else {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(kc);
+        cfg.blockDim = dim3(warps * 32);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kc;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int clusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&clusters, fn, &cfg) == cudaSuccess) n = clusters * kc;
+    }
+    (void)cudaGetLastError();
+    if (used < 256) cache[used++] = {fn, warps, kc, smem, n};
+    return n;
+}
+
+struct GemvShape { int rt, kw, kc; size_t smem; };
+
+// Pick (rt, kw, kc): all CTAs resident in one wave, as many warps streaming as
+// possible up to 24 per SM, then the fewest splits of d.  If nothing fits in
+// one wave, the shape with the fewest waves.
+static GemvShape choose_shape(const void* fn, int tiles, int d, int T, int r, int nt, int num_sms) {
+    struct Key { const void* fn; int tiles, d, T, r; GemvShape s; };
+    static Key memo[128];
+    static int used = 0;
+    for (int i = 0; i < used; ++i)
+        if (memo[i].fn == fn && memo[i].tiles == tiles && memo[i].d == d && memo[i].T == T && memo[i].r == r)
+            return memo[i].s;
+    const int ngroups = d / 128;
+    const long cap = (long)num_sms * 24;
+    GemvShape best = {0, 0, 0, 0};
+    double best_key[3] = {1e30, 1e30, 1e30};
+    for (int rt = 1; rt <= kMaxWarps; rt *= 2)
+        for (int kw = 1; rt * kw <= kMaxWarps; ++kw)
+            for (int kc = 1; kc <= 8; ++kc) {
+                if (kc > 1 && kw > 1) break;
+                if (kc > ngroups || ceil_div(ngroups, kc) < kw) continue;
+                const int warps = rt * kw;
+                const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, nt);
+                if (L.total > 220 * 1024) continue;
+                const int res = resident_ctas(fn, warps, kc, (size_t)L.total, num_sms);
+                if (res <= 0) continue;
+                const long ctas = (long)ceil_div(tiles, rt) * kc;
+                const double waves = (double)ctas / res;
+                double key[3];
+                if (waves <= 1.0) {
+                    key[0] = 0;
+                    key[1] = -(double)(ctas * warps < cap ? ctas * warps : cap);
+                    key[2] = kw * kc - 0.01 * rt;
+                } else {
+                    key[0] = waves;
+                    key[1] = 0;
+                    key[2] = kw * kc;
+                }
+                if (key[0] < best_key[0] || (key[0] == best_key[0] && (key[1] < best_key[1] ||
+                                                                       (key[1] == best_key[1] && key[2] < best_key[2])))) {
+                    best_key[0] = key[0];
+                    best_key[1] = key[1];
+                    best_key[2] = key[2];
+                    best = {rt, kw, kc, (size_t)L.total};
+                }
+            }
+    if (used < 128 && best.rt > 0) memo[used++] = {fn, tiles, d, T, r, best};
+    if (std::getenv("GLOWQ_VERBOSE"))
+        std::fprintf(stderr, "glowq decode shape: tiles=%d d=%d T=%d r=%d -> rt=%d kw=%d kc=%d smem=%zu ctas=%d\n",
+                     tiles, d, T, r, best.rt, best.kw, best.kc, best.smem,
+                     best.rt ? ceil_div(tiles, best.rt) * best.kc : 0);
+    return best;
+}
+
+cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
+                               const uint16_t* R, bool after_rproj, int num_sms, cudaStream_t st) {
+    GemvArgs a = {};
+    int tiles = 0;
+    for (int i = 0; i < m; ++i) {
+        a.mod[i].q = mods[i].q;
+        a.mod[i].s = reinterpret_cast<const __half*>(mods[i].s);
+        a.mod[i].z = mods[i].z;
+        a.mod[i].A = (r > 0) ? reinterpret_cast<const __half*>(mods[i].A) : nullptr;
+        a.mod[i].Y = reinterpret_cast<__half*>(mods[i].Y);
+        a.mod[i].ldY = mods[i].ldY;
+        a.mod[i].O = (int)mods[i].O;
+        a.mod[i].tile_begin = tiles;
+        tiles += (int)(mods[i].O / 16);
+    }
+    if (tiles == 0) return cudaSuccess;
+    const int nt = (T <= 8) ? 1 : 2;
+    const void* fn = (nt == 1) ? (const void*)corrected_gemv_kernel<1> : (const void*)corrected_gemv_kernel<2>;
+    static bool opted[2] = {false, false};
+    if (!opted[nt - 1]) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+        if (e != cudaSuccess) return e;
+        opted[nt - 1] = true;
+    }
+    const GemvShape sh = choose_shape(fn, tiles, d, T, r, nt, num_sms);
+    if (sh.rt == 0) return cudaErrorInvalidValue;
+    a.m = m;
+    a.d = d;
+    a.T = T;
+    a.r = r;
+    a.num_tiles = tiles;
+    a.rt = sh.rt;
+    a.kw = sh.kw;
+    a.kc = sh.kc;
+    a.wait_dep = after_rproj ? 1 : 0;
+    a.X = reinterpret_cast<const __half*>(X);
+    a.R = reinterpret_cast<const __half*>(R);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ceil_div(tiles, sh.rt) * sh.kc);
+    cfg.blockDim = dim3(sh.rt * sh.kw * 32);
+    cfg.dynamicSmemBytes = sh.smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = sh.kc;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+    if (after_rproj) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    void* args[] = {(void*)&a};
+    return cudaLaunchKernelExC(&cfg, fn, args);
+}
+
+}  // namespace glowq

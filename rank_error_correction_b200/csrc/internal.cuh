@@ -1,0 +1,45 @@
+// internal.cuh -- declarations shared by the translation units of libglowq.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "glowq.h"
+
+namespace glowq {
+
+// Host-side view of one module of a group (validated by api.cu).
+struct ModuleView {
+    const uint32_t* q;
+    const uint16_t* s;
+    const uint8_t* z;
+    const uint16_t* A;   // nullptr: correction off for this module
+    uint16_t* Y;
+    int64_t ldY;
+    int64_t O;
+};
+
+constexpr int kDecodeMaxTokens = 16;
+
+// Device address of this device's status word (bounded-wait timeouts).
+unsigned int* device_status_ptr();
+
+// decode.cu
+size_t decode_partial_bytes(int64_t T, int r);
+cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, float* partial,
+                                uint16_t* R, cudaStream_t st);
+cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
+                               const uint16_t* R, bool after_rproj, int num_sms, cudaStream_t st);
+// pack.cu
+cudaError_t launch_pack_int4(const float* W, int64_t O, int64_t d, uint32_t* q, uint16_t* s, uint8_t* z,
+                             cudaStream_t st);
+cudaError_t launch_dequant_int4(const uint32_t* q, const uint16_t* s, const uint8_t* z, int64_t O, int64_t d,
+                                uint16_t* out, cudaStream_t st);
+cudaError_t launch_error_norms(const float* W, const uint32_t* q, const uint16_t* s, const uint8_t* z,
+                               int64_t O, int64_t d, double* out_rows, cudaStream_t st);
+// prefill.cu
+glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r,
+                                   const uint16_t* X, int64_t T, uint16_t* R, int num_sms, cudaStream_t st);
+
+}  // namespace glowq

@@ -1,0 +1,257 @@
+"""Thin Python binding of libglowq (the C ABI declared in include/glowq.h).
+
+Argument marshalling only: every step of the corrected linear layer runs in
+the library's CUDA kernels.  PyTorch tensors provide device memory and the
+current CUDA stream; their data pointers are handed to the C entry points.
+There is no CPU fallback: if ``libglowq.so`` is missing or a call fails, an
+exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import dataclasses
+import os
+import re
+from typing import List, Optional, Sequence, Tuple
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libglowq.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "glowq.h")
+
+GROUP_SIZE = 128
+MAX_RANK = 256
+MAX_MODULES = 8
+
+STATUS = {0: "GLOWQ_OK", 1: "GLOWQ_ERR_ARG", 2: "GLOWQ_ERR_SHAPE", 3: "GLOWQ_ERR_ALIGN",
+          4: "GLOWQ_ERR_CUDA", 5: "GLOWQ_ERR_TIMEOUT", 6: "GLOWQ_ERR_UNSUPPORTED"}
+
+
+class GlowQError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({_status_string(code)})")
+
+
+class _Module(C.Structure):
+    _fields_ = [("qweight", C.c_void_p), ("scales", C.c_void_p), ("zeros", C.c_void_p),
+                ("A", C.c_void_p), ("out_features", C.c_int64), ("Y", C.c_void_p), ("ldY", C.c_int64)]
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libglowq.so (build it first with rank_error_correction_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libglowq.so not built at {LIB_PATH}; run "
+                               "`python -m rank_error_correction_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        p, i64, i32, st = C.c_void_p, C.c_int64, C.c_int32, C.c_int
+        L.glowq_pack_int4.argtypes = [p, i64, i64, i32, p, p, p, p]
+        L.glowq_dequant_int4.argtypes = [p, p, p, i64, i64, i32, p, p]
+        L.glowq_workspace_bytes.argtypes = [i64, i32]
+        L.glowq_workspace_bytes.restype = C.c_size_t
+        L.glowq_group_forward.argtypes = [C.POINTER(_Module), i32, i64, p, i32, p, i64, p, p, C.c_size_t, p]
+        L.glowq_solo_forward.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p, C.c_size_t, p]
+        L.glowq_select_restore.argtypes = [p, p, p, p, i32, i32, p, p, p]
+        L.glowq_error_norms.argtypes = [p, p, p, p, i64, i64, p, p]
+        L.glowq_get_device_status.argtypes = [p]
+        L.glowq_status_string.argtypes = [st]
+        L.glowq_status_string.restype = C.c_char_p
+        L.glowq_version.restype = C.c_char_p
+        for f in ("glowq_pack_int4", "glowq_dequant_int4", "glowq_group_forward", "glowq_solo_forward",
+                  "glowq_select_restore", "glowq_error_norms", "glowq_get_device_status"):
+            getattr(L, f).restype = st
+        _lib = L
+    return _lib
+
+
+def declared_symbols() -> List[str]:
+    """Entry points declared in include/glowq.h."""
+    txt = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"GLOWQ_API\s+[\w\s\*]+?\b(glowq_\w+)\s*\(", txt)))
+
+
+def _status_string(code: int) -> str:
+    try:
+        return lib().glowq_status_string(code).decode()
+    except Exception:  # pragma: no cover - only while reporting another error
+        return "?"
+
+
+def _check(code: int, what: str) -> None:
+    if code != 0:
+        raise GlowQError(code, what)
+
+
+def version() -> str:
+    return lib().glowq_version().decode()
+
+
+def _stream(stream=None):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libglowq operates on CUDA tensors only")
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+# ---------------------------------------------------------------- packing ----
+
+def pack_int4(W, stream=None):
+    """W (O x d fp32, CUDA) -> (qweight int32 [O, d/8], scales fp16 [O, d/128], zeros uint8 [O, d/128])."""
+    import torch
+    _require_cuda(W)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    O, d = W.shape
+    q = torch.empty((O, d // 8), dtype=torch.int32, device=W.device)
+    s = torch.empty((O, d // GROUP_SIZE), dtype=torch.float16, device=W.device)
+    z = torch.empty((O, d // GROUP_SIZE), dtype=torch.uint8, device=W.device)
+    _check(lib().glowq_pack_int4(_ptr(W), O, d, GROUP_SIZE, _ptr(q), _ptr(s), _ptr(z), _stream(stream)),
+           "glowq_pack_int4")
+    return q, s, z
+
+
+def dequant_int4(q, s, z, d: int, stream=None):
+    import torch
+    _require_cuda(q, s, z)
+    O = q.shape[0]
+    out = torch.empty((O, d), dtype=torch.float16, device=q.device)
+    _check(lib().glowq_dequant_int4(_ptr(q), _ptr(s), _ptr(z), O, d, GROUP_SIZE, _ptr(out), _stream(stream)),
+           "glowq_dequant_int4")
+    return out
+
+
+def error_norms(W, q, s, z, stream=None):
+    """Per-row (||W - w_hat||^2, ||W||^2) as a float64 CUDA tensor [O, 2]."""
+    import torch
+    _require_cuda(W, q, s, z)
+    O, d = W.shape
+    out = torch.empty((O, 2), dtype=torch.float64, device=W.device)
+    _check(lib().glowq_error_norms(_ptr(W), _ptr(q), _ptr(s), _ptr(z), O, d, _ptr(out), _stream(stream)),
+           "glowq_error_norms")
+    return out
+
+
+# ---------------------------------------------------------------- forward ----
+
+@dataclasses.dataclass
+class QModule:
+    """One INT4 g128 module: packed weight, scales, zeros and (optional) left factor A (O x r fp16)."""
+    qweight: "object"
+    scales: "object"
+    zeros: "object"
+    A: Optional["object"] = None
+
+    @property
+    def out_features(self) -> int:
+        return int(self.qweight.shape[0])
+
+    @property
+    def in_features(self) -> int:
+        return int(self.qweight.shape[1]) * 8
+
+
+def workspace_bytes(T: int, r: int) -> int:
+    return int(lib().glowq_workspace_bytes(T, r))
+
+
+def alloc_workspace(T: int, r: int, device="cuda"):
+    import torch
+    n = max(workspace_bytes(T, r), 16)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _module_structs(mods: Sequence[QModule], Ys, use_A: bool):
+    arr = (_Module * len(mods))()
+    for i, (m, Y) in enumerate(zip(mods, Ys)):
+        _require_cuda(m.qweight, m.scales, m.zeros, m.A)
+        arr[i].qweight = _ptr(m.qweight)
+        arr[i].scales = _ptr(m.scales)
+        arr[i].zeros = _ptr(m.zeros)
+        arr[i].A = _ptr(m.A) if use_A else None
+        arr[i].out_features = m.out_features
+        arr[i].Y = Y.data_ptr()
+        arr[i].ldY = Y.stride(0)
+    return arr
+
+
+def group_forward(mods: Sequence[QModule], B, X, Ys=None, R_out=None, workspace=None, stream=None):
+    """Input-sharing group: R = X B^T once, Y_i = X w_hat_i^T + R A_i^T.
+
+    B (r x d fp16) may be None (correction off for the whole group).  Ys are
+    optional preallocated outputs (T x ldY fp16 views, e.g. column slices of one
+    T x sum(O_i) buffer).  Returns (Ys, R).
+    """
+    import torch
+    _require_cuda(B, X)
+    T, d = X.shape
+    r = 0 if B is None else int(B.shape[0])
+    if Ys is None:
+        Ys = [torch.empty((T, m.out_features), dtype=torch.float16, device=X.device) for m in mods]
+    for Y in Ys:
+        if Y.stride(1) != 1:
+            raise ValueError("outputs must have unit column stride")
+    if r > 0 and R_out is None:
+        R_out = torch.empty((T, r), dtype=torch.float16, device=X.device)
+    if workspace is None and r > 0:
+        workspace = alloc_workspace(T, r, X.device)
+    arr = _module_structs(mods, Ys, r > 0)
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().glowq_group_forward(arr, len(mods), d, _ptr(B), r, _ptr(X), T, _ptr(R_out), _ptr(workspace),
+                                     ws_n, _stream(stream)), "glowq_group_forward")
+    return Ys, R_out
+
+
+def solo_forward(mod: QModule, B, X, Y=None, workspace=None, stream=None):
+    """Solo module: Y = X w_hat^T + (X B^T) A^T, R computed inline (nothing cached)."""
+    import torch
+    _require_cuda(B, X)
+    T, d = X.shape
+    r = 0 if B is None else int(B.shape[0])
+    if Y is None:
+        Y = torch.empty((T, mod.out_features), dtype=torch.float16, device=X.device)
+    if workspace is None and r > 0:
+        workspace = alloc_workspace(T, r, X.device)
+    arr = _module_structs([mod], [Y], r > 0)
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().glowq_solo_forward(arr, d, _ptr(B), r, _ptr(X), T, _ptr(workspace), ws_n, _stream(stream)),
+           "glowq_solo_forward")
+    return Y
+
+
+def device_status(stream=None) -> int:
+    """Reads and clears the device status word (0 = ok, 5 = a bounded wait ran out)."""
+    return int(lib().glowq_get_device_status(_stream(stream)))
+
+
+# ---------------------------------------------------------------- GlowQ-S ----
+
+def select_restore(err_fro2, w_fro2, layer_idx, kind, k: int) -> Tuple["object", "object", bool]:
+    """Host-only ranking by g_ner = err/w; returns (mask uint8[n], order int32[n], used_fallback)."""
+    import numpy as np
+    e = np.ascontiguousarray(err_fro2, dtype=np.float64)
+    w = np.ascontiguousarray(w_fro2, dtype=np.float64)
+    la = np.ascontiguousarray(layer_idx, dtype=np.int32)
+    ki = np.ascontiguousarray(kind, dtype=np.int32)
+    n = e.size
+    mask = np.zeros(n, np.uint8)
+    order = np.zeros(n, np.int32)
+    fb = C.c_int32(0)
+    p = lambda a: a.ctypes.data_as(C.c_void_p)
+    _check(lib().glowq_select_restore(p(e), p(w), p(la), p(ki), n, int(k), p(mask), p(order), C.byref(fb)),
+           "glowq_select_restore")
+    return mask, order, bool(fb.value)

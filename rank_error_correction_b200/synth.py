@@ -191,3 +191,30 @@ WORKLOADS: Dict[str, Workload] = {
          GroupSpec("down_proj", 13824, [5120], ALPHA_MLP, 64)], [1, 16, 64, 2048],
         layers=40, restore_fraction=0.5),
 }
+
+
+# ----------------------------------------------------------------------------
+# Device-side draws for the benchmark (same distributions, drawn on the GPU so
+# that hundreds of MB of weights need no host round trip).
+# ----------------------------------------------------------------------------
+
+def _torch_seed(seed: int, stream: int, sub: int) -> int:
+    return (int(seed) * 0x9E3779B1 + int(stream) * 0x85EBCA77 + int(sub) * 0xC2B2AE3D) & 0x7FFFFFFFFFFFFFFF
+
+
+def device_weights(O: int, d: int, seed: int, sub: int, device="cuda", std: float = 0.02):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(_torch_seed(seed, S_W, sub))
+    return torch.randn((O, d), generator=g, device=device, dtype=torch.float32) * std
+
+
+def device_factors(out_features: List[int], d: int, r: int, seed: int, sub: int, device="cuda",
+                   a_std: float = 0.005, b_std: float = 0.01):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(_torch_seed(seed, S_A, sub))
+    As = [(torch.randn((O, r), generator=g, device=device) * a_std).half() for O in out_features]
+    g.manual_seed(_torch_seed(seed, S_B, sub))
+    B = (torch.randn((r, d), generator=g, device=device) * b_std).half()
+    return As, B

@@ -1,0 +1,76 @@
+"""Shared builders for the GPU parity tests: seeded inputs, oracle-side packing
+and references, and the normwise comparison used as the parity bar."""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import numpy as np
+
+import oracle
+from rank_error_correction_b200 import synth
+
+# Normwise relative error bar for fp16 outputs with fp32 accumulation: the
+# output rounding alone contributes up to 2^-11 ~ 4.9e-4 per element; R's fp16
+# rounding enters only through the ~1-2% correction term.
+TOL = 2e-3
+
+
+@dataclasses.dataclass
+class HostModule:
+    W: np.ndarray            # fp32 O x d
+    q: np.ndarray
+    s: np.ndarray
+    z: np.ndarray
+    A: Optional[np.ndarray]  # fp16 O x r or None
+
+
+def make_modules(d: int, outs: List[int], seed: int, sub0: int = 0, outlier_cols: int = 0) -> List[HostModule]:
+    mods = []
+    for i, O in enumerate(outs):
+        W = synth.weights(O, d, seed=seed, stream_sub=sub0 + i, outlier_cols=outlier_cols)
+        q, s, z = oracle.quantize_int4(W)
+        mods.append(HostModule(W, q, s, z, None))
+    return mods
+
+
+def attach_random_factors(mods: List[HostModule], d: int, r: int, seed: int, sub: int = 0):
+    As, B = synth.random_factors([m.W.shape[0] for m in mods], d, r, seed=seed, sub=sub)
+    for m, A in zip(mods, As):
+        m.A = A
+    return B
+
+
+def attach_solved_factors(mods: List[HostModule], d: int, r: int, alpha: float, seed: int,
+                          basis=None, p: int = 16, q: int = 2):
+    """Whitened stacked solve (oracle) with the population covariance; returns B fp16."""
+    E = np.vstack([oracle.quant_error(m.W, m.q, m.s, m.z)[0] for m in mods])
+    basis = basis if basis is not None else synth.orthogonal_basis(d, seed=seed)
+    lam = synth.power_law_spectrum(d, alpha)
+    Sh, Shp = synth.covariance_half(basis, lam)
+    A, B, _ = oracle.group_solve(E, Sh, Shp, r, p=p, q=q,
+                                 Omega=synth.gaussian_test_matrix(d, r + p, seed=seed))
+    row = 0
+    for m in mods:
+        O = m.W.shape[0]
+        m.A = A[row:row + O].astype(np.float16)
+        row += O
+    return B.astype(np.float16)
+
+
+def normwise(y_gpu: np.ndarray, y_ref: np.ndarray) -> float:
+    den = np.linalg.norm(y_ref)
+    return float(np.linalg.norm(y_gpu.astype(np.float64) - y_ref) / (den if den > 0 else 1.0))
+
+
+def to_dev(mods: List[HostModule], device="cuda", with_A: bool = True):
+    import torch
+    from rank_error_correction_b200 import glowq
+    out = []
+    for m in mods:
+        out.append(glowq.QModule(
+            torch.from_numpy(m.q.view(np.int32)).to(device),
+            torch.from_numpy(m.s.view(np.float16)).to(device),
+            torch.from_numpy(m.z).to(device),
+            None if (m.A is None or not with_A) else torch.from_numpy(m.A).to(device)))
+    return out

@@ -1,0 +1,105 @@
+"""The C ABI library builds, loads and exports every entry point glowq.h declares.
+
+No GPU needed: only host-side calls run here (argument validation that returns
+before anything is enqueued, the workspace-size query, and the host-only
+GlowQ-S ranking, checked against the oracle).
+"""
+import ctypes as C
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from rank_error_correction_b200 import build, glowq
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return glowq.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    declared = glowq.declared_symbols()
+    assert len(declared) >= 10
+    out = subprocess.check_output(["nm", "-D", "--defined-only", glowq.LIB_PATH], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [s for s in declared if s not in exported]
+    assert not missing, missing
+    assert all(s.startswith("glowq_") for s in exported)   # nothing else leaks out
+    for s in declared:
+        getattr(L, s)
+
+
+def test_version_and_status_strings(L):
+    assert glowq.version().count(".") == 2
+    for code in range(7):
+        assert L.glowq_status_string(code)
+
+
+def test_workspace_bytes(L):
+    assert glowq.workspace_bytes(0, 64) == 0
+    assert glowq.workspace_bytes(16, 0) == 0
+    small = glowq.workspace_bytes(16, 64)
+    assert small >= 32 * 16 * 64 * 4 + 16 * 64 * 2       # split-d partials + solo R
+    big = glowq.workspace_bytes(2048, 64)
+    assert big >= 2048 * 64 * 2
+    assert small % 256 == 0 and big % 256 == 0
+
+
+def _mods(n, O=128, q=0x1000, Y=0x2000, ldY=128, A=0x3000):
+    arr = (glowq._Module * n)()
+    for i in range(n):
+        arr[i].qweight, arr[i].scales, arr[i].zeros = q, q + 0x100, q + 0x200
+        arr[i].A, arr[i].out_features, arr[i].Y, arr[i].ldY = A, O, Y, ldY
+    return arr
+
+
+def _gf(L, mods, m=1, d=256, B=0x4000, r=16, X=0x5000, T=4, R=0x6000, ws=0x7000, wsb=1 << 20):
+    return L.glowq_group_forward(mods, m, d, B, r, X, T, R, ws, wsb, None)
+
+
+def test_host_validation_errors(L):
+    # Each call is rejected on the host before any CUDA work (fake addresses).
+    assert _gf(L, _mods(1), d=200) == 2                 # d % 128
+    assert _gf(L, _mods(1), r=12) == 2                  # r % 8
+    assert _gf(L, _mods(1), r=512) == 2                 # r > 256
+    assert _gf(L, _mods(1, O=100)) == 2                 # out_features % 16
+    assert _gf(L, _mods(1), m=0) == 1
+    assert _gf(L, _mods(9), m=9) == 1                   # more than 8 modules
+    assert _gf(L, _mods(1), X=0x5001) == 3              # misaligned X
+    assert _gf(L, _mods(1, ldY=100)) == 3               # ldY < out_features
+    assert _gf(L, _mods(1, ldY=132)) == 3               # ldY % 8
+    assert _gf(L, _mods(1), B=None) == 1                # r > 0 needs B
+    assert _gf(L, _mods(1), R=None) == 1                # ... and R_out
+    assert _gf(L, _mods(1), wsb=16) == 1                # workspace too small
+    assert _gf(L, _mods(1), T=-1) == 1
+    assert _gf(L, _mods(1), T=0) == 0                   # empty batch: no-op
+    assert L.glowq_solo_forward(_mods(1), 256, 0x4000, 16, 0x5000, 4, None, 0, None) == 1
+    assert L.glowq_pack_int4(0x1000, 16, 256, 64, 0x2000, 0x3000, 0x4000, None) == 6
+    assert L.glowq_pack_int4(0x1000, 16, 200, 128, 0x2000, 0x3000, 0x4000, None) == 2
+    assert L.glowq_pack_int4(0x1000, 0, 256, 128, 0x2000, 0x3000, 0x4000, None) == 0
+    assert L.glowq_dequant_int4(0x1000, 0x2000, 0x3000, 16, 256, 128, 0x4008, None) == 3
+
+
+def test_select_restore_matches_oracle(L):
+    g = np.random.default_rng(0)
+    for trial in range(40):
+        n = int(g.integers(1, 60))
+        e = np.round(g.random(n) * 4, 1 if trial % 2 else 6)
+        w = np.round(g.random(n) * 4 + 0.1, 1 if trial % 2 else 6)
+        if trial % 7 == 3:
+            e = w * 0.25                                 # flat scores -> layer order
+        layer = g.integers(0, 12, n)
+        kind = g.integers(0, 4, n)
+        k = int(g.integers(0, n + 1))
+        m1, o1, f1 = glowq.select_restore(e, w, layer, kind, k)
+        m2, o2, _, f2 = oracle.select_restore(e, w, layer, kind, k)
+        assert f1 == f2
+        assert np.array_equal(o1, o2) and np.array_equal(m1, m2)
+
+
+def test_select_restore_rejects_bad_k(L):
+    with pytest.raises(glowq.GlowQError):
+        glowq.select_restore([1.0], [1.0], [0], [0], 2)
