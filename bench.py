@@ -247,6 +247,76 @@ def time_e2e(T, steps, device, reps, io):
     return ms, h2d, d2h, n
 
 
+# ------------------------------------------------------------------ prefill
+
+MLP_D, MLP_FFN = 4096, 11008
+
+
+def time_prefill(T, steps, warmup, device, n_rep=2, seed=0):
+    """LLaMA-2-7B MLP linears at T tokens: gate/up group + down_proj solo (tcgen05 path)."""
+    import torch
+    from rank_error_correction_b200 import glowq, synth
+    reps = []
+    for i in range(n_rep):
+        gu = []
+        for j in range(2):
+            W = synth.device_weights(MLP_FFN, MLP_D, seed, sub=5000 + 100 * i + j, device=device)
+            q, s, z = glowq.pack_int4(W)
+            del W
+            gu.append(glowq.QModule(q, s, z))
+        As, Bg = synth.device_factors([MLP_FFN] * 2, MLP_D, R_RANK, seed, sub=5000 + i, device=device)
+        for m, A in zip(gu, As):
+            m.A = A
+        W = synth.device_weights(MLP_D, MLP_FFN, seed, sub=6000 + i, device=device)
+        q, s, z = glowq.pack_int4(W)
+        del W
+        Ad, Bd = synth.device_factors([MLP_D], MLP_FFN, R_RANK, seed, sub=6000 + i, device=device)
+        reps.append((gu, Bg, glowq.QModule(q, s, z, Ad[0]), Bd))
+    torch.cuda.synchronize()
+    X = torch.from_numpy(synth.activations(T, MLP_D, synth.ALPHA_MLP, seed=seed)).to(device)
+    Xd = torch.from_numpy(synth.activations(T, MLP_FFN, synth.ALPHA_MLP, seed=seed, sub=1)).to(device)
+    Ygu = torch.empty((T, 2 * MLP_FFN), dtype=torch.float16, device=device)
+    views = [Ygu[:, :MLP_FFN], Ygu[:, MLP_FFN:]]
+    Yd = torch.empty((T, MLP_D), dtype=torch.float16, device=device)
+    R = torch.empty((T, R_RANK), dtype=torch.float16, device=device)
+    ws = glowq.alloc_workspace(T, R_RANK, device)
+    stream = torch.cuda.Stream(device=device)
+
+    def step(i):
+        gu, Bg, dn, Bd = reps[i % n_rep]
+        glowq.group_forward(gu, Bg, X, Ys=views, R_out=R, workspace=ws)
+        glowq.solo_forward(dn, Bd, Xd, Y=Yd, workspace=ws)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(warmup, 3)):
+            step(i)
+    stream.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            gu, Bg, dn, Bd = reps[i % n_rep]
+            evs[i][0].record()
+            glowq.group_forward(gu, Bg, X, Ys=views, R_out=R, workspace=ws)
+            evs[i][1].record()
+            glowq.solo_forward(dn, Bd, Xd, Y=Yd, workspace=ws)
+            evs[i][2].record()
+    g.replay()
+    stream.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record()
+        g.replay()
+        t1.record()
+    stream.synchronize()
+    total_ms = t0.elapsed_time(t1)
+    gu_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(steps))
+    dn_ms = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(steps))
+    del g
+    return dict(total_ms=total_ms, gu_ms=gu_ms, dn_ms=dn_ms)
+
+
 # ------------------------------------------------------------ oracle timing
 
 def oracle_sample(T=1, rows_per_module=512, seed=0):
@@ -312,6 +382,7 @@ def main():
     ap.add_argument("--replicas", type=int, default=8)
     ap.add_argument("--no-extra", action="store_true", help="skip the T=4/16 decode lines")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill line")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -365,6 +436,22 @@ def main():
                           "qkv_group_hbm_frac": b / (r2["qkv_ms"] * 1e-3) / 1e9 / hbm_peak})
             del r2
 
+    prefill = None
+    if not args.no_prefill:
+        Tp, sp = 2048, min(args.steps, 20)
+        pr = time_prefill(Tp, sp, args.warmup, device)
+        tf_gu = group_flops([MLP_FFN] * 2, MLP_D, R_RANK, Tp) / (pr["gu_ms"] * 1e-3) / 1e12
+        tf_dn = group_flops([MLP_D], MLP_FFN, R_RANK, Tp) / (pr["dn_ms"] * 1e-3) / 1e12
+        prefill = {"workload": "LLaMA-2-7B MLP linears, prefill T=2048: gate/up group (2x11008x4096) + "
+                               "down_proj solo (4096x11008), INT4 g128, r=64",
+                   "tokens": Tp, "steps": sp, "tok_s": world * Tp * sp / (pr["total_ms"] / 1e3),
+                   "ms_per_step": pr["total_ms"] / sp,
+                   "gate_up_us": pr["gu_ms"] * 1e3, "down_us": pr["dn_ms"] * 1e3,
+                   "roofline": {"bound": "tensor", "kernel": "glowq_group_forward (gate/up, T=2048)",
+                                "achieved": tf_gu, "peak": tf_peak, "peak_source": peak_src, "unit": "TFLOP/s",
+                                "frac": tf_gu / tf_peak, "down_proj_TFLOPs": tf_dn,
+                                "algorithmic_flops": group_flops([MLP_FFN] * 2, MLP_D, R_RANK, Tp)}}
+
     cpu = None
     if rank == 0 and not args.no_cpu:
         times, frac = [], None
@@ -406,6 +493,7 @@ def main():
             "clocks": res["clocks"],
             "cpu_baseline": cpu,
             "extra": extra,
+            "prefill": prefill,
         }
         print(json.dumps(line), flush=True)
     if pg is not None:
