@@ -150,6 +150,35 @@ GLOWQ_API glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, co
                                 size_t workspace_bytes, void* stream);
 
 /*
+ * Solo module forward that allocates nothing (the GlowQ pages have no
+ * counterpart: this is a deployment convenience of this library).
+ *
+ * Same computation and arguments as glowq_solo_forward, minus the workspace:
+ * the scratch it needs (R and, for T <= 16, its split-d partial sums) lives
+ * in a fixed array compiled into the library, glowq_noalloc_scratch_bytes()
+ * (1 MiB) on every device that loads the library, held until process exit.
+ * It is meant for callers that cannot allocate device memory when they call
+ * -- e.g. a custom op or plugin running inside another runtime's enqueue step,
+ * where that runtime owns every device allocation.  The call itself performs
+ * no cudaMalloc/cudaFree and no other allocation of device memory.
+ *   - Sizes whose scratch need, glowq_workspace_bytes(T, r), exceeds
+ *     glowq_noalloc_scratch_bytes() are rejected with GLOWQ_ERR_SHAPE before
+ *     anything is enqueued (at r = 64 that is T > 8192).
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - All calls on a device share the one array: calls that may overlap on the
+ *     GPU (different streams without ordering between them) race on it.  The
+ *     array keeps the last call's contents; every value a call reads there is
+ *     written earlier by the same call, so nothing needs clearing.
+ */
+GLOWQ_API glowq_status glowq_solo_forward_noalloc(const glowq_module* mod, int64_t d, const uint16_t* B,
+                                                  int32_t r, const uint16_t* X, int64_t T, void* stream);
+
+/* Size of the fixed scratch array used by glowq_solo_forward_noalloc. */
+GLOWQ_API size_t glowq_noalloc_scratch_bytes(void);
+
+/*
  * GlowQ-S selective restore (key design 4; about half of the units restored
  * in the pages' efficiency results).  Host-only.
  *   err_fro2[u] = ||E_u||_F^2, w_fro2[u] = ||W_u||_F^2  (host, n_units)

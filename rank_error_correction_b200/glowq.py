@@ -55,6 +55,8 @@ def lib() -> C.CDLL:
         L.glowq_workspace_bytes.restype = C.c_size_t
         L.glowq_group_forward.argtypes = [C.POINTER(_Module), i32, i64, p, i32, p, i64, p, p, C.c_size_t, p]
         L.glowq_solo_forward.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p, C.c_size_t, p]
+        L.glowq_solo_forward_noalloc.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p]
+        L.glowq_noalloc_scratch_bytes.restype = C.c_size_t
         L.glowq_select_restore.argtypes = [p, p, p, p, i32, i32, p, p, p]
         L.glowq_error_norms.argtypes = [p, p, p, p, i64, i64, p, p]
         L.glowq_get_device_status.argtypes = [p]
@@ -62,6 +64,7 @@ def lib() -> C.CDLL:
         L.glowq_status_string.restype = C.c_char_p
         L.glowq_version.restype = C.c_char_p
         for f in ("glowq_pack_int4", "glowq_dequant_int4", "glowq_group_forward", "glowq_solo_forward",
+                  "glowq_solo_forward_noalloc",
                   "glowq_select_restore", "glowq_error_norms", "glowq_get_device_status"):
             getattr(L, f).restype = st
         _lib = L
@@ -231,6 +234,27 @@ def solo_forward(mod: QModule, B, X, Y=None, workspace=None, stream=None):
     _check(lib().glowq_solo_forward(arr, d, _ptr(B), r, _ptr(X), T, _ptr(workspace), ws_n, _stream(stream)),
            "glowq_solo_forward")
     return Y
+
+
+def solo_forward_noalloc(mod: QModule, B, X, Y=None, stream=None):
+    """Solo module forward with no workspace argument: the library's fixed
+    scratch array is used, so the call allocates no device memory.  For callers
+    that cannot allocate at call time (e.g. inside another runtime's enqueue).
+    Only the output Y is allocated here when not given."""
+    import torch
+    _require_cuda(B, X)
+    T, d = X.shape
+    r = 0 if B is None else int(B.shape[0])
+    if Y is None:
+        Y = torch.empty((T, mod.out_features), dtype=torch.float16, device=X.device)
+    arr = _module_structs([mod], [Y], r > 0)
+    _check(lib().glowq_solo_forward_noalloc(arr, d, _ptr(B), r, _ptr(X), T, _stream(stream)),
+           "glowq_solo_forward_noalloc")
+    return Y
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(lib().glowq_noalloc_scratch_bytes())
 
 
 def device_status(stream=None) -> int:
