@@ -166,8 +166,13 @@ def run_step(rep, io, stream=None):
 
 
 def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
-    """Graph-replayed timing of `steps` steps; also per-group-call event timing."""
+    """Time exactly `steps` decode steps replayed from one CUDA graph (value),
+    then replay an instrumented copy with event nodes around each call to get
+    the per-call durations used for the roofline (event nodes break the
+    programmatic-dependent-launch overlap between calls, so they are kept out
+    of the timed graph)."""
     import torch
+    from rank_error_correction_b200 import glowq
     reps = build_replicas(n_rep, T, device)
     io = make_io(T, device)
     stream = torch.cuda.Stream(device=device)
@@ -176,21 +181,11 @@ def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
         for i in range(max(warmup, 3)):
             run_step(reps[i % n_rep], io)
     stream.synchronize()
-    # one graph holding all timed steps, with event-record nodes around each group call
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    # timed graph: all steps back to back
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
         for i in range(steps):
-            rep = reps[i % n_rep]
-            evs[i][0].record()
-            mods, B = rep["qkv"]
-            from rank_error_correction_b200 import glowq
-            glowq.group_forward(mods, B, io["X"], Ys=io["views"], R_out=io["R"], workspace=io["ws"])
-            evs[i][1].record()
-            mo, Bo = rep["o_proj"]
-            glowq.solo_forward(mo[0], Bo, io["X2"], Y=io["Yo"], workspace=io["ws"])
-            evs[i][2].record()
-    # warm the graph once (untimed), then time one replay of exactly `steps` steps
+            run_step(reps[i % n_rep], io)
     g.replay()
     stream.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
@@ -207,9 +202,28 @@ def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
     if sampler:
         sampler.__exit__()
     total_ms = t0.elapsed_time(t1)
+    del g
+    # instrumented graph: event-record nodes around each call
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    gi = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gi, stream=stream):
+        for i in range(steps):
+            rep = reps[i % n_rep]
+            mods, B = rep["qkv"]
+            evs[i][0].record()
+            glowq.group_forward(mods, B, io["X"], Ys=io["views"], R_out=io["R"], workspace=io["ws"])
+            evs[i][1].record()
+            mo, Bo = rep["o_proj"]
+            glowq.solo_forward(mo[0], Bo, io["X2"], Y=io["Yo"], workspace=io["ws"])
+            evs[i][2].record()
+    gi.replay()
+    stream.synchronize()
+    with torch.cuda.stream(stream):
+        gi.replay()
+    stream.synchronize()
     qkv_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(steps)]
     o_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(steps)]
-    del g
+    del gi
     return dict(total_ms=total_ms, qkv_ms=statistics.mean(qkv_ms), o_ms=statistics.mean(o_ms),
                 qkv_ms_median=statistics.median(qkv_ms), clocks=sampler.summary() if sampler else None,
                 reps=reps, io=io)
@@ -480,7 +494,9 @@ def main():
                                    "o_proj solo (4096x4096), INT4 g128 asym, r=64 fp16 factors",
                        "tokens": T, "replicas": args.replicas,
                        "l2": f"inputs larger than L2: {args.replicas} weight replicas rotated "
-                             f"({args.replicas * 38.4:.0f} MB)", "graph": "one CUDA graph of all timed steps",
+                             f"({args.replicas * 38.4:.0f} MB)",
+                       "graph": "one CUDA graph of all timed steps (per-call roofline times from a second, "
+                                "event-instrumented replay)",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "roofline": {"bound": "hbm", "kernel": "glowq_group_forward (Q/K/V, T=1)", "achieved": achieved,
                          "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s", "frac": achieved / hbm_peak,

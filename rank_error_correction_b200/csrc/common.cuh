@@ -83,6 +83,13 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void* src, uin
         ::"r"(dst_smem), "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// 2-D tiled TMA load (tensor map in parameter/constant space) completing on an mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, uint64_t* bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
 // Order this thread's earlier generic-proxy shared-memory accesses before
 // later async-proxy (bulk copy) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {

@@ -50,8 +50,8 @@ template <int NT>
 __global__ void __launch_bounds__(512) rproj_partial_kernel(const __half* __restrict__ X,
                                                              const __half* __restrict__ B, int T, int d,
                                                              int r, int chunks, float* __restrict__ partial) {
+    pdl_launch_dependents();    // the next kernels may start their own prologues
     pdl_wait();                 // X may come from the previous kernel in the stream
-    pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int j0 = warp * 16 + g, j1 = j0 + 8;
@@ -129,8 +129,9 @@ __global__ void __launch_bounds__(256) rproj_reduce_kernel(const float* __restri
 // exact and the offset costs ~3 of fp32's 24 bits.  S is computed once per CTA.
 //
 // Shared memory (dynamic), in this order:
-//   ring [warps][kStages][128] uint4 packed-weight stream (cp.async, lane-private;
-//                                    a stage holds two 128-groups)
+//   ring [warps][S][16][32] u32      packed-weight stream: a stage is one 2-D TMA
+//                                    box of the warp's 16 rows x 2 groups (2 KB)
+//   bars [warps][S] u64              mbarriers of the weight stream
 //   xs   [T+1][wpt_max] uint4        the CTA's activation slice (row T all zero,
 //                                    read by the lanes of padding tokens); each
 //                                    8-element word stored as the half2 pairs
@@ -142,7 +143,9 @@ __global__ void __launch_bounds__(256) rproj_reduce_kernel(const float* __restri
 //   as   [fin_slots][16][r+8] f16    A rows of the tiles this CTA finalises
 // ---------------------------------------------------------------------------
 constexpr int kMaxWarps = 8;
-constexpr int kStages = 4;     // pipeline stages per warp, 2 groups of 128 (2 KB) each
+// Pipeline stages per warp (one 2-D TMA box of 16 rows x 2 groups of 128,
+// 2 KB) are a template parameter S in {4, 8}: the host trades ring depth
+// against resident warps.
 
 struct GemvModule {
     const uint32_t* q;
@@ -156,6 +159,7 @@ struct GemvModule {
 };
 
 struct GemvArgs {
+    CUtensorMap tmq[GLOWQ_MAX_MODULES];   // qweight [O][d/8] u32, box {32 words, 16 rows}
     GemvModule mod[GLOWQ_MAX_MODULES];
     int m;
     int d;
@@ -165,9 +169,9 @@ struct GemvArgs {
     int rt;            // row tiles per CTA
     int kw;            // in-CTA splits of d
     int kc;            // CTAs per cluster splitting d (kw == 1 when kc > 1)
-    int wait_dep;      // launched behind the R kernels: griddepcontrol.wait before R
     const __half* X;   // T x d
     const __half* R;   // T x r (read after the wait)
+    unsigned int* status;   // device status word (bounded-wait timeouts)
 };
 
 struct GemvLayout {    // byte offsets into dynamic shared memory
@@ -175,9 +179,15 @@ struct GemvLayout {    // byte offsets into dynamic shared memory
     int wpt_max, ncta_max, nsub_max, fin_slots;
 };
 
+// Launch-time constants computed on the host (no divisions in the kernel).
+struct GemvPlan {
+    GemvLayout L;
+    int gsplit[9];     // group boundaries of split j = crank * kw + ks, j in [0, kc * kw]
+};
+
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-__host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, int kw, int kc, int nt) {
+__host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, int kw, int kc, int nt, int stages) {
     GemvLayout L;
     const int warps = rt * kw;
     const int ngroups = d / 128;
@@ -186,7 +196,9 @@ __host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, i
     L.wpt_max = L.ncta_max * 16;
     L.fin_slots = (kc > 1) ? ceil_div(rt, kc) : rt;
     const int nslots = (kc > 1) ? kc * L.fin_slots : (kw > 1 ? kw * rt : 0);
-    int off = warps * kStages * 128 * 16;
+    int off = warps * stages * 2048;          // TMA ring (offset 0, 1024-aligned base)
+    off += warps * stages * 8;                // mbarriers
+    off = (off + 15) / 16 * 16;
     L.xs = off;
     off += (T + 1) * L.wpt_max * 16;
     L.xsum = off;
@@ -209,19 +221,6 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-// Issue one pipeline stage: groups Ga and Ga+1 (the second only if < G1) of
-// rows g (qlo) and g+8 (qhi) into ring slot `slot` of this lane.
-__device__ __forceinline__ void issue_stage(uint32_t ring_base, const uint32_t* qlo, const uint32_t* qhi, int Ga,
-                                            int G1, int slot) {
-    const uint32_t sb = ring_base + (uint32_t)(slot * 128 * 16);
-    cp_async16(sb, qlo + Ga * 16);
-    cp_async16(sb + 32 * 16, qhi + Ga * 16);
-    if (Ga + 1 < G1) {
-        cp_async16(sb + 64 * 16, qlo + (Ga + 1) * 16);
-        cp_async16(sb + 96 * 16, qhi + (Ga + 1) * 16);
-    }
-}
-
 // D = A * B with a zero accumulator (starts an independent chain)
 __device__ __forceinline__ void mma_16816_zc(float c[4], const uint32_t a[4], const uint32_t b[2]) {
     asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
@@ -240,18 +239,20 @@ __device__ __forceinline__ void unpack_offset64(uint32_t w, uint32_t out[4]) {
     out[3] = ((w >> 8) & 0x00F000F0u) | 0x54005400u;
 }
 
-template <int NT>
-__global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const __grid_constant__ GemvArgs args) {
+template <int NT, int S>
+__global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const __grid_constant__ GemvArgs args,
+                                                                           const __grid_constant__ GemvPlan plan) {
     pdl_launch_dependents();
-    extern __shared__ __align__(16) unsigned char smem[];
+    extern __shared__ __align__(1024) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int rt = args.rt, kw = args.kw, kc = args.kc;
     const int warps = rt * kw;
     const int d = args.d, T = args.T, r = args.r;
     const int ngroups = d / 128;
-    const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, NT);
-    uint4* ring = reinterpret_cast<uint4*>(smem);
+    const GemvLayout& L = plan.L;
+    unsigned char* ring = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + warps * S * 2048);
     uint4* xs = reinterpret_cast<uint4*>(smem + L.xs);
     float* xsum = reinterpret_cast<float*>(smem + L.xsum);
     float2* szs = reinterpret_cast<float2*>(smem + L.sz);
@@ -260,12 +261,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
 
     const int crank = blockIdx.x % kc;          // rank in the cluster (cluster dims (kc,1,1))
     const int block = blockIdx.x / kc;
-    const int C0 = (int)((int64_t)crank * ngroups / kc), C1 = (int)((int64_t)(crank + 1) * ngroups / kc);
+    const int C0 = plan.gsplit[crank * kw], C1 = plan.gsplit[crank * kw + kw];
     const int ncta = C1 - C0;
     const int wpt = ncta * 16;                  // 8-element words per token in the CTA's slice
     const int tl = warp % rt, ks = warp / rt;   // tile within the CTA, split index
-    const int G0 = C0 + (int)((int64_t)ks * ncta / kw);
-    const int G1 = C0 + (int)((int64_t)(ks + 1) * ncta / kw);
+    const int G0 = plan.gsplit[crank * kw + ks];
+    const int G1 = plan.gsplit[crank * kw + ks + 1];
     const int tile = block * rt + tl;
     const bool active = tile < args.num_tiles;
     int mi = 0;
@@ -280,18 +281,25 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
     const bool finaliser = ks == 0 && owner == crank;
     const bool has_corr = r > 0 && M.A != nullptr;
 
-    // 1) start the weight stream: one commit group per stage (two 128-groups)
-    const int64_t wpr = d / 8;
-    const uint32_t* qlo = M.q + (int64_t)row_lo * wpr + 4 * t;
-    const uint32_t* qhi = M.q + (int64_t)row_hi * wpr + 4 * t;
-    uint4* my_ring = ring + warp * kStages * 128;
-    const uint32_t ring_base = (uint32_t)__cvta_generic_to_shared(my_ring) + (uint32_t)lane * 16u;
+    // 1) start the weight stream: per warp, S mbarriers; lane 0 issues one 2-D
+    //    TMA box (16 rows x 2 groups) per stage
+    constexpr int kStages = S;
+    uint64_t* my_bars = bars + warp * kStages;
+    unsigned char* my_ring = ring + warp * kStages * 2048;
+    const uint32_t ring_smem = smem_u32(my_ring);
+    const CUtensorMap* tmq = &args.tmq[mi];
     const int nsub = G1 - G0;
     const int npairs = (nsub + 1) / 2;
-#pragma unroll
-    for (int i = 0; i < kStages; ++i) {
-        if (active && i < npairs) issue_stage(ring_base, qlo, qhi, G0 + 2 * i, G1, i);
-        cp_async_commit();
+    if (active) {
+        if (lane == 0) {
+            for (int i = 0; i < kStages; ++i) mbar_init(my_bars + i, 1);
+            fence_mbar_init();
+            for (int i = 0; i < kStages && i < npairs; ++i) {
+                mbar_arrive_expect_tx(my_bars + i, 2048u);
+                tma_load_2d(ring_smem + i * 2048, tmq, my_bars + i, (G0 + 2 * i) * 16, tile_row);
+            }
+        }
+        __syncwarp();
     }
     // 1b) the finalising warp prefetches its tile's rows of A
     if (active && has_corr && finaliser) {
@@ -309,30 +317,32 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
     const int sz_stride = L.nsub_max + 1;
     float2* my_sz = szs + warp * 16 * sz_stride;
     if (active) {
-        const int items = 16 * nsub;
-        for (int base = lane; base < items; base += 16 * 32) {
+        // lane -> row (lane & 15) and every other group starting at lane >> 4
+        const int rr = lane & 15;
+        const int64_t obase = (int64_t)(tile_row + rr) * ngroups + G0;
+        for (int g0 = lane >> 4; g0 < nsub; g0 += 32) {
             unsigned short sv[16];
             unsigned char zv[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const int i = base + j * 32;
-                if (i < items) {
-                    const int rr = i / nsub, gg = i - rr * nsub;
-                    const int64_t o = (int64_t)(tile_row + rr) * ngroups + G0 + gg;
-                    sv[j] = __half_as_ushort(M.s[o]);
-                    zv[j] = M.z[o];
+                const int gg = g0 + 2 * j;
+                if (gg < nsub) {
+                    sv[j] = __half_as_ushort(M.s[obase + gg]);
+                    zv[j] = M.z[obase + gg];
                 }
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
-                const int i = base + j * 32;
-                if (i < items) {
-                    const int rr = i / nsub, gg = i - rr * nsub;
+                const int gg = g0 + 2 * j;
+                if (gg < nsub)
                     my_sz[rr * sz_stride + gg] = make_float2(__half2float(__ushort_as_half(sv[j])), 64.0f + (float)zv[j]);
-                }
             }
         }
     }
+    // Everything above reads only static weight data; activations (and R) may
+    // be produced by the preceding kernels, so wait for them here (a no-op when
+    // launched without programmatic serialization).
+    pdl_wait();
     // 3) the CTA's activation slice, paired and swizzled (all loads of a batch first)
     const int stride = warps * 32;
     {
@@ -402,21 +412,37 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
             xrow[n] = xs + tok * wpt + (G0 - C0) * 16;
         }
         const float* xsum_w = xsum + (G0 - C0) * 8 * NT + 2 * t;
-        const uint4* rd = my_ring + lane;
+        // lane (g, t) reads 16 B of rows g and g+8 per group; odd rows read the
+        // second group first so each quarter-warp hits 8 distinct bank groups
+        const int par = g & 1;
+        const unsigned char* rd_lo = my_ring + g * 128 + t * 16;
+        const unsigned char* rd_hi = rd_lo + 8 * 128;
+        bool ok = true;
         for (int p0 = 0; p0 < npairs; p0 += kStages) {
 #pragma unroll
             for (int i = 0; i < kStages; ++i) {
                 const int p = p0 + i;
                 if (p < npairs) {
-                    cp_async_wait<kStages - 1>();     // the oldest stage has landed
+                    if (ok) ok = mbar_wait(my_bars + i, (uint32_t)((p / kStages) & 1), args.status);
+                    const unsigned char* sl = rd_lo + i * 2048;
+                    const unsigned char* sh = rd_hi + i * 2048;
+                    const uint4 l_first = *reinterpret_cast<const uint4*>(sl + par * 64);
+                    const uint4 h_first = *reinterpret_cast<const uint4*>(sh + par * 64);
+                    const uint4 l_second = *reinterpret_cast<const uint4*>(sl + (par ^ 1) * 64);
+                    const uint4 h_second = *reinterpret_cast<const uint4*>(sh + (par ^ 1) * 64);
                     uint4 w4[2][2];
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        w4[h][0] = rd[i * 128 + h * 64];
-                        w4[h][1] = rd[i * 128 + h * 64 + 32];
+                    w4[0][0] = par ? l_second : l_first;
+                    w4[1][0] = par ? l_first : l_second;
+                    w4[0][1] = par ? h_second : h_first;
+                    w4[1][1] = par ? h_first : h_second;
+                    if (p + kStages < npairs) {
+                        fence_proxy_async_smem();   // this lane's reads of the slot precede the refill
+                        __syncwarp();
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(my_bars + i, 2048u);
+                            tma_load_2d(ring_smem + i * 2048, tmq, my_bars + i, (G0 + 2 * (p + kStages)) * 16, tile_row);
+                        }
                     }
-                    if (p + kStages < npairs) issue_stage(ring_base, qlo, qhi, G0 + 2 * (p + kStages), G1, i);
-                    cp_async_commit();
                     const bool two = 2 * p + 1 < nsub;    // warp-uniform
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -463,10 +489,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
     cp_async_wait<0>();
     __syncwarp();   // A rows copied by other lanes of this warp are visible
 
-    // 6) the R kernels have finished once this returns
-    if (args.wait_dep) pdl_wait();
-
-    // 7) split-d reduction in a fixed order, into the finalising warp
+    // 6) split-d reduction in a fixed order, into the finalising warp
     if (kc > 1) {
         // cluster: partials of tile tl go to rank tl % kc, slot [crank][tl / kc]
         const int idx0 = (crank * L.fin_slots + fslot) * NT * 4 * 32 + lane;
@@ -516,7 +539,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
     }
     if (!active) return;
 
-    // 8) rank-r correction A_i R^T, accumulated into the same fp32 registers
+    // 7) rank-r correction A_i R^T, accumulated into the same fp32 registers
     if (has_corr) {
         const __half* a_lo = as + (fslot * 16 + g) * (r + 8);
         const __half* a_hi = a_lo + 8 * (r + 8);
@@ -540,7 +563,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
         }
     }
 
-    // 9) fp16 outputs (round to nearest even)
+    // 8) fp16 outputs (round to nearest even)
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
         const int tk = n * 8 + 2 * t;
@@ -634,56 +657,68 @@ static int resident_ctas(const void* fn, int warps, int kc, size_t smem, int num
     return n;
 }
 
-struct GemvShape { int rt, kw, kc; size_t smem; };
+struct GemvShape { int rt, kw, kc, stages; size_t smem; };
 
-// Pick (rt, kw, kc): all CTAs resident in one wave, as many warps streaming as
-// possible up to 24 per SM, then the fewest splits of d.  If nothing fits in
-// one wave, the shape with the fewest waves.
-static GemvShape choose_shape(const void* fn, int tiles, int d, int T, int r, int nt, int num_sms) {
-    struct Key { const void* fn; int tiles, d, T, r; GemvShape s; };
+static const void* gemv_fn(int nt, int stages) {
+    if (nt == 1) return stages == 8 ? (const void*)corrected_gemv_kernel<1, 8> : (const void*)corrected_gemv_kernel<1, 4>;
+    return stages == 8 ? (const void*)corrected_gemv_kernel<2, 8> : (const void*)corrected_gemv_kernel<2, 4>;
+}
+
+// Pick (rt, kw, kc, stages): all CTAs resident in one wave; then as many SMs
+// busy as possible; then as many resident warps per SM as possible (up to 16);
+// then as many weight bytes in flight per SM as possible (up to 128 KB); then
+// the fewest splits of d.  If nothing fits in one wave, the fewest waves.
+static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sms) {
+    struct Key { int tiles, d, T, r, nt; GemvShape s; };
     static Key memo[128];
     static int used = 0;
     for (int i = 0; i < used; ++i)
-        if (memo[i].fn == fn && memo[i].tiles == tiles && memo[i].d == d && memo[i].T == T && memo[i].r == r)
+        if (memo[i].tiles == tiles && memo[i].d == d && memo[i].T == T && memo[i].r == r && memo[i].nt == nt)
             return memo[i].s;
     const int ngroups = d / 128;
-    const long cap = (long)num_sms * 24;
-    GemvShape best = {0, 0, 0, 0};
-    double best_key[3] = {1e30, 1e30, 1e30};
-    for (int rt = 1; rt <= kMaxWarps; rt *= 2)
-        for (int kw = 1; rt * kw <= kMaxWarps; ++kw)
-            for (int kc = 1; kc <= 8; ++kc) {
-                if (kc > 1 && kw > 1) break;
-                if (kc > ngroups || ceil_div(ngroups, kc) < kw) continue;
-                const int warps = rt * kw;
-                const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, nt);
-                if (L.total > 220 * 1024) continue;
-                const int res = resident_ctas(fn, warps, kc, (size_t)L.total, num_sms);
-                if (res <= 0) continue;
-                const long ctas = (long)ceil_div(tiles, rt) * kc;
-                const double waves = (double)ctas / res;
-                double key[3];
-                if (waves <= 1.0) {
-                    key[0] = 0;
-                    key[1] = -(double)(ctas * warps < cap ? ctas * warps : cap);
-                    key[2] = kw * kc - 0.01 * rt;
-                } else {
-                    key[0] = waves;
-                    key[1] = 0;
-                    key[2] = kw * kc;
+    GemvShape best = {0, 0, 0, 0, 0};
+    double best_key[5] = {1e30, 1e30, 1e30, 1e30, 1e30};
+    for (int stages = 4; stages <= 8; stages *= 2)
+        for (int rt = 1; rt <= kMaxWarps; rt *= 2)
+            for (int kw = 1; rt * kw <= kMaxWarps; ++kw)
+                for (int kc = 1; kc <= 8; ++kc) {
+                    if (kc > 1 && kw > 1) break;
+                    if (kc > ngroups || ngroups / kc < kw) continue;
+                    const int warps = rt * kw;
+                    const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, nt, stages);
+                    if (L.total > 220 * 1024) continue;
+                    const void* fn = gemv_fn(nt, stages);
+                    const int res = resident_ctas(fn, warps, kc, (size_t)L.total, num_sms);
+                    if (res <= 0) continue;
+                    const long ctas = (long)ceil_div(tiles, rt) * kc;
+                    const double waves = (double)ctas / res;
+                    const long sms = ctas < num_sms ? ctas : num_sms;
+                    const double warps_sm = (double)(ctas * warps) / sms;
+                    // bytes a warp can have in flight: its ring, or its whole slice if smaller
+                    const int groups_warp = ceil_div(ceil_div(ngroups, kc), kw);
+                    const double inflight_warp = 1024.0 * (groups_warp < 2 * stages ? groups_warp : 2 * stages);
+                    const double inflight_sm = inflight_warp * warps_sm;
+                    double key[5];
+                    key[0] = waves <= 1.0 ? 0.0 : waves;
+                    key[1] = -(double)sms;
+                    key[2] = -(warps_sm < 16.0 ? warps_sm : 16.0);
+                    key[3] = -(inflight_sm < 131072.0 ? inflight_sm : 131072.0);
+                    key[4] = kw * kc + 0.1 * stages - 0.01 * rt;
+                    bool better = false;
+                    for (int j = 0; j < 5; ++j) {
+                        if (key[j] < best_key[j] - 1e-9) { better = true; break; }
+                        if (key[j] > best_key[j] + 1e-9) break;
+                    }
+                    if (better) {
+                        for (int j = 0; j < 5; ++j) best_key[j] = key[j];
+                        best = {rt, kw, kc, stages, (size_t)L.total};
+                    }
                 }
-                if (key[0] < best_key[0] || (key[0] == best_key[0] && (key[1] < best_key[1] ||
-                                                                       (key[1] == best_key[1] && key[2] < best_key[2])))) {
-                    best_key[0] = key[0];
-                    best_key[1] = key[1];
-                    best_key[2] = key[2];
-                    best = {rt, kw, kc, (size_t)L.total};
-                }
-            }
-    if (used < 128 && best.rt > 0) memo[used++] = {fn, tiles, d, T, r, best};
+    if (used < 128 && best.rt > 0) memo[used++] = {tiles, d, T, r, nt, best};
     if (std::getenv("GLOWQ_VERBOSE"))
-        std::fprintf(stderr, "glowq decode shape: tiles=%d d=%d T=%d r=%d -> rt=%d kw=%d kc=%d smem=%zu ctas=%d\n",
-                     tiles, d, T, r, best.rt, best.kw, best.kc, best.smem,
+        std::fprintf(stderr,
+                     "glowq decode shape: tiles=%d d=%d T=%d r=%d -> rt=%d kw=%d kc=%d stages=%d smem=%zu ctas=%d\n",
+                     tiles, d, T, r, best.rt, best.kw, best.kc, best.stages, best.smem,
                      best.rt ? ceil_div(tiles, best.rt) * best.kc : 0);
     return best;
 }
@@ -702,18 +737,40 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
         a.mod[i].O = (int)mods[i].O;
         a.mod[i].tile_begin = tiles;
         tiles += (int)(mods[i].O / 16);
+        if (!make_map(&a.tmq[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, mods[i].q, (uint64_t)(d / 8), (uint64_t)mods[i].O,
+                      (uint64_t)d / 2, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
+            return cudaErrorInvalidValue;
     }
     if (tiles == 0) return cudaSuccess;
     const int nt = (T <= 8) ? 1 : 2;
-    const void* fn = (nt == 1) ? (const void*)corrected_gemv_kernel<1> : (const void*)corrected_gemv_kernel<2>;
-    static bool opted[2] = {false, false};
-    if (!opted[nt - 1]) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-        if (e != cudaSuccess) return e;
-        opted[nt - 1] = true;
+    static bool opted = false;
+    if (!opted) {
+        for (int n = 1; n <= 2; ++n)
+            for (int sg = 4; sg <= 8; sg *= 2) {
+                cudaError_t e = cudaFuncSetAttribute(gemv_fn(n, sg), cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+                if (e != cudaSuccess) return e;
+            }
+        opted = true;
     }
-    const GemvShape sh = choose_shape(fn, tiles, d, T, r, nt, num_sms);
+    GemvShape sh = choose_shape(tiles, d, T, r, nt, num_sms);
+    // Tuning override: GLOWQ_DECODE_SHAPE="rt,kw,kc,stages" (validated here).
+    if (const char* env = std::getenv("GLOWQ_DECODE_SHAPE")) {
+        int v[4] = {0, 0, 0, 0};
+        if (std::sscanf(env, "%d,%d,%d,%d", &v[0], &v[1], &v[2], &v[3]) == 4 && v[0] >= 1 && v[1] >= 1 &&
+            v[2] >= 1 && v[2] <= 8 && (v[0] & (v[0] - 1)) == 0 && v[0] * v[1] <= kMaxWarps && (v[2] == 1 || v[1] == 1) &&
+            (v[3] == 4 || v[3] == 8) && v[2] <= d / 128 && (d / 128) / v[2] >= v[1]) {
+            const GemvLayout L = gemv_layout(T, d, r, v[0], v[1], v[2], nt, v[3]);
+            if (L.total <= 220 * 1024) sh = {v[0], v[1], v[2], v[3], (size_t)L.total};
+        }
+    }
     if (sh.rt == 0) return cudaErrorInvalidValue;
+    GemvPlan plan = {};
+    plan.L = gemv_layout(T, d, r, sh.rt, sh.kw, sh.kc, nt, sh.stages);
+    const int ngroups = d / 128;
+    for (int c = 0; c < sh.kc; ++c) {
+        const int c0 = c * ngroups / sh.kc, c1 = (c + 1) * ngroups / sh.kc;
+        for (int k = 0; k <= sh.kw; ++k) plan.gsplit[c * sh.kw + k] = c0 + k * (c1 - c0) / sh.kw;
+    }
     a.m = m;
     a.d = d;
     a.T = T;
@@ -722,9 +779,10 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     a.rt = sh.rt;
     a.kw = sh.kw;
     a.kc = sh.kc;
-    a.wait_dep = after_rproj ? 1 : 0;
+    (void)after_rproj;   // the kernel always waits for its predecessors before reading X and R
     a.X = reinterpret_cast<const __half*>(X);
     a.R = reinterpret_cast<const __half*>(R);
+    a.status = device_status_ptr();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ceil_div(tiles, sh.rt) * sh.kc);
     cfg.blockDim = dim3(sh.rt * sh.kw * 32);
@@ -737,15 +795,14 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     attr[na].val.clusterDim.y = 1;
     attr[na].val.clusterDim.z = 1;
     ++na;
-    if (after_rproj) {
-        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
+    // always programmatic: the weight stream starts while the preceding kernel finishes
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
     cfg.attrs = attr;
     cfg.numAttrs = na;
-    void* args[] = {(void*)&a};
-    return cudaLaunchKernelExC(&cfg, fn, args);
+    void* args[] = {(void*)&a, (void*)&plan};
+    return cudaLaunchKernelExC(&cfg, gemv_fn(nt, sh.stages), args);
 }
 
 }  // namespace glowq

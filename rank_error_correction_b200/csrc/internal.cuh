@@ -1,6 +1,7 @@
 // internal.cuh -- declarations shared by the translation units of libglowq.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -38,7 +39,14 @@ cudaError_t launch_dequant_int4(const uint32_t* q, const uint16_t* s, const uint
                                 uint16_t* out, cudaStream_t st);
 cudaError_t launch_error_norms(const float* W, const uint32_t* q, const uint16_t* s, const uint8_t* z,
                                int64_t O, int64_t d, double* out_rows, cudaStream_t st);
-// prefill.cu
+// prefill.cu: TMA tensor maps (driver entry point resolved at run time)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn();
+// 2-D row-major tensor [outer][inner], row pitch `pitch` bytes, box {box_inner, box_outer}.
+bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+              uint64_t pitch, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r,
                                    const uint16_t* X, int64_t T, uint16_t* R, int num_sms, cudaStream_t st);
 
