@@ -107,8 +107,30 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 2-D tiled TMA store (shared -> global), bulk-group completion.
+__device__ __forceinline__ void tma_store_2d(const void* map, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // ---------------------------------------------------------------------------
-// Corrected GEMM (one 128 x 256 output tile per CTA)
+// Corrected GEMM: persistent, one CTA per SM, 128 x 256 output tiles taken
+// round-robin; the fp32 accumulator is double-buffered in TMEM (2 x 256
+// columns) so the epilogue of one tile overlaps the main loop of the next.
+// Warp roles (448 threads):
+//   warp 0       TMA producer (X tiles, INT4 tiles; A_i / R tiles of the slab)
+//   warp 1       TMEM allocation; one thread issues tcgen05.mma
+//   warps 2-9    transform: INT4 tile -> exact fp16 w_hat (SW128 K-major);
+//                two threads per row, each half of the k-block
+//   warps 10-13  epilogue: TMEM -> fp16 y
 // ---------------------------------------------------------------------------
 constexpr int kBM = 128;          // output rows per tile (TMEM lanes)
 constexpr int kBN = 256;          // tokens per tile (TMEM columns)
@@ -116,9 +138,13 @@ constexpr int kBK = 64;           // k per stage: one 128-byte swizzle atom of f
 constexpr int kGemmStages = 4;
 constexpr int kXBytes = kBN * kBK * 2;       // 32 KB
 constexpr int kWBytes = kBM * kBK * 2;       // 16 KB
-constexpr int kQBytes = kBM * (kBK / 8) * 4; // 4 KB packed codes
+constexpr int kQBytes = kBM * (kBK / 8) * 4; // 4 KB packed codes (32B-swizzled rows)
 constexpr int kStageBytesG = kXBytes + kWBytes + kQBytes;   // multiple of 1024
-constexpr int kGemmThreads = 192;            // 6 warps
+constexpr int kGemmThreads = 448;            // 14 warps
+constexpr int kTransformThreads = 256;
+constexpr int kAccCols = 2 * kBN;            // double-buffered accumulator
+constexpr int kEpiChunk = 32;                // tokens per epilogue chunk (TMEM columns)
+constexpr int kEpiBytes = kEpiChunk * kBM * 2;   // 8 KB: [32 tokens][128 rows] fp16
 
 struct PrefillModule {
     const __half* s;
@@ -133,57 +159,69 @@ struct PrefillModule {
 struct PrefillArgs {
     CUtensorMap tmX;                       // X [T][d] fp16, box {64, 256}, SW128
     CUtensorMap tmR;                       // R [T][r] fp16, box {64, 256}, SW128
-    CUtensorMap tmQ[GLOWQ_MAX_MODULES];    // qweight [O][d/8] u32, box {8, 128}
+    CUtensorMap tmQ[GLOWQ_MAX_MODULES];    // qweight [O][d/8] u32, box {8, 128}, SW32
     CUtensorMap tmA[GLOWQ_MAX_MODULES];    // A [O][r] fp16, box {64, 128}, SW128
+    CUtensorMap tmY[GLOWQ_MAX_MODULES];    // Y [T][ldY] fp16 (O columns), box {128, 32} (TMA store)
     PrefillModule mod[GLOWQ_MAX_MODULES];
     int m;
     int d;
     int T;
     int r;
     int ntiles_n;                          // token tiles
+    int ntiles;                            // all tiles
     int wait_dep;                          // R comes from the preceding (PDL) kernel
     unsigned int* status;
 };
 
 struct __align__(8) GemmBarriers {
     uint64_t full[kGemmStages];    // TMA bytes landed (expect_tx by the producer)
-    uint64_t dq[kGemmStages];      // transform warps wrote w_hat (128 arrivals)
+    uint64_t dq[kGemmStages];      // transform warps wrote w_hat (256 arrivals)
     uint64_t empty[kGemmStages];   // MMAs reading the stage completed (tcgen05.commit)
-    uint64_t acc;                  // accumulator complete
+    uint64_t acc_full[2];          // accumulator buffer complete (tcgen05.commit)
+    uint64_t acc_empty[2];         // accumulator buffer drained (128 epilogue arrivals)
     uint32_t tmem_base;
 };
+
+struct TileCoord {
+    int mi, m0, n0, nslab;
+};
+
+__device__ __forceinline__ TileCoord tile_coord(const PrefillArgs& args, int tile) {
+    TileCoord c;
+    const int mt = tile / args.ntiles_n;
+    const int nt = tile - mt * args.ntiles_n;
+    int mi = 0;
+    for (int i = 1; i < args.m; ++i)
+        if (mt >= args.mod[i].mtile_begin) mi = i;
+    c.mi = mi;
+    c.m0 = (mt - args.mod[mi].mtile_begin) * kBM;
+    c.n0 = nt * kBN;
+    c.nslab = (args.r > 0 && args.mod[mi].has_A) ? (args.r + kBK - 1) / kBK : 0;
+    return c;
+}
 
 __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const __grid_constant__ PrefillArgs args) {
     extern __shared__ __align__(1024) unsigned char gsm_raw[];
     // 1024-byte alignment of the stage buffers (swizzle atoms)
     unsigned char* gsm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
-    GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(gsm + kGemmStages * kStageBytesG);
+    unsigned char* epi = gsm + kGemmStages * kStageBytesG;            // 2 x kEpiBytes
+    GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(epi + 2 * kEpiBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    // tile -> (module, m tile, n tile)
-    const int ntn = args.ntiles_n;
-    const int mt_global = blockIdx.x / ntn;
-    const int nt = blockIdx.x % ntn;
-    int mi = 0;
-    for (int i = 1; i < args.m; ++i)
-        if (mt_global >= args.mod[i].mtile_begin) mi = i;
-    const PrefillModule& M = args.mod[mi];
-    const int m0 = (mt_global - M.mtile_begin) * kBM;   // module-local first row
-    const int n0 = nt * kBN;
     const int nkb = args.d / kBK;
-    const int nslab = (args.r > 0 && M.has_A) ? (args.r + kBK - 1) / kBK : 0;
-    const int nblocks = nkb + nslab;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
             mbar_init(&bars->full[s], 1);
-            mbar_init(&bars->dq[s], 128);
+            mbar_init(&bars->dq[s], kTransformThreads);
             mbar_init(&bars->empty[s], 1);
         }
-        mbar_init(&bars->acc, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bars->acc_full[b], 1);
+            mbar_init(&bars->acc_empty[b], 128);
+        }
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(&bars->tmem_base, kBN);
+    if (warp == 1) tmem_alloc(&bars->tmem_base, kAccCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -193,22 +231,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
     if (warp == 0) {
         // ---------------- producer ----------------
         if (lane == 0) {
-            bool ok = true;
-            for (int i = 0; i < nblocks; ++i) {
-                const int s = i % kGemmStages;
-                if (i >= kGemmStages && ok) ok = mbar_wait(&bars->empty[s], ((i / kGemmStages) - 1) & 1, args.status);
-                unsigned char* st = gsm + s * kStageBytesG;
-                const uint32_t xs = smem_u32(st), ws = smem_u32(st + kXBytes), qs = smem_u32(st + kXBytes + kWBytes);
-                if (i < nkb) {
-                    mbar_arrive_expect_tx(&bars->full[s], kXBytes + kQBytes);
-                    tma_load_2d(xs, &args.tmX, &bars->full[s], i * kBK, n0);
-                    tma_load_2d(qs, &args.tmQ[mi], &bars->full[s], i * (kBK / 8), m0);
-                } else {
-                    if (i == nkb && args.wait_dep) pdl_wait();   // R is complete
-                    const int j = i - nkb;
-                    mbar_arrive_expect_tx(&bars->full[s], kXBytes + kWBytes);
-                    tma_load_2d(xs, &args.tmR, &bars->full[s], j * kBK, n0);
-                    tma_load_2d(ws, &args.tmA[mi], &bars->full[s], j * kBK, m0);
+            bool ok = true, waited = false;
+            int g = 0;   // global k-block counter of this CTA (ring position)
+            for (int tile = blockIdx.x; tile < args.ntiles; tile += gridDim.x) {
+                const TileCoord c = tile_coord(args, tile);
+                const int nblocks = nkb + c.nslab;
+                for (int i = 0; i < nblocks; ++i, ++g) {
+                    const int s = g % kGemmStages;
+                    if (g >= kGemmStages && ok) ok = mbar_wait(&bars->empty[s], ((g / kGemmStages) - 1) & 1, args.status);
+                    unsigned char* st = gsm + s * kStageBytesG;
+                    const uint32_t xs = smem_u32(st), ws = smem_u32(st + kXBytes), qs = smem_u32(st + kXBytes + kWBytes);
+                    if (i < nkb) {
+                        mbar_arrive_expect_tx(&bars->full[s], kXBytes + kQBytes);
+                        tma_load_2d(xs, &args.tmX, &bars->full[s], i * kBK, c.n0);
+                        tma_load_2d(qs, &args.tmQ[c.mi], &bars->full[s], i * (kBK / 8), c.m0);
+                    } else {
+                        if (!waited && args.wait_dep) {   // R is complete
+                            pdl_wait();
+                            waited = true;
+                        }
+                        const int j = i - nkb;
+                        mbar_arrive_expect_tx(&bars->full[s], kXBytes + kWBytes);
+                        tma_load_2d(xs, &args.tmR, &bars->full[s], j * kBK, c.n0);
+                        tma_load_2d(ws, &args.tmA[c.mi], &bars->full[s], j * kBK, c.m0);
+                    }
                 }
             }
         }
@@ -217,96 +263,158 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
         if (lane == 0) {
             constexpr uint32_t idesc = f16_idesc(kBM, kBN);
             bool ok = true;
-            for (int i = 0; i < nblocks; ++i) {
-                const int s = i % kGemmStages;
-                const uint32_t par = (i / kGemmStages) & 1;
-                if (ok) ok = (i < nkb) ? mbar_wait(&bars->dq[s], par, args.status) : mbar_wait(&bars->full[s], par, args.status);
+            int g = 0, tl = 0;
+            for (int tile = blockIdx.x; tile < args.ntiles; tile += gridDim.x, ++tl) {
+                const TileCoord c = tile_coord(args, tile);
+                const int nblocks = nkb + c.nslab;
+                const int buf = tl & 1;
+                if (tl >= 2 && ok) ok = mbar_wait(&bars->acc_empty[buf], ((tl >> 1) - 1) & 1, args.status);
                 tc_fence_after();
-                unsigned char* st = gsm + s * kStageBytesG;
-                const uint32_t xs = smem_u32(st), ws = smem_u32(st + kXBytes);
+                const uint32_t dacc = tmem + (uint32_t)(buf * kBN);
+                for (int i = 0; i < nblocks; ++i, ++g) {
+                    const int s = g % kGemmStages;
+                    const uint32_t par = (g / kGemmStages) & 1;
+                    // dq completes once per block (slab blocks too, after their TMA landed)
+                    if (ok) ok = mbar_wait(&bars->dq[s], par, args.status);
+                    tc_fence_after();
+                    unsigned char* st = gsm + s * kStageBytesG;
+                    const uint32_t xs = smem_u32(st), ws = smem_u32(st + kXBytes);
 #pragma unroll
-                for (int k = 0; k < kBK / 16; ++k) {
-                    const uint64_t ad = sw128_kmajor_desc(ws + k * 32);
-                    const uint64_t bd = sw128_kmajor_desc(xs + k * 32);
-                    umma_f16(tmem, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        const uint64_t ad = sw128_kmajor_desc(ws + k * 32);
+                        const uint64_t bd = sw128_kmajor_desc(xs + k * 32);
+                        umma_f16(dacc, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit(&bars->empty[s]);   // frees the stage once these MMAs complete
                 }
-                umma_commit(&bars->empty[s]);   // frees the stage once these MMAs complete
+                umma_commit(&bars->acc_full[buf]);  // this tile's accumulator is complete
             }
-            umma_commit(&bars->acc);
+        }
+    } else if (warp < 10) {
+        // ---------------- transform (warps 2..9) ----------------
+        const int tt = threadIdx.x - 64;
+        const int row = tt & 127;                      // tile row owned by this thread
+        const int half = tt >> 7;                      // which 32 k of the 64-k block
+        const int ngroups = args.d / 128;
+        const uint32_t swz = (uint32_t)(row & 7);
+        bool ok = true;
+        int g = 0;
+        // scale/zero of the current and the next 3 groups (a shift register
+        // refilled 4 groups ahead, across tile boundaries)
+        int cur_tile = blockIdx.x;
+        TileCoord cc = tile_coord(args, cur_tile < args.ntiles ? cur_tile : 0);
+        int f_tile = cur_tile, f_grp = 0;              // next group to fetch
+        TileCoord fc = cc;
+        auto fetch = [&]() -> uint32_t {
+            uint32_t v = 0;
+            if (f_tile < args.ntiles) {
+                const int orow = fc.m0 + row;
+                const PrefillModule& FM = args.mod[fc.mi];
+                if (orow < FM.O) {
+                    const int64_t o = (int64_t)orow * ngroups + f_grp;
+                    v = (uint32_t)__half_as_ushort(FM.s[o]) | ((uint32_t)FM.z[o] << 16);
+                }
+                if (++f_grp == ngroups) {
+                    f_grp = 0;
+                    f_tile += gridDim.x;
+                    if (f_tile < args.ntiles) fc = tile_coord(args, f_tile);
+                }
+            }
+            return v;
+        };
+        uint32_t sz0 = fetch(), sz1 = fetch(), sz2 = fetch(), sz3 = fetch();
+        for (; cur_tile < args.ntiles; cur_tile += gridDim.x) {
+            cc = tile_coord(args, cur_tile);
+            const int nblocks = nkb + cc.nslab;
+            for (int i = 0; i < nkb; ++i, ++g) {
+                const int s = g % kGemmStages;
+                if (ok) ok = mbar_wait(&bars->full[s], (g / kGemmStages) & 1, args.status);
+                unsigned char* st = gsm + s * kStageBytesG;
+                // 32-byte-swizzled INT4 rows: 16-byte half h of row r sits at r*32 + ((h ^ (r>>2)&1) << 4)
+                const unsigned char* qrow = st + kXBytes + kWBytes + row * 32;
+                const uint32_t hsw = (uint32_t)((row >> 2) & 1);
+                const uint4 q0 = *reinterpret_cast<const uint4*>(qrow + (((uint32_t)half ^ hsw) << 4));
+                const uint32_t sz = sz0;                             // group i/2
+                if ((i & 1) == 1) {                                  // group done: shift, fetch 4 ahead
+                    sz0 = sz1;
+                    sz1 = sz2;
+                    sz2 = sz3;
+                    sz3 = fetch();
+                }
+                const __half2 sc = __half2half2(__ushort_as_half((unsigned short)(sz & 0xffffu)));
+                const __half2 bz = __half2half2(__ushort_as_half((unsigned short)(0x6400u | ((sz >> 16) & 0xffu))));
+                const uint32_t words[4] = {q0.x, q0.y, q0.z, q0.w};
+                // row `row` of the W tile: 8 chunks of 16 B (8 fp16 in k order), chunk c at c ^ (row % 8)
+                unsigned char* wrow = st + kXBytes + (row >> 3) * 1024 + (row & 7) * 128;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int c = half * 4 + j;
+                    __half2 p[4];
+                    dequant_word(words[j], bz, sc, p);   // pairs (0,4) (1,5) (2,6) (3,7), exact w_hat
+                    const uint32_t u0 = h2_as_u32(p[0]), u1 = h2_as_u32(p[1]), u2 = h2_as_u32(p[2]), u3 = h2_as_u32(p[3]);
+                    uint4 o;
+                    o.x = pair_lo(u0, u1);   // (0,1)
+                    o.y = pair_lo(u2, u3);   // (2,3)
+                    o.z = pair_hi(u0, u1);   // (4,5)
+                    o.w = pair_hi(u2, u3);   // (6,7)
+                    *reinterpret_cast<uint4*>(wrow + (((uint32_t)c ^ swz) << 4)) = o;
+                }
+                fence_proxy_async_smem();   // generic-proxy writes visible to the tensor cores
+                mbar_arrive(&bars->dq[s]);
+            }
+            // slab blocks are filled by TMA alone; still advance dq once per block
+            // (after the TMA landed) so its phases follow the ring position
+            for (int i = nkb; i < nblocks; ++i, ++g) {
+                const int s = g % kGemmStages;
+                if (ok) ok = mbar_wait(&bars->full[s], (g / kGemmStages) & 1, args.status);
+                mbar_arrive(&bars->dq[s]);
+            }
         }
     } else {
-        // ---------------- transform + epilogue (warps 2..5) ----------------
+        // ---------------- epilogue (warps 10..13) ----------------
+        // Each 32-token chunk of the accumulator is transposed through shared
+        // memory ([32 tokens][128 rows] fp16) and written by one TMA store,
+        // which clips rows >= O and tokens >= T.  Two staging buffers: a buffer
+        // is rewritten only after the store issued from it two chunks earlier
+        // has finished reading it.
         const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
-        const int row = quarter * 32 + lane;           // tile row owned by this thread
-        const int orow = m0 + row;                     // module-local output row
-        const bool row_ok = orow < M.O;
-        const int ngroups = args.d / 128;
-        const __half* srow = M.s + (int64_t)(row_ok ? orow : 0) * ngroups;
-        const uint8_t* zrow = M.z + (int64_t)(row_ok ? orow : 0) * ngroups;
-        // scale/zero of the current and the next 3 groups (a shift register,
-        // refilled 4 groups ahead so the loads are long complete when used)
-        auto load_sz = [&](int gi) -> uint32_t {
-            return (row_ok && gi < ngroups) ? ((uint32_t)__half_as_ushort(srow[gi]) | ((uint32_t)zrow[gi] << 16)) : 0u;
-        };
-        uint32_t sz0 = load_sz(0), sz1 = load_sz(1), sz2 = load_sz(2), sz3 = load_sz(3);
+        const int row = quarter * 32 + lane;
+        const bool leader = (warp == 10 && lane == 0);
         bool ok = true;
-        const uint32_t swz = (uint32_t)(row & 7);
-        for (int i = 0; i < nkb; ++i) {
-            const int s = i % kGemmStages;
-            if (ok) ok = mbar_wait(&bars->full[s], (i / kGemmStages) & 1, args.status);
-            unsigned char* st = gsm + s * kStageBytesG;
-            const uint4* qrow = reinterpret_cast<const uint4*>(st + kXBytes + kWBytes + row * 32);
-            const uint4 q0 = qrow[0], q1 = qrow[1];
-            const uint32_t sz = sz0;                             // group i/2
-            if ((i & 1) == 1) {                                  // group done: shift, fetch the one 4 ahead
-                sz0 = sz1;
-                sz1 = sz2;
-                sz2 = sz3;
-                sz3 = load_sz((i >> 1) + 4);
-            }
-            const __half2 sc = __half2half2(__ushort_as_half((unsigned short)(sz & 0xffffu)));
-            const __half2 bz = __half2half2(__ushort_as_half((unsigned short)(0x6400u | ((sz >> 16) & 0xffu))));
-            const uint32_t words[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-            // row `row` of the W tile: 8 chunks of 16 B (8 fp16 in k order), chunk c at c ^ (row % 8)
-            unsigned char* wrow = st + kXBytes + (row >> 3) * 1024 + (row & 7) * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                __half2 p[4];
-                dequant_word(words[c], bz, sc, p);   // pairs (0,4) (1,5) (2,6) (3,7), exact w_hat
-                const uint32_t u0 = h2_as_u32(p[0]), u1 = h2_as_u32(p[1]), u2 = h2_as_u32(p[2]), u3 = h2_as_u32(p[3]);
-                uint4 o;
-                o.x = pair_lo(u0, u1);   // (0,1)
-                o.y = pair_lo(u2, u3);   // (2,3)
-                o.z = pair_hi(u0, u1);   // (4,5)
-                o.w = pair_hi(u2, u3);   // (6,7)
-                *reinterpret_cast<uint4*>(wrow + (((uint32_t)c ^ swz) << 4)) = o;
-            }
-            fence_proxy_async_smem();   // generic-proxy writes visible to the tensor cores
-            mbar_arrive(&bars->dq[s]);
-        }
-        // ---- epilogue: TMEM -> fp16 y ----
-        if (ok) mbar_wait(&bars->acc, 0, args.status);
-        tc_fence_after();
-        const uint32_t tl = tmem + ((uint32_t)(quarter * 32) << 16);
-        __half* ybase = M.Y + orow;
-        const int T = args.T;
+        int tl = 0, chunk = 0;
+        for (int tile = blockIdx.x; tile < args.ntiles; tile += gridDim.x, ++tl) {
+            const TileCoord c = tile_coord(args, tile);
+            const int buf = tl & 1;
+            if (ok) ok = mbar_wait(&bars->acc_full[buf], (tl >> 1) & 1, args.status);
+            tc_fence_after();
+            const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN);
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
-            uint32_t v[32];
-            tmem_ld32(tl + c * 32, v);
-            if (row_ok) {
-                const int t0 = n0 + c * 32;
+            for (int ch = 0; ch < kBN / kEpiChunk; ++ch, ++chunk) {
+                uint32_t v[32];
+                tmem_ld32(tacc + ch * kEpiChunk, v);
+                unsigned char* sb = epi + (chunk & 1) * kEpiBytes;
+                if (leader) bulk_wait_read<1>();          // the store from this buffer is done reading
+                named_barrier_sync(1, 128);
+                __half* col = reinterpret_cast<__half*>(sb) + row;
 #pragma unroll
-                for (int j = 0; j < 32; ++j)
-                    if (t0 + j < T) ybase[(int64_t)(t0 + j) * M.ldY] = __float2half_rn(__uint_as_float(v[j]));
+                for (int j = 0; j < 32; ++j) col[j * kBM] = __float2half_rn(__uint_as_float(v[j]));
+                fence_proxy_async_smem();
+                named_barrier_sync(1, 128);
+                if (leader) {
+                    tma_store_2d(&args.tmY[c.mi], smem_u32(sb), c.m0, c.n0 + ch * kEpiChunk);
+                    bulk_commit();
+                }
             }
+            tc_fence_before();
+            mbar_arrive(&bars->acc_empty[buf]);        // buffer may be overwritten
         }
+        if (leader) bulk_wait_all();
     }
     // the R kernel is complete before this grid is (even if no tile read R)
     if (args.wait_dep) pdl_wait();
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, kBN);
+    if (warp == 1) tmem_dealloc(tmem, kAccCols);
 }
 
 // ---------------------------------------------------------------------------
@@ -457,7 +565,9 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t gemm_smem_bytes() { return (size_t)kGemmStages * kStageBytesG + sizeof(GemmBarriers) + 1024; }
+static size_t gemm_smem_bytes() {
+    return (size_t)kGemmStages * kStageBytesG + 2 * kEpiBytes + sizeof(GemmBarriers) + 1024;
+}
 static size_t rproj_smem_bytes(int rn) { return (size_t)kRStages * rproj_stage_bytes(rn) + sizeof(RprojBarriers) + 1024; }
 
 static cudaError_t launch_with(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
@@ -506,7 +616,6 @@ cudaError_t launch_rproj_prefill(const uint16_t* X, const uint16_t* B, int64_t T
 
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r, const uint16_t* X,
                                    int64_t T, uint16_t* R, int num_sms, cudaStream_t st) {
-    (void)num_sms;
     if (T > ((int64_t)1 << 30)) return GLOWQ_ERR_SHAPE;
     if (!encode_fn()) return GLOWQ_ERR_CUDA;
     const bool use_r = r > 0 && B != nullptr;
@@ -531,11 +640,13 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     for (int i = 0; i < m && ok; ++i) {
         const ModuleView& mv = mods[i];
         ok = ok && make_map(&a->tmQ[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, mv.q, (uint64_t)(d / 8), (uint64_t)mv.O,
-                            (uint64_t)d / 2, kBK / 8, kBM, CU_TENSOR_MAP_SWIZZLE_NONE);
+                            (uint64_t)d / 2, kBK / 8, kBM, CU_TENSOR_MAP_SWIZZLE_32B);
         const bool has_A = use_r && mv.A != nullptr;
         if (has_A)
             ok = ok && make_map(&a->tmA[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, mv.A, (uint64_t)r, (uint64_t)mv.O,
                                 (uint64_t)r * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
+        ok = ok && make_map(&a->tmY[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, mv.Y, (uint64_t)mv.O, (uint64_t)T,
+                            (uint64_t)mv.ldY * 2, kBM, kEpiChunk, CU_TENSOR_MAP_SWIZZLE_NONE);
         a->mod[i].s = reinterpret_cast<const __half*>(mv.s);
         a->mod[i].z = mv.z;
         a->mod[i].Y = reinterpret_cast<__half*>(mv.Y);
@@ -556,8 +667,11 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     a->ntiles_n = (int)((T + kBN - 1) / kBN);
     a->wait_dep = use_r ? 1 : 0;
     a->status = device_status_ptr();
+    const int64_t ntiles = (int64_t)mtiles * a->ntiles_n;
+    a->ntiles = (int)ntiles;
     void* args[] = {(void*)a};
-    const int64_t grid = (int64_t)mtiles * a->ntiles_n;
+    // persistent grid: one CTA per SM (fewer if there are fewer tiles)
+    const int64_t grid = ntiles < num_sms ? ntiles : num_sms;
     cudaError_t e = cudaSuccess;
     if (grid > 0)
         e = launch_with((const void*)corrected_gemm_kernel, dim3((unsigned)grid), dim3(kGemmThreads), gemm_smem_bytes(),
