@@ -10,22 +10,25 @@
 //   rproj_tc_kernel        R = X B^T (T x r), M = 128 tokens per CTA, N = r,
 //                          both operands fp16 by TMA, fp32 TMEM accumulator,
 //                          rounded to fp16.
-//   corrected_gemm_kernel  one 128-row x 256-token tile of y per CTA:
+//   corrected_gemm_kernel  one 256-row x 256-token tile of y per CTA pair
+//                          (thread-block cluster of 2, tcgen05 cta_group::2):
 //                          D[o][t] = sum_k w_hat[o][k] X[t][k] + sum_j A[o][j] R[t][j]
-//                          - a producer warp streams X tiles (SW128) and packed
-//                            INT4 tiles with TMA into a 4-stage ring;
-//                          - four transform warps dequantise each INT4 tile to
-//                            the exact fp16 w_hat = fp16((q - z) s) straight into
-//                            the canonical K-major 128B-swizzled layout the MMA
-//                            reads;
-//                          - one thread issues tcgen05.mma (M=128, N=256, K=16)
-//                            into a 256-column fp32 TMEM accumulator;
+//                          - in each CTA a producer warp streams its half of the
+//                            X tile (SW128) and its 128 rows of packed INT4 with
+//                            TMA into a 5-stage ring;
+//                          - eight transform warps per CTA dequantise each INT4
+//                            tile to the exact fp16 w_hat = fp16((q - z) s)
+//                            straight into the canonical K-major 128B-swizzled
+//                            layout the MMA reads;
+//                          - one thread of the leader CTA issues tcgen05.mma
+//                            (M=256, N=256, K=16) into fp32 TMEM accumulators
+//                            split across the pair (128 rows each);
 //                          - the rank-r correction is one more K=64 slab of the
 //                            same accumulator, A_i and R tiles fetched by TMA
 //                            (zero-filled beyond r), so no separate kernel or
 //                            extra pass over y runs;
-//                          - the transform warps then drain TMEM (tcgen05.ld)
-//                            and store y in fp16.
+//                          - four epilogue warps per CTA drain TMEM (tcgen05.ld)
+//                            and store y in fp16 with TMA.
 // Every wait on an mbarrier is bounded; a wait that runs out records
 // GLOWQ_ERR_TIMEOUT in the device status word.
 #include <cuda.h>
@@ -122,29 +125,51 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
 }
 
 // ---------------------------------------------------------------------------
-// Corrected GEMM: persistent, one CTA per SM, 128 x 256 output tiles taken
-// round-robin; the fp32 accumulator is double-buffered in TMEM (2 x 256
-// columns) so the epilogue of one tile overlaps the main loop of the next.
-// Warp roles (448 threads):
-//   warp 0       TMA producer (X tiles, INT4 tiles; A_i / R tiles of the slab)
-//   warp 1       TMEM allocation; one thread issues tcgen05.mma
+// Corrected GEMM on CTA pairs.  A cluster of two CTAs computes one 256-row x
+// 256-token tile of y with tcgen05.mma.cta_group::2 (M = 256, N = 256, K = 16):
+// CTA p of the pair stages W rows [128p, 128p+128) of the tile (dequantised by
+// its own transform warps) and tokens [128p, 128p+128) of X; the pair's tensor
+// cores read both halves of X, and CTA p's TMEM receives the fp32 accumulator
+// of its 128 W rows for all 256 tokens.  Per SM this halves the X tile staged
+// in shared memory and read by the MMA, relative to a 128 x 256 tile on one SM.
+// Persistent: clusters take pair tiles round-robin; the accumulator is double-
+// buffered in TMEM (2 x 256 columns) so the drain of one tile overlaps the main
+// loop of the next.
+// Synchronisation inside a pair:
+//   full[s]      per CTA: TMA bytes of its own halves landed
+//   dq[s]        leader only: w_hat written and the stage's TMA landed, in both
+//                CTAs (each warp of the owning transform group arrives, 2 x 4)
+//   empty[s]     per CTA: the pair's MMAs reading stage s completed (the
+//                leader's tcgen05.commit arrives on both CTAs' barriers)
+//   acc_full[b]  per CTA: accumulator buffer b complete (leader's commit, both)
+//   acc_empty[b] leader only: both CTAs drained buffer b (one arrival per
+//                epilogue warp, 2 x 4)
+// Warp roles (448 threads per CTA):
+//   warp 0       TMA producer of this CTA's halves (X, INT4; R, A_i for the slab)
+//   warp 1       TMEM allocation (both CTAs); the leader's lane 0 issues the MMAs
 //   warps 2-9    transform: INT4 tile -> exact fp16 w_hat (SW128 K-major);
-//                two threads per row, each half of the k-block
-//   warps 10-13  epilogue: TMEM -> fp16 y
+//                two groups of four warps on alternate k-blocks, one thread per row
+//   warps 10-13  epilogue: TMEM -> fp16 y of this CTA's 128 rows
 // ---------------------------------------------------------------------------
-constexpr int kBM = 128;          // output rows per tile (TMEM lanes)
-constexpr int kBN = 256;          // tokens per tile (TMEM columns)
+constexpr int kBM = 128;          // W rows per CTA (TMEM lanes)
+constexpr int kPairM = 2 * kBM;   // W rows per pair tile (MMA M)
+constexpr int kBN = 256;          // tokens per pair tile (MMA N, TMEM columns)
+constexpr int kHalfN = kBN / 2;   // tokens staged by each CTA
 constexpr int kBK = 64;           // k per stage: one 128-byte swizzle atom of fp16
-constexpr int kGemmStages = 4;
-constexpr int kXBytes = kBN * kBK * 2;       // 32 KB
+constexpr int kGemmStages = 6;                // even: each stage belongs to one transform group
+constexpr int kEpiBufs = 1;                   // epilogue staging buffers
+constexpr int kXBytes = kHalfN * kBK * 2;    // 16 KB
 constexpr int kWBytes = kBM * kBK * 2;       // 16 KB
 constexpr int kQBytes = kBM * (kBK / 8) * 4; // 4 KB packed codes (32B-swizzled rows)
 constexpr int kStageBytesG = kXBytes + kWBytes + kQBytes;   // multiple of 1024
 constexpr int kGemmThreads = 448;            // 14 warps
 constexpr int kTransformThreads = 256;
+constexpr int kEpiThreads = 128;
 constexpr int kAccCols = 2 * kBN;            // double-buffered accumulator
 constexpr int kEpiChunk = 32;                // tokens per epilogue chunk (TMEM columns)
 constexpr int kEpiBytes = kEpiChunk * kBM * 2;   // 8 KB: [32 tokens][128 rows] fp16
+static_assert(kGemmStages % 2 == 0, "transform groups own alternate stages");
+static_assert(kGemmStages * kStageBytesG + kEpiBufs * kEpiBytes + 1024 + 256 <= 232448, "shared memory per CTA");
 
 struct PrefillModule {
     const __half* s;
@@ -157,8 +182,8 @@ struct PrefillModule {
 };
 
 struct PrefillArgs {
-    CUtensorMap tmX;                       // X [T][d] fp16, box {64, 256}, SW128
-    CUtensorMap tmR;                       // R [T][r] fp16, box {64, 256}, SW128
+    CUtensorMap tmX;                       // X [T][d] fp16, box {64, 128}, SW128
+    CUtensorMap tmR;                       // R [T][r] fp16, box {64, 128}, SW128
     CUtensorMap tmQ[GLOWQ_MAX_MODULES];    // qweight [O][d/8] u32, box {8, 128}, SW32
     CUtensorMap tmA[GLOWQ_MAX_MODULES];    // A [O][r] fp16, box {64, 128}, SW128
     CUtensorMap tmY[GLOWQ_MAX_MODULES];    // Y [T][ldY] fp16 (O columns), box {128, 32} (TMA store)
@@ -168,17 +193,17 @@ struct PrefillArgs {
     int T;
     int r;
     int ntiles_n;                          // token tiles
-    int ntiles;                            // all tiles
+    int ntiles;                            // all pair tiles
     int wait_dep;                          // R comes from the preceding (PDL) kernel
     unsigned int* status;
 };
 
 struct __align__(8) GemmBarriers {
-    uint64_t full[kGemmStages];    // TMA bytes landed (expect_tx by the producer)
-    uint64_t dq[kGemmStages];      // transform warps wrote w_hat (256 arrivals)
-    uint64_t empty[kGemmStages];   // MMAs reading the stage completed (tcgen05.commit)
-    uint64_t acc_full[2];          // accumulator buffer complete (tcgen05.commit)
-    uint64_t acc_empty[2];         // accumulator buffer drained (128 epilogue arrivals)
+    uint64_t full[kGemmStages];
+    uint64_t dq[kGemmStages];
+    uint64_t empty[kGemmStages];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
     uint32_t tmem_base;
 };
 
@@ -186,6 +211,7 @@ struct TileCoord {
     int mi, m0, n0, nslab;
 };
 
+// m0: first W row of the pair tile within module mi; n0: first token.
 __device__ __forceinline__ TileCoord tile_coord(const PrefillArgs& args, int tile) {
     TileCoord c;
     const int mt = tile / args.ntiles_n;
@@ -194,34 +220,144 @@ __device__ __forceinline__ TileCoord tile_coord(const PrefillArgs& args, int til
     for (int i = 1; i < args.m; ++i)
         if (mt >= args.mod[i].mtile_begin) mi = i;
     c.mi = mi;
-    c.m0 = (mt - args.mod[mi].mtile_begin) * kBM;
+    c.m0 = (mt - args.mod[mi].mtile_begin) * kPairM;
     c.n0 = nt * kBN;
     c.nslab = (args.r > 0 && args.mod[mi].has_A) ? (args.r + kBK - 1) / kBK : 0;
     return c;
 }
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on a barrier of either CTA of the pair (default .release.cta semantics,
+// as for a local arrive: the consumer of these arrivals is the tensor core of
+// the pair's leader, which reads this CTA's shared memory through the async
+// proxy after the fence.proxy.async of the writers).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t caddr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(caddr) : "memory");
+}
+// Bounded wait whose completing arrivals may come from the other CTA of the pair.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, unsigned int* status,
+                                                  uint32_t limit = (1u << 20)) {
+    const uint32_t a = smem_u32(bar);
+    for (uint32_t it = 0; it < limit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    record_status(status, GLOWQ_ERR_TIMEOUT);
+    return false;
+}
+// One k-block of pair MMAs (4 x K=16) plus the commits that free its stage in
+// both CTAs, preceded by a non-blocking probe of another barrier's phase.  The
+// probe's result is consumed only after the MMAs and commits are issued, so its
+// shared-memory round trip overlaps the issue.  `adesc` / `bdesc` describe the
+// first K=16 slice of the stage; slice k starts 32 bytes further (+2 in the
+// descriptor's 16-byte address field).  Returns the probe result.
+__device__ __forceinline__ uint32_t umma_kblock_pair_probe(uint32_t dacc, uint64_t adesc, uint64_t bdesc,
+                                                           uint32_t idesc, uint32_t accumulate, uint32_t empty_local,
+                                                           uint32_t empty_peer, uint32_t probe_bar,
+                                                           uint32_t probe_parity) {
+    uint32_t ready;
+    asm volatile(
+        "{\n\t.reg .pred pr, pa, pt;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 pr, [%6], %7;\n\t"
+        "setp.ne.b32 pa, %3, 0;\n\t"
+        "setp.eq.b32 pt, %3, %3;\n\t"
+        "add.s64 a1, %8, 2;\n\tadd.s64 a2, %8, 4;\n\tadd.s64 a3, %8, 6;\n\t"
+        "add.s64 b1, %9, 2;\n\tadd.s64 b2, %9, 4;\n\tadd.s64 b3, %9, 6;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], %8, %9, %2, pa;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], a1, b1, %2, pt;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], a2, b2, %2, pt;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%1], a3, b3, %2, pt;\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%4];\n\t"
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+        "selp.u32 %0, 1, 0, pr;\n\t}"
+        : "=r"(ready)
+        : "r"(dacc), "r"(idesc), "r"(accumulate), "r"(empty_local), "r"(empty_peer), "r"(probe_bar),
+          "r"(probe_parity), "l"(adesc), "l"(bdesc)
+        : "memory");
+    return ready;
+}
+__device__ __forceinline__ void umma_f16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                              uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// Arrive on the barrier at cluster address `caddr` once the pair MMAs issued so far complete.
+__device__ __forceinline__ void umma_commit_pair(uint32_t caddr) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(caddr)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
 __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const __grid_constant__ PrefillArgs args) {
     extern __shared__ __align__(1024) unsigned char gsm_raw[];
-    // 1024-byte alignment of the stage buffers (swizzle atoms)
+    // 1024-byte alignment of the stage buffers (swizzle atoms); the same offset in both CTAs
     unsigned char* gsm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* epi = gsm + kGemmStages * kStageBytesG;            // 2 x kEpiBytes
-    GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(epi + 2 * kEpiBytes);
+    unsigned char* epi = gsm + kGemmStages * kStageBytesG;            // kEpiBufs x kEpiBytes
+    GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(epi + kEpiBufs * kEpiBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nkb = args.d / kBK;
+    const uint32_t crank = cluster_ctarank();            // 0 = leader (issues the MMAs)
+    const int first_tile = (int)cluster_id_x();
+    const int tile_step = (int)cluster_count_x();
+    const int row_off = (int)crank * kBM;                // this CTA's W rows within the pair tile
+    const int tok_off = (int)crank * kHalfN;             // this CTA's tokens within the pair tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
             mbar_init(&bars->full[s], 1);
-            mbar_init(&bars->dq[s], kTransformThreads);
+            mbar_init(&bars->dq[s], 2 * kTransformThreads / 64);    // one arrival per warp of the owning group
             mbar_init(&bars->empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bars->acc_full[b], 1);
-            mbar_init(&bars->acc_empty[b], 128);
+            mbar_init(&bars->acc_empty[b], 2 * kEpiThreads / 32);
         }
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(&bars->tmem_base, kAccCols);
+    cluster_sync_all();                                  // barriers of both CTAs initialised
+    if (warp == 1) tmem_alloc_pair(&bars->tmem_base, kAccCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -229,11 +365,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
     pdl_launch_dependents();
 
     if (warp == 0) {
-        // ---------------- producer ----------------
+        // ---------------- producer (both CTAs) ----------------
         if (lane == 0) {
             bool ok = true, waited = false;
-            int g = 0;   // global k-block counter of this CTA (ring position)
-            for (int tile = blockIdx.x; tile < args.ntiles; tile += gridDim.x) {
+            int g = 0;   // ring position of this CTA
+            for (int tile = first_tile; tile < args.ntiles; tile += tile_step) {
                 const TileCoord c = tile_coord(args, tile);
                 const int nblocks = nkb + c.nslab;
                 for (int i = 0; i < nblocks; ++i, ++g) {
@@ -243,8 +379,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                     const uint32_t xs = smem_u32(st), ws = smem_u32(st + kXBytes), qs = smem_u32(st + kXBytes + kWBytes);
                     if (i < nkb) {
                         mbar_arrive_expect_tx(&bars->full[s], kXBytes + kQBytes);
-                        tma_load_2d(xs, &args.tmX, &bars->full[s], i * kBK, c.n0);
-                        tma_load_2d(qs, &args.tmQ[c.mi], &bars->full[s], i * (kBK / 8), c.m0);
+                        tma_load_2d(xs, &args.tmX, &bars->full[s], i * kBK, c.n0 + tok_off);
+                        tma_load_2d(qs, &args.tmQ[c.mi], &bars->full[s], i * (kBK / 8), c.m0 + row_off);
                     } else {
                         if (!waited && args.wait_dep) {   // R is complete
                             pdl_wait();
@@ -252,63 +388,88 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                         }
                         const int j = i - nkb;
                         mbar_arrive_expect_tx(&bars->full[s], kXBytes + kWBytes);
-                        tma_load_2d(xs, &args.tmR, &bars->full[s], j * kBK, c.n0);
-                        tma_load_2d(ws, &args.tmA[c.mi], &bars->full[s], j * kBK, c.m0);
+                        tma_load_2d(xs, &args.tmR, &bars->full[s], j * kBK, c.n0 + tok_off);
+                        tma_load_2d(ws, &args.tmA[c.mi], &bars->full[s], j * kBK, c.m0 + row_off);
                     }
                 }
             }
+            // the leader's commits for the last stages land here before this CTA may exit
+            for (int p = (g > kGemmStages ? g - kGemmStages : 0); p < g && ok; ++p)
+                ok = mbar_wait(&bars->empty[p % kGemmStages], (p / kGemmStages) & 1, args.status);
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            constexpr uint32_t idesc = f16_idesc(kBM, kBN);
+        // ---------------- MMA issuer (leader CTA) ----------------
+        if (crank == 0 && lane == 0) {
+            constexpr uint32_t idesc = f16_idesc(kPairM, kBN);
+            constexpr uint64_t kStageDesc = (uint64_t)(kStageBytesG >> 4);   // descriptor step per stage
+            // loop-invariant addresses: everything per stage is base + stage * step
+            const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(gsm + kXBytes));   // W of stage 0
+            const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(gsm));             // X of stage 0
+            const uint32_t empty_l0 = smem_u32(&bars->empty[0]);
+            const uint32_t empty_p0 = cluster_addr(&bars->empty[0], 1);
+            const uint32_t dq0 = smem_u32(&bars->dq[0]);
             bool ok = true;
-            int g = 0, tl = 0;
-            for (int tile = blockIdx.x; tile < args.ntiles; tile += gridDim.x, ++tl) {
+            int tl = 0;
+            int s = 0;              // stage of the current ring position
+            uint32_t ph = 0;        // its phase parity
+            // The barrier of the next ring position is probed (non-blocking) while
+            // this position's MMAs are issued, so the shared-memory round trip of
+            // the probe does not idle the tensor pipe.
+            bool next_ready = false;
+            for (int tile = first_tile; tile < args.ntiles; tile += tile_step, ++tl) {
                 const TileCoord c = tile_coord(args, tile);
                 const int nblocks = nkb + c.nslab;
                 const int buf = tl & 1;
-                if (tl >= 2 && ok) ok = mbar_wait(&bars->acc_empty[buf], ((tl >> 1) - 1) & 1, args.status);
+                if (tl >= 2 && ok) ok = mbar_wait_cluster(&bars->acc_empty[buf], ((tl >> 1) - 1) & 1, args.status);
                 tc_fence_after();
                 const uint32_t dacc = tmem + (uint32_t)(buf * kBN);
-                for (int i = 0; i < nblocks; ++i, ++g) {
-                    const int s = g % kGemmStages;
-                    const uint32_t par = (g / kGemmStages) & 1;
-                    // dq completes once per block (slab blocks too, after their TMA landed)
-                    if (ok) ok = mbar_wait(&bars->dq[s], par, args.status);
+                for (int i = 0; i < nblocks; ++i) {
+                    // both CTAs' w_hat written and TMA landed (slab blocks: TMA only)
+                    if (!next_ready && ok) ok = mbar_wait_cluster(&bars->dq[s], ph, args.status);
                     tc_fence_after();
-                    unsigned char* st = gsm + s * kStageBytesG;
-                    const uint32_t xs = smem_u32(st), ws = smem_u32(st + kXBytes);
-#pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k) {
-                        const uint64_t ad = sw128_kmajor_desc(ws + k * 32);
-                        const uint64_t bd = sw128_kmajor_desc(xs + k * 32);
-                        umma_f16(dacc, ad, bd, idesc, (i > 0 || k > 0) ? 1u : 0u);
-                    }
-                    umma_commit(&bars->empty[s]);   // frees the stage once these MMAs complete
+                    const int sn = (s + 1 == kGemmStages) ? 0 : s + 1;
+                    const uint32_t phn = (s + 1 == kGemmStages) ? (ph ^ 1u) : ph;
+                    // frees stage s in both CTAs once these MMAs complete; probes the next
+                    // position (all earlier phases of its barrier completed and were
+                    // waited on, so the parity probe cannot see a stale phase)
+                    next_ready = umma_kblock_pair_probe(dacc, adesc0 + (uint64_t)s * kStageDesc,
+                                                        bdesc0 + (uint64_t)s * kStageDesc, idesc, i > 0 ? 1u : 0u,
+                                                        empty_l0 + 8u * (uint32_t)s, empty_p0 + 8u * (uint32_t)s,
+                                                        dq0 + 8u * (uint32_t)sn, phn) != 0;
+                    s = sn;
+                    ph = phn;
                 }
-                umma_commit(&bars->acc_full[buf]);  // this tile's accumulator is complete
+                umma_commit_pair(smem_u32(&bars->acc_full[buf]));
+                umma_commit_pair(cluster_addr(&bars->acc_full[buf], 1));
             }
+            // both epilogues' releases of the last buffers land before the pair may exit
+            for (int t = (tl > 2 ? tl - 2 : 0); t < tl && ok; ++t)
+                ok = mbar_wait_cluster(&bars->acc_empty[t & 1], (t >> 1) & 1, args.status);
         }
     } else if (warp < 10) {
-        // ---------------- transform (warps 2..9) ----------------
+        // ---------------- transform (warps 2..9, both CTAs) ----------------
+        // Warps 2-5 take the even ring positions, warps 6-9 the odd ones, so two
+        // k-blocks are converted at once; one thread per W row converts all
+        // 64 k of its row (8 packed words).  With an even number of stages each
+        // stage always belongs to the same warp group, which therefore waits on
+        // every phase of its barriers in order.
         const int tt = threadIdx.x - 64;
         const int row = tt & 127;                      // tile row owned by this thread
-        const int half = tt >> 7;                      // which 32 k of the 64-k block
+        const int par = tt >> 7;                       // ring-position parity of this warp group
         const int ngroups = args.d / 128;
         const uint32_t swz = (uint32_t)(row & 7);
+        const uint32_t hsw = (uint32_t)((row >> 2) & 1);
         bool ok = true;
-        int g = 0;
+        int gbase = 0;                                 // ring position of the tile's first block
         // scale/zero of the current and the next 3 groups (a shift register
         // refilled 4 groups ahead, across tile boundaries)
-        int cur_tile = blockIdx.x;
-        TileCoord cc = tile_coord(args, cur_tile < args.ntiles ? cur_tile : 0);
+        int cur_tile = first_tile;
         int f_tile = cur_tile, f_grp = 0;              // next group to fetch
-        TileCoord fc = cc;
+        TileCoord fc = tile_coord(args, cur_tile < args.ntiles ? cur_tile : 0);
         auto fetch = [&]() -> uint32_t {
             uint32_t v = 0;
             if (f_tile < args.ntiles) {
-                const int orow = fc.m0 + row;
+                const int orow = fc.m0 + row_off + row;
                 const PrefillModule& FM = args.mod[fc.mi];
                 if (orow < FM.O) {
                     const int64_t o = (int64_t)orow * ngroups + f_grp;
@@ -316,75 +477,73 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                 }
                 if (++f_grp == ngroups) {
                     f_grp = 0;
-                    f_tile += gridDim.x;
+                    f_tile += tile_step;
                     if (f_tile < args.ntiles) fc = tile_coord(args, f_tile);
                 }
             }
             return v;
         };
         uint32_t sz0 = fetch(), sz1 = fetch(), sz2 = fetch(), sz3 = fetch();
-        for (; cur_tile < args.ntiles; cur_tile += gridDim.x) {
-            cc = tile_coord(args, cur_tile);
+        for (; cur_tile < args.ntiles; cur_tile += tile_step) {
+            const TileCoord cc = tile_coord(args, cur_tile);
             const int nblocks = nkb + cc.nslab;
-            for (int i = 0; i < nkb; ++i, ++g) {
+            // nkb is even, so block i of the tile (group i/2) is ours when (gbase + i) % 2 == par
+            for (int i = (par ^ gbase) & 1; i < nblocks; i += 2) {
+                const int g = gbase + i;
                 const int s = g % kGemmStages;
                 if (ok) ok = mbar_wait(&bars->full[s], (g / kGemmStages) & 1, args.status);
-                unsigned char* st = gsm + s * kStageBytesG;
-                // 32-byte-swizzled INT4 rows: 16-byte half h of row r sits at r*32 + ((h ^ (r>>2)&1) << 4)
-                const unsigned char* qrow = st + kXBytes + kWBytes + row * 32;
-                const uint32_t hsw = (uint32_t)((row >> 2) & 1);
-                const uint4 q0 = *reinterpret_cast<const uint4*>(qrow + (((uint32_t)half ^ hsw) << 4));
-                const uint32_t sz = sz0;                             // group i/2
-                if ((i & 1) == 1) {                                  // group done: shift, fetch 4 ahead
+                if (i < nkb) {
+                    unsigned char* st = gsm + s * kStageBytesG;
+                    // 32-byte-swizzled INT4 rows: 16-byte half h of row r sits at r*32 + ((h ^ (r>>2)&1) << 4)
+                    const unsigned char* qrow = st + kXBytes + kWBytes + row * 32;
+                    const uint4 qa = *reinterpret_cast<const uint4*>(qrow + (hsw << 4));
+                    const uint4 qb = *reinterpret_cast<const uint4*>(qrow + ((hsw ^ 1u) << 4));
+                    const uint32_t sz = sz0;                         // group i/2 (one block of it is ours)
                     sz0 = sz1;
                     sz1 = sz2;
                     sz2 = sz3;
                     sz3 = fetch();
-                }
-                const __half2 sc = __half2half2(__ushort_as_half((unsigned short)(sz & 0xffffu)));
-                const __half2 bz = __half2half2(__ushort_as_half((unsigned short)(0x6400u | ((sz >> 16) & 0xffu))));
-                const uint32_t words[4] = {q0.x, q0.y, q0.z, q0.w};
-                // row `row` of the W tile: 8 chunks of 16 B (8 fp16 in k order), chunk c at c ^ (row % 8)
-                unsigned char* wrow = st + kXBytes + (row >> 3) * 1024 + (row & 7) * 128;
+                    const __half2 sc = __half2half2(__ushort_as_half((unsigned short)(sz & 0xffffu)));
+                    const __half2 bz = __half2half2(__ushort_as_half((unsigned short)(0x6400u | ((sz >> 16) & 0xffu))));
+                    const uint32_t words[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+                    // row `row` of the W tile: 8 chunks of 16 B (8 fp16 in k order), chunk c at c ^ (row % 8)
+                    unsigned char* wrow = st + kXBytes + (row >> 3) * 1024 + (row & 7) * 128;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int c = half * 4 + j;
-                    __half2 p[4];
-                    dequant_word(words[j], bz, sc, p);   // pairs (0,4) (1,5) (2,6) (3,7), exact w_hat
-                    const uint32_t u0 = h2_as_u32(p[0]), u1 = h2_as_u32(p[1]), u2 = h2_as_u32(p[2]), u3 = h2_as_u32(p[3]);
-                    uint4 o;
-                    o.x = pair_lo(u0, u1);   // (0,1)
-                    o.y = pair_lo(u2, u3);   // (2,3)
-                    o.z = pair_hi(u0, u1);   // (4,5)
-                    o.w = pair_hi(u2, u3);   // (6,7)
-                    *reinterpret_cast<uint4*>(wrow + (((uint32_t)c ^ swz) << 4)) = o;
+                    for (int c = 0; c < 8; ++c) {
+                        __half2 p[4];
+                        dequant_word(words[c], bz, sc, p);   // pairs (0,4) (1,5) (2,6) (3,7), exact w_hat
+                        const uint32_t u0 = h2_as_u32(p[0]), u1 = h2_as_u32(p[1]), u2 = h2_as_u32(p[2]), u3 = h2_as_u32(p[3]);
+                        uint4 o;
+                        o.x = pair_lo(u0, u1);   // (0,1)
+                        o.y = pair_lo(u2, u3);   // (2,3)
+                        o.z = pair_hi(u0, u1);   // (4,5)
+                        o.w = pair_hi(u2, u3);   // (6,7)
+                        *reinterpret_cast<uint4*>(wrow + (((uint32_t)c ^ swz) << 4)) = o;
+                    }
+                    fence_proxy_async_smem();   // generic-proxy writes visible to the tensor cores
                 }
-                fence_proxy_async_smem();   // generic-proxy writes visible to the tensor cores
-                mbar_arrive(&bars->dq[s]);
+                // slab blocks are filled by TMA alone; they are still reported (after
+                // the TMA landed) so the leader's dq phases follow the ring position
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(cluster_addr(&bars->dq[s], 0));   // one arrival per warp
             }
-            // slab blocks are filled by TMA alone; still advance dq once per block
-            // (after the TMA landed) so its phases follow the ring position
-            for (int i = nkb; i < nblocks; ++i, ++g) {
-                const int s = g % kGemmStages;
-                if (ok) ok = mbar_wait(&bars->full[s], (g / kGemmStages) & 1, args.status);
-                mbar_arrive(&bars->dq[s]);
-            }
+            gbase += nblocks;
         }
     } else {
-        // ---------------- epilogue (warps 10..13) ----------------
-        // Each 32-token chunk of the accumulator is transposed through shared
-        // memory ([32 tokens][128 rows] fp16) and written by one TMA store,
-        // which clips rows >= O and tokens >= T.  Two staging buffers: a buffer
-        // is rewritten only after the store issued from it two chunks earlier
-        // has finished reading it.
+        // ---------------- epilogue (warps 10..13, both CTAs) ----------------
+        // Each 32-token chunk of this CTA's accumulator is transposed through
+        // shared memory ([32 tokens][128 rows] fp16) and written by one TMA
+        // store, which clips rows >= O and tokens >= T.  A staging buffer is
+        // rewritten only after the store issued from it has finished reading it.
         const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;
         const bool leader = (warp == 10 && lane == 0);
         bool ok = true;
         int tl = 0, chunk = 0;
-        for (int tile = blockIdx.x; tile < args.ntiles; tile += gridDim.x, ++tl) {
+        for (int tile = first_tile; tile < args.ntiles; tile += tile_step, ++tl) {
             const TileCoord c = tile_coord(args, tile);
             const int buf = tl & 1;
+            const int orow0 = c.m0 + row_off;
             if (ok) ok = mbar_wait(&bars->acc_full[buf], (tl >> 1) & 1, args.status);
             tc_fence_after();
             const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN);
@@ -392,29 +551,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
             for (int ch = 0; ch < kBN / kEpiChunk; ++ch, ++chunk) {
                 uint32_t v[32];
                 tmem_ld32(tacc + ch * kEpiChunk, v);
-                unsigned char* sb = epi + (chunk & 1) * kEpiBytes;
-                if (leader) bulk_wait_read<1>();          // the store from this buffer is done reading
-                named_barrier_sync(1, 128);
+                unsigned char* sb = epi + (chunk % kEpiBufs) * kEpiBytes;
+                if (leader) bulk_wait_read<kEpiBufs - 1>();   // the store from this buffer is done reading
+                named_barrier_sync(1, kEpiThreads);
                 __half* col = reinterpret_cast<__half*>(sb) + row;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) col[j * kBM] = __float2half_rn(__uint_as_float(v[j]));
                 fence_proxy_async_smem();
-                named_barrier_sync(1, 128);
-                if (leader) {
-                    tma_store_2d(&args.tmY[c.mi], smem_u32(sb), c.m0, c.n0 + ch * kEpiChunk);
+                named_barrier_sync(1, kEpiThreads);
+                const int tok0 = c.n0 + ch * kEpiChunk;
+                if (leader && orow0 < args.mod[c.mi].O && tok0 < args.T) {
+                    tma_store_2d(&args.tmY[c.mi], smem_u32(sb), orow0, tok0);
                     bulk_commit();
                 }
             }
             tc_fence_before();
-            mbar_arrive(&bars->acc_empty[buf]);        // buffer may be overwritten
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(cluster_addr(&bars->acc_empty[buf], 0));   // buffer may be overwritten
         }
         if (leader) bulk_wait_all();
     }
     // the R kernel is complete before this grid is (even if no tile read R)
     if (args.wait_dep) pdl_wait();
     tc_fence_before();
-    __syncthreads();
-    if (warp == 1) tmem_dealloc(tmem, kAccCols);
+    __syncwarp();
+    cluster_sync_all();                                  // no arrivals or MMA reads into either CTA remain
+    if (warp == 1) tmem_dealloc_pair(tmem, kAccCols);
 }
 
 // ---------------------------------------------------------------------------
@@ -566,7 +728,35 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
 }
 
 static size_t gemm_smem_bytes() {
-    return (size_t)kGemmStages * kStageBytesG + 2 * kEpiBytes + sizeof(GemmBarriers) + 1024;
+    return (size_t)kGemmStages * kStageBytesG + kEpiBufs * kEpiBytes + sizeof(GemmBarriers) + 1024;
+}
+// CTA pairs of the GEMM that can be resident at once (one CTA per SM).
+static int gemm_max_pairs(int num_sms) {
+    static int cached_dev = -1, cached = 0;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev == cached_dev) return cached;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(num_sms / 2 * 2));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = gemm_smem_bytes();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, (const void*)corrected_gemm_kernel, &cfg) != cudaSuccess ||
+        clusters <= 0) {
+        cudaGetLastError();
+        clusters = num_sms / 2;
+    }
+    if (std::getenv("GLOWQ_VERBOSE")) std::fprintf(stderr, "glowq prefill: %d resident CTA pairs\n", clusters);
+    cached_dev = dev;
+    cached = clusters;
+    return cached;
 }
 static size_t rproj_smem_bytes(int rn) { return (size_t)kRStages * rproj_stage_bytes(rn) + sizeof(RprojBarriers) + 1024; }
 
@@ -632,10 +822,10 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     PrefillArgs* a = new PrefillArgs;
     std::memset(a, 0, sizeof(*a));
     bool ok = make_map(&a->tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, (uint64_t)d, (uint64_t)T, (uint64_t)d * 2, kBK,
-                       kBN, CU_TENSOR_MAP_SWIZZLE_128B);
+                       kHalfN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (use_r)
         ok = ok && make_map(&a->tmR, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, R, (uint64_t)r, (uint64_t)T, (uint64_t)r * 2, kBK,
-                            kBN, CU_TENSOR_MAP_SWIZZLE_128B);
+                            kHalfN, CU_TENSOR_MAP_SWIZZLE_128B);
     int mtiles = 0;
     for (int i = 0; i < m && ok; ++i) {
         const ModuleView& mv = mods[i];
@@ -654,7 +844,7 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
         a->mod[i].O = (int)mv.O;
         a->mod[i].mtile_begin = mtiles;
         a->mod[i].has_A = has_A ? 1 : 0;
-        mtiles += (int)((mv.O + kBM - 1) / kBM);
+        mtiles += (int)((mv.O + kPairM - 1) / kPairM);
     }
     if (!ok) {
         delete a;
@@ -670,12 +860,26 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     const int64_t ntiles = (int64_t)mtiles * a->ntiles_n;
     a->ntiles = (int)ntiles;
     void* args[] = {(void*)a};
-    // persistent grid: one CTA per SM (fewer if there are fewer tiles)
-    const int64_t grid = ntiles < num_sms ? ntiles : num_sms;
+    // persistent grid: as many CTA pairs as fit at once (fewer if there are fewer tiles)
+    const int64_t pairs = ntiles < gemm_max_pairs(num_sms) ? ntiles : gemm_max_pairs(num_sms);
     cudaError_t e = cudaSuccess;
-    if (grid > 0)
-        e = launch_with((const void*)corrected_gemm_kernel, dim3((unsigned)grid), dim3(kGemmThreads), gemm_smem_bytes(),
-                        st, use_r, args);
+    if (pairs > 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(2 * pairs));
+        cfg.blockDim = dim3(kGemmThreads);
+        cfg.dynamicSmemBytes = gemm_smem_bytes();
+        cfg.stream = st;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = use_r ? 2 : 1;
+        e = cudaLaunchKernelExC(&cfg, (const void*)corrected_gemm_kernel, args);
+    }
     delete a;
     return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
 }
