@@ -33,9 +33,12 @@ static int device_sm_count() {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// fp32 partial sums of R = X B^T: split along d (decode: up to 32 slices;
+// prefill: up to 8 slices when the token tiles alone would not fill the GPU)
 static size_t workspace_partial_bytes(int64_t T, int32_t r) {
-    if (r <= 0 || T <= 0 || T > kDecodeMaxTokens) return 0;
-    return align_up(decode_partial_bytes(T, r), 256);
+    if (r <= 0 || T <= 0) return 0;
+    if (T <= kDecodeMaxTokens) return align_up(decode_partial_bytes(T, r), 256);
+    return align_up(prefill_partial_bytes(T, r), 256);
 }
 
 static size_t workspace_solo_R_bytes(int64_t T, int32_t r) {
@@ -88,8 +91,9 @@ static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d,
         return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
     }
     (void)any_A;
-    (void)ws_bytes;
-    return prefill_group_forward(hm, m, (int)d, use_r ? B : nullptr, use_r ? r : 0, X, T, R,
+    float* partial = (use_r && workspace && ws_bytes >= workspace_partial_bytes(T, r))
+                         ? reinterpret_cast<float*>(workspace) : nullptr;
+    return prefill_group_forward(hm, m, (int)d, use_r ? B : nullptr, use_r ? r : 0, X, T, R, partial,
                                  device_sm_count(), st);
 }
 

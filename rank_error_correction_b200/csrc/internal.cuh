@@ -47,7 +47,11 @@ EncodeTiledFn encode_fn();
 // 2-D row-major tensor [outer][inner], row pitch `pitch` bytes, box {box_inner, box_outer}.
 bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
               uint64_t pitch, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
+// `partial`: scratch of prefill_partial_bytes(T, r) for the split R projection
+// (nullptr: one slice of d per CTA, R written directly).
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r,
-                                   const uint16_t* X, int64_t T, uint16_t* R, int num_sms, cudaStream_t st);
+                                   const uint16_t* X, int64_t T, uint16_t* R, float* partial, int num_sms,
+                                   cudaStream_t st);
+size_t prefill_partial_bytes(int64_t T, int r);
 
 }  // namespace glowq

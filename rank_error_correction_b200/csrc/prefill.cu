@@ -580,16 +580,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
 }
 
 // ---------------------------------------------------------------------------
-// R = X B^T on the tensor cores: one 128-token tile per CTA, N = r (padded to 16)
+// R = X B^T on the tensor cores: CTA (x, y) computes tokens [128x, 128x+128)
+// over the y-th of `chunks` slices of d (N = r padded to 16).  With one chunk
+// it writes R in fp16; otherwise fp32 partial sums partial[y][t][j], which
+// rproj_sum_kernel adds in ascending y (a fixed order: R is deterministic).
+// Splitting d keeps ~all SMs busy when T / 128 is far below the SM count.
 // ---------------------------------------------------------------------------
 constexpr int kRStages = 4;
 constexpr int kRThreads = 192;
+constexpr int kRMaxChunks = 8;
 
 struct RprojArgs {
     CUtensorMap tmX;   // X [T][d], box {64, 128}, SW128
     CUtensorMap tmB;   // B [r][d], box {64, rn}, SW128
-    __half* R;         // T x r
-    int d, T, r, rn;
+    __half* R;         // T x r (chunks == 1)
+    float* partial;    // chunks x T x r (chunks > 1)
+    int d, T, r, rn, chunks;
     unsigned int* status;
 };
 
@@ -614,7 +620,10 @@ __global__ void __launch_bounds__(kRThreads, 1) rproj_tc_kernel(const __grid_con
     RprojBarriers* bars = reinterpret_cast<RprojBarriers*>(rsm + kRStages * sbytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int t0 = blockIdx.x * 128;
-    const int nkb = args.d / kBK;
+    const int nkb_all = args.d / kBK;
+    const int kb0 = (int)((int64_t)blockIdx.y * nkb_all / args.chunks);
+    const int kb1 = (int)((int64_t)(blockIdx.y + 1) * nkb_all / args.chunks);
+    const int nkb = kb1 - kb0;
     const uint32_t ncols = tmem_cols_for(args.rn);
 
     if (threadIdx.x == 0) {
@@ -642,8 +651,8 @@ __global__ void __launch_bounds__(kRThreads, 1) rproj_tc_kernel(const __grid_con
                 if (i >= kRStages && ok) ok = mbar_wait(&bars->empty[s], ((i / kRStages) - 1) & 1, args.status);
                 unsigned char* st = rsm + s * sbytes;
                 mbar_arrive_expect_tx(&bars->full[s], bytes);
-                tma_load_2d(smem_u32(st), &args.tmX, &bars->full[s], i * kBK, t0);
-                tma_load_2d(smem_u32(st + 128 * kBK * 2), &args.tmB, &bars->full[s], i * kBK, 0);
+                tma_load_2d(smem_u32(st), &args.tmX, &bars->full[s], (kb0 + i) * kBK, t0);
+                tma_load_2d(smem_u32(st + 128 * kBK * 2), &args.tmB, &bars->full[s], (kb0 + i) * kBK, 0);
             }
         }
     } else if (warp == 1) {
@@ -675,7 +684,20 @@ __global__ void __launch_bounds__(kRThreads, 1) rproj_tc_kernel(const __grid_con
         for (int c = 0; c < args.rn; c += 32) {
             uint32_t v[32];
             tmem_ld32(tl + c, v);
-            if (tok < args.T) {
+            if (tok < args.T && args.chunks > 1) {
+                float* dst = args.partial + ((int64_t)blockIdx.y * args.T + tok) * r + c;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    if (c + j < r) {   // r % 8 == 0: 4-column chunks are all-or-nothing
+                        float4 o;
+                        o.x = __uint_as_float(v[j]);
+                        o.y = __uint_as_float(v[j + 1]);
+                        o.z = __uint_as_float(v[j + 2]);
+                        o.w = __uint_as_float(v[j + 3]);
+                        *reinterpret_cast<float4*>(dst + j) = o;
+                    }
+                }
+            } else if (tok < args.T) {
                 __half* dst = args.R + (int64_t)tok * r + c;
 #pragma unroll
                 for (int j = 0; j < 32; j += 8) {
@@ -695,6 +717,38 @@ __global__ void __launch_bounds__(kRThreads, 1) rproj_tc_kernel(const __grid_con
     __syncthreads();
     if (warp == 1) tmem_dealloc(tmem, ncols);
 }
+
+// R[i] = fp16_RN(sum_y partial[y][i]) in ascending y, four elements per thread.
+__global__ void __launch_bounds__(256) rproj_sum_kernel(const float4* __restrict__ partial, int chunks, int n4,
+                                                         uint2* __restrict__ R) {
+    pdl_launch_dependents();
+    pdl_wait();                 // partial sums complete
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n4) return;
+    float4 acc = partial[i];
+    for (int y = 1; y < chunks; ++y) {
+        const float4 v = partial[(int64_t)y * n4 + i];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+    }
+    uint2 o;
+    o.x = h2_as_u32(__floats2half2_rn(acc.x, acc.y));
+    o.y = h2_as_u32(__floats2half2_rn(acc.z, acc.w));
+    R[i] = o;
+}
+
+// Number of d slices of the prefill R projection: enough CTAs to cover the
+// SMs, at most kRMaxChunks, at least 4 k-blocks per slice.
+int prefill_r_chunks(int64_t T, int d, int num_sms) {
+    const int ntok = (int)((T + 127) / 128);
+    int c = num_sms / (ntok > 0 ? ntok : 1);
+    if (c > kRMaxChunks) c = kRMaxChunks;
+    if (c > d / kBK / 4) c = d / kBK / 4;
+    return c < 1 ? 1 : c;
+}
+size_t prefill_partial_bytes(int64_t T, int r) { return (size_t)kRMaxChunks * (size_t)T * (size_t)r * sizeof(float); }
 
 // ---------------------------------------------------------------------------
 // Host side: tensor maps and launches
@@ -776,7 +830,7 @@ static cudaError_t launch_with(const void* fn, dim3 grid, dim3 block, size_t sme
 }
 
 cudaError_t launch_rproj_prefill(const uint16_t* X, const uint16_t* B, int64_t T, int d, int r, uint16_t* R,
-                                 cudaStream_t st) {
+                                 float* partial, int num_sms, cudaStream_t st) {
     static bool opted = false;
     if (!opted) {
         cudaError_t e = cudaFuncSetAttribute((const void*)rproj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -793,24 +847,33 @@ cudaError_t launch_rproj_prefill(const uint16_t* X, const uint16_t* B, int64_t T
     if (!make_map(&a.tmB, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, B, (uint64_t)d, (uint64_t)r, (uint64_t)d * 2, kBK,
                   (uint32_t)rn, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
+    const int chunks = partial ? prefill_r_chunks(T, d, num_sms) : 1;
     a.R = reinterpret_cast<__half*>(R);
+    a.partial = partial;
     a.d = d;
     a.T = (int)T;
     a.r = r;
     a.rn = rn;
+    a.chunks = chunks;
     a.status = device_status_ptr();
     void* args[] = {(void*)&a};
-    return launch_with((const void*)rproj_tc_kernel, dim3((unsigned)((T + 127) / 128)), dim3(kRThreads),
-                       rproj_smem_bytes(rn), st, true, args);
+    cudaError_t e = launch_with((const void*)rproj_tc_kernel, dim3((unsigned)((T + 127) / 128), (unsigned)chunks),
+                                dim3(kRThreads), rproj_smem_bytes(rn), st, true, args);
+    if (e != cudaSuccess || chunks == 1) return e;
+    const float4* p4 = reinterpret_cast<const float4*>(partial);
+    const int n4 = (int)(T * r / 4);
+    uint2* R4 = reinterpret_cast<uint2*>(R);
+    void* a2[] = {(void*)&p4, (void*)&chunks, (void*)&n4, (void*)&R4};
+    return launch_with((const void*)rproj_sum_kernel, dim3((unsigned)((n4 + 255) / 256)), dim3(256), 0, st, true, a2);
 }
 
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r, const uint16_t* X,
-                                   int64_t T, uint16_t* R, int num_sms, cudaStream_t st) {
+                                   int64_t T, uint16_t* R, float* partial, int num_sms, cudaStream_t st) {
     if (T > ((int64_t)1 << 30)) return GLOWQ_ERR_SHAPE;
     if (!encode_fn()) return GLOWQ_ERR_CUDA;
     const bool use_r = r > 0 && B != nullptr;
     if (use_r) {
-        if (launch_rproj_prefill(X, B, T, d, r, R, st) != cudaSuccess) return GLOWQ_ERR_CUDA;
+        if (launch_rproj_prefill(X, B, T, d, r, R, partial, num_sms, st) != cudaSuccess) return GLOWQ_ERR_CUDA;
     }
     static bool opted = false;
     if (!opted) {
