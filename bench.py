@@ -435,7 +435,7 @@ def main():
     value = world * T * args.steps / (total_ms / 1e3)
     qkv_bytes = group_bytes(QKV_OUTS, D, R_RANK, T)
     achieved = qkv_bytes / (res["qkv_ms"] * 1e-3) / 1e9
-    launches_per_step = 3 + 3          # (rproj_partial, rproj_reduce, corrected_gemv) x 2 calls
+    launches_per_step = 2 + 2          # (rproj_cluster, corrected_gemv) x 2 calls
     e2e_ms, h2d, d2h, _ = time_e2e(T, args.steps, device, res["reps"], res["io"])
 
     extra = []

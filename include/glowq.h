@@ -110,12 +110,12 @@ GLOWQ_API glowq_status glowq_dequant_int4(const uint32_t* qweight, const uint16_
                                 int32_t group_size, uint16_t* W_deq, void* stream);
 
 /*
- * Bytes of device scratch the forward calls need for T tokens at rank r: the
- * fp32 partial sums of R = X B^T split along d (up to 32 slices for T <= 16,
- * up to 8 for larger T; they are added in a fixed order, so R does not depend
- * on timing), plus the solo call's R.  0 when r == 0.  The caller allocates it
- * once and may reuse it across calls issued in order on one stream; calls that
- * may overlap need separate workspaces.
+ * Bytes of device scratch the forward calls need for T tokens at rank r: for
+ * T > 16 the fp32 partial sums of R = X B^T split along d into up to 8 slices
+ * (added in a fixed order, so R does not depend on timing), plus the solo
+ * call's R.  0 when r == 0.  The caller allocates it once and may reuse it
+ * across calls issued in order on one stream; calls that may overlap need
+ * separate workspaces.
  */
 GLOWQ_API size_t glowq_workspace_bytes(int64_t T, int32_t r);
 

@@ -33,11 +33,11 @@ static int device_sm_count() {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// fp32 partial sums of R = X B^T: split along d (decode: up to 32 slices;
-// prefill: up to 8 slices when the token tiles alone would not fill the GPU)
+// fp32 partial sums of R = X B^T for T > 16 (split along d into up to 8
+// slices when the token tiles alone would not fill the GPU); the decode path
+// reduces its partial sums on chip.
 static size_t workspace_partial_bytes(int64_t T, int32_t r) {
-    if (r <= 0 || T <= 0) return 0;
-    if (T <= kDecodeMaxTokens) return align_up(decode_partial_bytes(T, r), 256);
+    if (r <= 0 || T <= kDecodeMaxTokens) return 0;
     return align_up(prefill_partial_bytes(T, r), 256);
 }
 
@@ -83,8 +83,7 @@ static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d,
     const bool use_r = r > 0;
     if (T <= kDecodeMaxTokens) {
         if (use_r) {
-            float* partial = reinterpret_cast<float*>(workspace);
-            cudaError_t e = launch_rproj_decode(X, B, (int)T, (int)d, r, partial, R, st);
+            cudaError_t e = launch_rproj_decode(X, B, (int)T, (int)d, r, R, st);
             if (e != cudaSuccess) return GLOWQ_ERR_CUDA;
         }
         cudaError_t e = launch_gemv_decode(hm, m, (int)d, (int)T, use_r ? r : 0, X, R, use_r, device_sm_count(), st);

@@ -6,30 +6,29 @@
 //
 // At T <= 16 the layer is a weight-streaming GEMV: every INT4 weight byte is
 // read once from HBM and meets at most 16 tokens, so the kernels are HBM-bound.
-// Design:
-//   * rproj_partial / rproj_reduce: R = X B^T split along d over up to 32 CTAs
-//     (fp32 partial sums in the caller's workspace, reduced in a fixed order so
-//     the result is deterministic), rounded to fp16.
+// One call is two launches chained with programmatic dependent launch:
+//   * rproj_cluster: R = X B^T by one cluster of 8 CTAs splitting d; the
+//     partial sums meet on chip in a fixed order (deterministic), R is rounded
+//     to fp16 once and written to the caller's R buffer.
 //   * corrected_gemv: one launch over the stacked rows of all modules of the
-//     group.  128-bit streaming loads of the packed weights (4 groups of 128
-//     in flight per warp, issued before anything else); nibbles unpacked in
-//     registers to the exact fp16 integers (q - z) (half2 bias trick); the
-//     multiply-accumulate runs on the tensor cores with register operands
-//     (mma.sync m16n8k16, fp32 accumulate) so the ALU cost per weight stays
-//     below two instructions; the group scale s is applied in fp32 to each
-//     128-group's dot product.  The k order inside an MMA is permuted
+//     group.  Each warp streams its 16 rows of packed weights with 2-D TMA
+//     boxes into a private ring of mbarrier-tracked stages, issued before the
+//     wait on the preceding kernel (weights and scales are static), so the
+//     stream overlaps the projection.  Nibbles become the exact fp16 values
+//     64 + q in one LOP3 per pair; the multiply-accumulate runs on the tensor
+//     cores with register operands (mma.sync m16n8k16, fp32 accumulate) and
+//     each 128-group's dot product is finished in fp32 as
+//     s * (D - (64 + z) * sum_k x_k).  The k order inside an MMA is permuted
 //     identically on both operands (a permutation of the contraction index
-//     leaves the dot product unchanged) so that packed words map straight onto
-//     fragments.  Activations and scales/zeros sit in shared memory; d is
-//     split across a thread-block cluster whose partial sums meet in
-//     distributed shared memory; the rank-r correction A_i R is one more short
-//     MMA slab on the same fp32 accumulators, after a programmatic-dependent-
-//     launch wait on the R kernels, so the weight stream overlaps the
-//     projection.
-//   * Numerics: the products (q - z) x are exact; each group's sum is scaled
-//     by s in fp32, i.e. the effective weight is the exact (q - z) s rather
-//     than its fp16 rounding (a difference of at most 2^-12 relative per
-//     weight, far inside the parity bar).
+//     leaves the dot product unchanged) so packed words map straight onto
+//     fragments.  d may be split inside the CTA or across a thread-block
+//     cluster whose partial sums meet in distributed shared memory; the
+//     rank-r correction A_i R is one more short MMA slab on the same fp32
+//     accumulators.
+//   * Numerics: the products (64 + q) x are exact in fp32 accumulation up to
+//     rounding of the sums; the effective weight is the exact (q - z) s rather
+//     than its fp16 rounding (at most 2^-12 relative per weight, far inside the
+//     parity bar).
 #include <cstdio>
 #include <cstdlib>
 
@@ -39,76 +38,119 @@
 namespace glowq {
 
 
-constexpr int kRprojMaxChunks = 32;
 
 // ---------------------------------------------------------------------------
-// R = X B^T, split along d.  Block: ceil(r/16) warps, warp w owns B rows
-// 16w .. 16w+15; block kc owns a slice of d in steps of 32.
-// partial[kc][t][j] (fp32).
+// R = X B^T for T <= 16 in one launch.  A cluster of kRcCtas CTAs splits d
+// (CTA c takes the c-th slice of the 32-wide k steps).  Inside a CTA, warp w
+// takes B rows 16*(w % nrb) .. +15 (nrb = ceil(r/16) row blocks) and every kl-th
+// k step of the slice (kl = 16 / nrb k-lanes), with two steps' loads in flight.
+// Partial sums meet in a fixed order: k-lanes in shared memory, then the CTAs
+// of the cluster through distributed shared memory (ascending rank), so R does
+// not depend on timing.  R is rounded to fp16 once.
 // ---------------------------------------------------------------------------
-template <int NT>
-__global__ void __launch_bounds__(512) rproj_partial_kernel(const __half* __restrict__ X,
-                                                             const __half* __restrict__ B, int T, int d,
-                                                             int r, int chunks, float* __restrict__ partial) {
-    pdl_launch_dependents();    // the next kernels may start their own prologues
-    pdl_wait();                 // X may come from the previous kernel in the stream
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int j0 = warp * 16 + g, j1 = j0 + 8;
-    const int kc = blockIdx.x;
-    const int nsteps = d / 32;
-    const int s0 = (int)((int64_t)kc * nsteps / chunks), s1 = (int)((int64_t)(kc + 1) * nsteps / chunks);
-    float acc[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-    const uint4 zero4 = make_uint4(0, 0, 0, 0);
-    for (int st = s0; st < s1; ++st) {
-        const int k = st * 32 + 8 * t;
-        const uint4 blo = (j0 < r) ? ldg_128(B + (int64_t)j0 * d + k) : zero4;
-        const uint4 bhi = (j1 < r) ? ldg_128(B + (int64_t)j1 * d + k) : zero4;
-        uint4 xv[NT];
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int tok = n * 8 + g;
-            xv[n] = (tok < T) ? ldg_128(X + (int64_t)tok * d + k) : zero4;
-        }
-        const uint32_t a0[4] = {blo.x, bhi.x, blo.y, bhi.y};
-        const uint32_t a1[4] = {blo.z, bhi.z, blo.w, bhi.w};
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const uint32_t b0[2] = {xv[n].x, xv[n].y};
-            const uint32_t b1[2] = {xv[n].z, xv[n].w};
-            mma_16816(acc[n], a0, b0);
-            mma_16816(acc[n], a1, b1);
-        }
-    }
-    float* out = partial + (int64_t)kc * T * r;
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-        const int tk = n * 8 + 2 * t;
-        if (j0 < r) {
-            if (tk < T) out[(int64_t)tk * r + j0] = acc[n][0];
-            if (tk + 1 < T) out[(int64_t)(tk + 1) * r + j0] = acc[n][1];
-        }
-        if (j1 < r) {
-            if (tk < T) out[(int64_t)tk * r + j1] = acc[n][2];
-            if (tk + 1 < T) out[(int64_t)(tk + 1) * r + j1] = acc[n][3];
-        }
-    }
+constexpr int kRcCtas = 8;
+constexpr int kRcWarps = 16;
+
+__host__ __device__ inline int rc_row_blocks(int r) { return (r + 15) / 16; }
+// shared memory: per-k-lane partials [kl][8*NT][r] + the CTA partial [8*NT][r] (fp32)
+__host__ __device__ inline int rc_smem_bytes(int r, int nt) {
+    const int nrb = rc_row_blocks(r), kl = kRcWarps / nrb;
+    return (kl + 1) * 8 * nt * r * 4;
 }
 
-// R[t][j] = fp16_RN(sum_kc partial[kc][t][j]) in ascending kc.
-__global__ void __launch_bounds__(256) rproj_reduce_kernel(const float* __restrict__ partial, int chunks,
-                                                            int T, int r, __half* __restrict__ R) {
-    pdl_launch_dependents();    // let the GEMV start streaming weights now
-    pdl_wait();                 // partial sums complete
-    const int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= T * r) return;
-    float acc = 0.f;
-    for (int kc = 0; kc < chunks; ++kc) acc += partial[(int64_t)kc * T * r + i];
-    R[i] = __float2half_rn(acc);
+template <int NT>
+__global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32)
+    rproj_cluster_kernel(const __half* __restrict__ X, const __half* __restrict__ B, int T, int d, int r,
+                         __half* __restrict__ R) {
+    pdl_launch_dependents();    // the GEMV may start streaming weights now
+    pdl_wait();                 // X may come from the previous kernel in the stream
+    extern __shared__ __align__(16) float rc_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int nrb = rc_row_blocks(r), kl = kRcWarps / nrb;
+    const int rb = warp % nrb, kq = warp / nrb;
+    const int TP = 8 * NT;                       // padded token count
+    float* part = rc_smem;                       // [kl][TP][r]
+    float* cpart = rc_smem + kl * TP * r;        // [TP][r]
+    uint32_t crank;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
+    const int nsteps = d / 32;
+    const int s0 = (int)((int64_t)crank * nsteps / kRcCtas), s1 = (int)((int64_t)(crank + 1) * nsteps / kRcCtas);
+    if (kq < kl) {
+        const int j0 = rb * 16 + g, j1 = j0 + 8;
+        float acc[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+        const uint4 zero4 = make_uint4(0, 0, 0, 0);
+        for (int st = s0 + kq; st < s1; st += 2 * kl) {
+            // two k steps per iteration, all loads issued before the MMAs
+            uint4 blo[2], bhi[2], xv[2][NT];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int su = st + u * kl;
+                const bool in = su < s1;
+                const int k = su * 32 + 8 * t;
+                blo[u] = (in && j0 < r) ? ldg_128(B + (int64_t)j0 * d + k) : zero4;
+                bhi[u] = (in && j1 < r) ? ldg_128(B + (int64_t)j1 * d + k) : zero4;
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const int tok = n * 8 + g;
+                    xv[u][n] = (in && tok < T) ? ldg_128(X + (int64_t)tok * d + k) : zero4;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t a0[4] = {blo[u].x, bhi[u].x, blo[u].y, bhi[u].y};
+                const uint32_t a1[4] = {blo[u].z, bhi[u].z, blo[u].w, bhi[u].w};
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const uint32_t b0[2] = {xv[u][n].x, xv[u][n].y};
+                    const uint32_t b1[2] = {xv[u][n].z, xv[u][n].w};
+                    mma_16816(acc[n], a0, b0);
+                    mma_16816(acc[n], a1, b1);
+                }
+            }
+        }
+        float* my = part + kq * TP * r;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int tk = n * 8 + 2 * t;
+            if (j0 < r) {
+                my[tk * r + j0] = acc[n][0];
+                my[(tk + 1) * r + j0] = acc[n][1];
+            }
+            if (j1 < r) {
+                my[tk * r + j1] = acc[n][2];
+                my[(tk + 1) * r + j1] = acc[n][3];
+            }
+        }
+    }
+    __syncthreads();
+    // this CTA's partial: k-lanes in ascending order
+    for (int i = threadIdx.x; i < T * r; i += blockDim.x) {
+        float v = part[i];
+        for (int q = 1; q < kl; ++q) v += part[q * TP * r + i];
+        cpart[i] = v;
+    }
+    // all CTAs' partials are complete and visible in the cluster
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    const uint32_t cbase = (uint32_t)__cvta_generic_to_shared(cpart);
+    for (int i = (int)crank * blockDim.x + threadIdx.x; i < T * r; i += kRcCtas * blockDim.x) {
+        float v = 0.f;
+#pragma unroll
+        for (int c = 0; c < kRcCtas; ++c) {
+            uint32_t ra;
+            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(cbase + 4u * (uint32_t)i), "r"(c));
+            float pv;
+            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pv) : "r"(ra) : "memory");
+            v = (c == 0) ? pv : v + pv;
+        }
+        R[i] = __float2half_rn(v);
+    }
+    // no CTA leaves while another may still read its shared memory
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -581,15 +623,6 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
 // ---------------------------------------------------------------------------
 // Host-side launchers (called from api.cu after validation).
 // ---------------------------------------------------------------------------
-static int rproj_chunks(int d) {
-    const int nsteps = d / 32;
-    return nsteps < kRprojMaxChunks ? nsteps : kRprojMaxChunks;
-}
-
-size_t decode_partial_bytes(int64_t T, int r) {
-    return (size_t)kRprojMaxChunks * (size_t)T * (size_t)r * sizeof(float);
-}
-
 static cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
                              void** args) {
     cudaLaunchConfig_t cfg = {};
@@ -605,22 +638,16 @@ static cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem,
     return cudaLaunchKernelExC(&cfg, fn, args);
 }
 
-// R = X B^T into R (fp16), via fp32 partials in `partial`.
-cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, float* partial,
-                                uint16_t* R, cudaStream_t st) {
-    const int chunks = rproj_chunks(d);
-    const int warps = (r + 15) / 16;
+// R = X B^T into R (fp16) with one cluster of kRcCtas CTAs.
+cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, uint16_t* R,
+                                cudaStream_t st) {
+    const int nt = (T <= 8) ? 1 : 2;
     const __half* Xh = reinterpret_cast<const __half*>(X);
     const __half* Bh = reinterpret_cast<const __half*>(B);
-    void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&chunks, (void*)&partial};
-    const void* fn = (T <= 8) ? (const void*)rproj_partial_kernel<1> : (const void*)rproj_partial_kernel<2>;
-    cudaError_t e = launch_ex(fn, dim3(chunks), dim3(warps * 32), 0, st, true, a1);
-    if (e != cudaSuccess) return e;
     __half* Rh = reinterpret_cast<__half*>(R);
-    const float* pc = partial;
-    void* a2[] = {(void*)&pc, (void*)&chunks, (void*)&T, (void*)&r, (void*)&Rh};
-    const int n = T * r;
-    return launch_ex((const void*)rproj_reduce_kernel, dim3((n + 255) / 256), dim3(256), 0, st, true, a2);
+    void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&Rh};
+    const void* fn = (nt == 1) ? (const void*)rproj_cluster_kernel<1> : (const void*)rproj_cluster_kernel<2>;
+    return launch_ex(fn, dim3(kRcCtas), dim3(kRcWarps * 32), (size_t)rc_smem_bytes(r, nt), st, true, a1);
 }
 
 

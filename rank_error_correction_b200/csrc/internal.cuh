@@ -27,9 +27,9 @@ constexpr int kDecodeMaxTokens = 16;
 unsigned int* device_status_ptr();
 
 // decode.cu
-size_t decode_partial_bytes(int64_t T, int r);
-cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, float* partial,
-                                uint16_t* R, cudaStream_t st);
+// R = X B^T (T <= 16) by one thread-block cluster, written to R in fp16.
+cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, uint16_t* R,
+                                cudaStream_t st);
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
                                const uint16_t* R, bool after_rproj, int num_sms, cudaStream_t st);
 // pack.cu
