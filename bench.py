@@ -266,8 +266,9 @@ def time_e2e(T, steps, device, reps, io):
 MLP_D, MLP_FFN = 4096, 11008
 
 
-def time_prefill(T, steps, warmup, device, n_rep=2, seed=0):
-    """LLaMA-2-7B MLP linears at T tokens: gate/up group + down_proj solo (tcgen05 path)."""
+def time_prefill(T, steps, warmup, device, n_rep=2, seed=0, eager_steps=None):
+    """LLaMA-2-7B MLP linears at T tokens: gate/up group + down_proj solo (tcgen05 path).
+    With `eager_steps`, run that many plain steps and return None (profiling)."""
     import torch
     from rank_error_correction_b200 import glowq, synth
     reps = []
@@ -300,6 +301,11 @@ def time_prefill(T, steps, warmup, device, n_rep=2, seed=0):
         gu, Bg, dn, Bd = reps[i % n_rep]
         glowq.group_forward(gu, Bg, X, Ys=views, R_out=R, workspace=ws)
         glowq.solo_forward(dn, Bd, Xd, Y=Yd, workspace=ws)
+
+    if eager_steps is not None:
+        for i in range(eager_steps):
+            step(i)
+        return None
 
     with torch.cuda.stream(stream):
         for i in range(max(warmup, 3)):
@@ -385,6 +391,28 @@ def run_reference(args, rank, world):
     return 0
 
 
+# ------------------------------------------------------------ profile cases
+
+def profile_case(case, device, steps=4):
+    """A few untimed steps of one bench workload (no JSON line): the command
+    that the ncu summaries under profiles/ are captured from.  Launch order per
+    step -- decode: rproj_cluster, corrected_gemv (Q/K/V group), rproj_cluster,
+    corrected_gemv (o_proj); prefill: rproj_tc, rproj_sum, corrected_gemm
+    (gate/up), rproj_tc, rproj_sum, corrected_gemm (down_proj)."""
+    import torch
+    from rank_error_correction_b200 import glowq
+    if case == "decode":
+        reps = build_replicas(8, 1, device)
+        io = make_io(1, device)
+        for i in range(steps):
+            run_step(reps[i % len(reps)], io)
+    else:
+        time_prefill(2048, 1, 0, device, n_rep=1, eager_steps=steps)
+    torch.cuda.synchronize()
+    print(f"profile case {case}: {steps} steps done", flush=True)
+    return 0
+
+
 # --------------------------------------------------------------------- main
 
 def main():
@@ -397,6 +425,8 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the T=4/16 decode lines")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill line")
+    ap.add_argument("--profile-case", choices=["decode", "prefill"],
+                    help="run a few untimed steps of one workload and exit (for ncu captures)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -422,6 +452,9 @@ def main():
         pg = dist
         dist.barrier()
     glowq.lib()
+
+    if args.profile_case:
+        return profile_case(args.profile_case, device)
 
     hbm_peak, tf_peak, tf_sust, peak_src = _peaks()
     T = 1

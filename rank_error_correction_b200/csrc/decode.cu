@@ -14,19 +14,20 @@
 //     group.  Each warp streams its 16 rows of packed weights with 2-D TMA
 //     boxes into a private ring of mbarrier-tracked stages, issued before the
 //     wait on the preceding kernel (weights and scales are static), so the
-//     stream overlaps the projection.  Nibbles become the exact fp16 values
-//     64 + q in one LOP3 per pair; the multiply-accumulate runs on the tensor
-//     cores with register operands (mma.sync m16n8k16, fp32 accumulate) and
-//     each 128-group's dot product is finished in fp32 as
-//     s * (D - (64 + z) * sum_k x_k).  The k order inside an MMA is permuted
+//     stream overlaps the projection.  Nibbles become exact fp16 values
+//     (16 + q/64 for even k, 64 + q for odd k) with one LOP3 per pair; the
+//     multiply-accumulate runs on the tensor cores with register operands
+//     (mma.sync m16n8k16, fp32 accumulate, one chain per parity) and each
+//     128-group's dot product is finished in fp32 from the two chains and the
+//     even/odd activation sums.  The k order inside an MMA is permuted
 //     identically on both operands (a permutation of the contraction index
 //     leaves the dot product unchanged) so packed words map straight onto
 //     fragments.  d may be split inside the CTA or across a thread-block
 //     cluster whose partial sums meet in distributed shared memory; the
 //     rank-r correction A_i R is one more short MMA slab on the same fp32
 //     accumulators.
-//   * Numerics: the products (64 + q) x are exact in fp32 accumulation up to
-//     rounding of the sums; the effective weight is the exact (q - z) s rather
+//   * Numerics: the operand products are exact, sums are fp32; the
+//     effective weight is the exact (q - z) s rather
 //     than its fp16 rounding (at most 2^-12 relative per weight, far inside the
 //     parity bar).
 #include <cstdio>
@@ -43,7 +44,7 @@ namespace glowq {
 // R = X B^T for T <= 16 in one launch.  A cluster of kRcCtas CTAs splits d
 // (CTA c takes the c-th slice of the 32-wide k steps).  Inside a CTA, warp w
 // takes B rows 16*(w % nrb) .. +15 (nrb = ceil(r/16) row blocks) and every kl-th
-// k step of the slice (kl = 16 / nrb k-lanes), with two steps' loads in flight.
+// k step of the slice (kl = 16 / nrb k-lanes), with four steps' loads in flight.
 // Partial sums meet in a fixed order: k-lanes in shared memory, then the CTAs
 // of the cluster through distributed shared memory (ascending rank), so R does
 // not depend on timing.  R is rounded to fp16 once.
@@ -84,11 +85,11 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
         const uint4 zero4 = make_uint4(0, 0, 0, 0);
-        for (int st = s0 + kq; st < s1; st += 2 * kl) {
-            // two k steps per iteration, all loads issued before the MMAs
-            uint4 blo[2], bhi[2], xv[2][NT];
+        constexpr int U = 4;   // k steps per iteration, all loads issued before the MMAs
+        for (int st = s0 + kq; st < s1; st += U * kl) {
+            uint4 blo[U], bhi[U], xv[U][NT];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const int su = st + u * kl;
                 const bool in = su < s1;
                 const int k = su * 32 + 8 * t;
@@ -101,7 +102,7 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32)
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+            for (int u = 0; u < U; ++u) {
                 const uint32_t a0[4] = {blo[u].x, bhi[u].x, blo[u].y, bhi[u].y};
                 const uint32_t a1[4] = {blo[u].z, bhi[u].z, blo[u].w, bhi[u].w};
 #pragma unroll
@@ -163,12 +164,14 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32)
 //   * optionally a thread-block cluster of `kc` CTAs splits d further (then
 //     kw == 1); partial sums meet in distributed shared memory.
 //
-// Arithmetic of one 128-group (row o, tokens t, codes q, zero z, scale s):
-//   sum_k (q_k - z) s x_k = s * (D - (64 + z) * S),
-//   D = sum_k (64 + q_k) x_k  (tensor cores, fp32 accumulate),  S = sum_k x_k.
-// 64 + q is built in one LOP3 per half2 by placing the nibble in mantissa bits
-// 4..7 of the fp16 constant 64.0 (no subtraction per weight); the products are
-// exact and the offset costs ~3 of fp32's 24 bits.  S is computed once per CTA.
+// Arithmetic of one 128-group (row o, tokens t, codes q, zero z, scale s), with
+// E / O the even / odd k of the group:
+//   sum_k (q_k - z) s x_k = s * (64 D_E + D_O - (1024 + z) S_E - (64 + z) S_O),
+//   D_E = sum_{k in E} (16 + q_k / 64) x_k,  D_O = sum_{k in O} (64 + q_k) x_k
+//   (two tensor-core chains, fp32 accumulate),  S_E / S_O = sums of x over E / O.
+// Both operand forms are exact fp16 values built without subtracting anything
+// per weight: the nibble lands in mantissa bits 0..3 of 16.0 or 4..7 of 64.0,
+// one shift and four LOP3 per 8 codes.  S_E and S_O are computed once per CTA.
 //
 // Shared memory (dynamic), in this order:
 //   ring [warps][S][16][32] u32      packed-weight stream: a stage is one 2-D TMA
@@ -244,7 +247,7 @@ __host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, i
     L.xs = off;
     off += (T + 1) * L.wpt_max * 16;
     L.xsum = off;
-    off += L.ncta_max * 8 * nt * 4;
+    off += L.ncta_max * 2 * 8 * nt * 4;
     off = (off + 15) / 16 * 16;
     L.sz = off;
     off += warps * 16 * (L.nsub_max + 1) * 8;
@@ -271,14 +274,18 @@ __device__ __forceinline__ void mma_16816_zc(float c[4], const uint32_t a[4], co
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "f"(0.0f));
 }
 
-// One packed word (8 codes, low nibble first) -> four half2 holding the exact
-// values 64 + q of codes (0,4), (1,5), (2,6), (3,7): each nibble lands in
-// mantissa bits 4..7 of 64.0 (0x5400).
-__device__ __forceinline__ void unpack_offset64(uint32_t w, uint32_t out[4]) {
-    out[0] = ((w << 4) & 0x00F000F0u) | 0x54005400u;
-    out[1] = (w & 0x00F000F0u) | 0x54005400u;
-    out[2] = ((w >> 4) & 0x00F000F0u) | 0x54005400u;
-    out[3] = ((w >> 8) & 0x00F000F0u) | 0x54005400u;
+// One packed word (8 codes, low nibble first) -> four half2 of exact values,
+// one shift and four LOP3:
+//   ev[0] = 16 + q/64 of codes (0,4)   nibble in mantissa bits 0..3 of 16.0
+//   ev[1] = 16 + q/64 of codes (2,6)
+//   od[0] = 64 + q    of codes (1,5)   nibble in mantissa bits 4..7 of 64.0
+//   od[1] = 64 + q    of codes (3,7)
+__device__ __forceinline__ void unpack_even_odd(uint32_t w, uint32_t ev[2], uint32_t od[2]) {
+    const uint32_t w8 = w >> 8;
+    ev[0] = (w & 0x000F000Fu) | 0x4C004C00u;
+    od[0] = (w & 0x00F000F0u) | 0x54005400u;
+    ev[1] = (w8 & 0x000F000Fu) | 0x4C004C00u;
+    od[1] = (w8 & 0x00F000F0u) | 0x54005400u;
 }
 
 template <int NT, int S>
@@ -417,21 +424,24 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
         for (int i = threadIdx.x; i < wpt; i += stride) xs[T * wpt + i] = make_uint4(0, 0, 0, 0);
     }
     __syncthreads();
-    // 4) per-group activation sums S (fixed summation order; 0 for padding tokens)
+    // 4) per-group activation sums over even and odd k, S_E and S_O (fixed
+    //    summation order; 0 for padding tokens): xsum[(2 * group + e)][token]
     for (int i = threadIdx.x; i < ncta * 8 * NT; i += stride) {
         const int gc = i / (8 * NT), tok = i - gc * (8 * NT);
-        float acc_s = 0.f;
+        float se = 0.f, so = 0.f;
         if (tok < T) {
             const uint4* src = xs + tok * wpt + gc * 16;
 #pragma unroll 4
             for (int wd = 0; wd < 16; ++wd) {
-                const uint4 v = src[wd];
+                const uint4 v = src[wd];   // (x0,x4) (x1,x5) (x2,x6) (x3,x7)
                 const float2 f0 = __half22float2(u32_as_h2(v.x)), f1 = __half22float2(u32_as_h2(v.y));
                 const float2 f2 = __half22float2(u32_as_h2(v.z)), f3 = __half22float2(u32_as_h2(v.w));
-                acc_s += ((f0.x + f0.y) + (f1.x + f1.y)) + ((f2.x + f2.y) + (f3.x + f3.y));
+                se += (f0.x + f0.y) + (f2.x + f2.y);
+                so += (f1.x + f1.y) + (f3.x + f3.y);
             }
         }
-        xsum[gc * 8 * NT + tok] = acc_s;
+        xsum[(2 * gc) * 8 * NT + tok] = se;
+        xsum[(2 * gc + 1) * 8 * NT + tok] = so;
     }
     __syncthreads();
 
@@ -453,10 +463,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
             const int tok = (n * 8 + g < T) ? n * 8 + g : T;
             xrow[n] = xs + tok * wpt + (G0 - C0) * 16;
         }
-        const float* xsum_w = xsum + (G0 - C0) * 8 * NT + 2 * t;
-        // lane (g, t) reads 16 B of rows g and g+8 per group; odd rows read the
-        // second group first so each quarter-warp hits 8 distinct bank groups
-        const int par = g & 1;
+        const float* xsum_w = xsum + (G0 - C0) * 2 * 8 * NT + 2 * t;
+        // lane (g, t) reads 16 B of rows g and g+8 per group
         const unsigned char* rd_lo = my_ring + g * 128 + t * 16;
         const unsigned char* rd_hi = rd_lo + 8 * 128;
         bool ok = true;
@@ -468,15 +476,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
                     if (ok) ok = mbar_wait(my_bars + i, (uint32_t)((p / kStages) & 1), args.status);
                     const unsigned char* sl = rd_lo + i * 2048;
                     const unsigned char* sh = rd_hi + i * 2048;
-                    const uint4 l_first = *reinterpret_cast<const uint4*>(sl + par * 64);
-                    const uint4 h_first = *reinterpret_cast<const uint4*>(sh + par * 64);
-                    const uint4 l_second = *reinterpret_cast<const uint4*>(sl + (par ^ 1) * 64);
-                    const uint4 h_second = *reinterpret_cast<const uint4*>(sh + (par ^ 1) * 64);
                     uint4 w4[2][2];
-                    w4[0][0] = par ? l_second : l_first;
-                    w4[1][0] = par ? l_first : l_second;
-                    w4[0][1] = par ? h_second : h_first;
-                    w4[1][1] = par ? h_first : h_second;
+                    w4[0][0] = *reinterpret_cast<const uint4*>(sl);
+                    w4[0][1] = *reinterpret_cast<const uint4*>(sh);
+                    w4[1][0] = *reinterpret_cast<const uint4*>(sl + 64);
+                    w4[1][1] = *reinterpret_cast<const uint4*>(sh + 64);
                     if (p + kStages < npairs) {
                         fence_proxy_async_smem();   // this lane's reads of the slot precede the refill
                         __syncwarp();
@@ -492,36 +496,48 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const
                         const int gl = 2 * p + h;          // group within the warp's split
                         const uint32_t wl[4] = {w4[h][0].x, w4[h][0].y, w4[h][0].z, w4[h][0].w};
                         const uint32_t wh[4] = {w4[h][1].x, w4[h][1].y, w4[h][1].z, w4[h][1].w};
-                        float ta[NT][4], tb[NT][4];
+                        // two MMA chains: even k (A = 16 + q/64) and odd k (A = 64 + q)
+                        float te[NT][4], to[NT][4];
 #pragma unroll
                         for (int w = 0; w < 4; ++w) {
-                            uint32_t pl[4], ph[4];
-                            unpack_offset64(wl[w], pl);   // 64 + codes (i, i+4) of row g
-                            unpack_offset64(wh[w], ph);   // row g + 8
-                            const uint32_t a0[4] = {pl[0], ph[0], pl[1], ph[1]};
-                            const uint32_t a1[4] = {pl[2], ph[2], pl[3], ph[3]};
+                            uint32_t el[2], ol[2], eh[2], oh[2];
+                            unpack_even_odd(wl[w], el, ol);   // row g
+                            unpack_even_odd(wh[w], eh, oh);   // row g + 8
+                            const uint32_t ae[4] = {el[0], eh[0], el[1], eh[1]};
+                            const uint32_t ao[4] = {ol[0], oh[0], ol[1], oh[1]};
 #pragma unroll
                             for (int n = 0; n < NT; ++n) {
                                 const uint4 x = xrow[n][gl * 16 + ((4 * t + w) ^ xsw)];
-                                const uint32_t b0[2] = {x.x, x.y};   // (x0,x4) (x1,x5)
-                                const uint32_t b1[2] = {x.z, x.w};   // (x2,x6) (x3,x7)
+                                const uint32_t be[2] = {x.x, x.z};   // (x0,x4) (x2,x6)
+                                const uint32_t bo[2] = {x.y, x.w};   // (x1,x5) (x3,x7)
                                 if (w == 0) {
-                                    mma_16816_zc(ta[n], a0, b0);
-                                    mma_16816_zc(tb[n], a1, b1);
+                                    mma_16816_zc(te[n], ae, be);
+                                    mma_16816_zc(to[n], ao, bo);
                                 } else {
-                                    mma_16816(ta[n], a0, b0);
-                                    mma_16816(tb[n], a1, b1);
+                                    mma_16816(te[n], ae, be);
+                                    mma_16816(to[n], ao, bo);
                                 }
                             }
                         }
+                        // sum_k (q - z) x = 64 D_E + D_O - (1024 + z) S_E - (64 + z) S_O, times s
                         const float2 zl = sz_lo[gl], zh = sz_hi[gl];   // (s, 64 + z)
+                        const float cel = zl.y + 960.0f, ceh = zh.y + 960.0f;
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
-                            const float2 sx = *reinterpret_cast<const float2*>(xsum_w + gl * 8 * NT + n * 8);
-                            acc[n][0] = fmaf(zl.x, fmaf(-zl.y, sx.x, ta[n][0] + tb[n][0]), acc[n][0]);
-                            acc[n][1] = fmaf(zl.x, fmaf(-zl.y, sx.y, ta[n][1] + tb[n][1]), acc[n][1]);
-                            acc[n][2] = fmaf(zh.x, fmaf(-zh.y, sx.x, ta[n][2] + tb[n][2]), acc[n][2]);
-                            acc[n][3] = fmaf(zh.x, fmaf(-zh.y, sx.y, ta[n][3] + tb[n][3]), acc[n][3]);
+                            const float2 se = *reinterpret_cast<const float2*>(xsum_w + (2 * gl) * 8 * NT + n * 8);
+                            const float2 so = *reinterpret_cast<const float2*>(xsum_w + (2 * gl + 1) * 8 * NT + n * 8);
+                            float v0 = fmaf(64.0f, te[n][0], to[n][0]);
+                            float v1 = fmaf(64.0f, te[n][1], to[n][1]);
+                            float v2 = fmaf(64.0f, te[n][2], to[n][2]);
+                            float v3 = fmaf(64.0f, te[n][3], to[n][3]);
+                            v0 = fmaf(-zl.y, so.x, fmaf(-cel, se.x, v0));
+                            v1 = fmaf(-zl.y, so.y, fmaf(-cel, se.y, v1));
+                            v2 = fmaf(-zh.y, so.x, fmaf(-ceh, se.x, v2));
+                            v3 = fmaf(-zh.y, so.y, fmaf(-ceh, se.y, v3));
+                            acc[n][0] = fmaf(zl.x, v0, acc[n][0]);
+                            acc[n][1] = fmaf(zl.x, v1, acc[n][1]);
+                            acc[n][2] = fmaf(zh.x, v2, acc[n][2]);
+                            acc[n][3] = fmaf(zh.x, v3, acc[n][3]);
                         }
                     }
                 }
