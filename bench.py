@@ -33,6 +33,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "GlowQ linear tok/s (decode T=1, prefill T=2048); % of HBM / tensor roofline"
 WORKLOAD = "llama2_7b_attn_decode"
+DECODE_WORKLOAD = ("LLaMA-2-7B attention linears, decode T=1: Q/K/V group (3x4096x4096) + "
+                   "o_proj solo (4096x4096), INT4 g128 asym, r=64 fp16 factors")
 R_RANK = 64
 D = 4096
 QKV_OUTS = [4096, 4096, 4096]
@@ -382,8 +384,8 @@ def run_reference(args, rank, world):
     line = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
             "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": f"{WORKLOAD} (QKV group + o_proj solo, d=4096, r=64, INT4 g128)",
-                       "tokens": T, "sample": f"{rows} rows per module of 16384; scaled by row fraction"},
+            "config": {"workload": DECODE_WORKLOAD, "tokens": T,
+                       "sample": f"{rows} rows per module of 16384; scaled by row fraction"},
             "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle",
                              "sample": f"{rows} of 4096 rows per module x 4 modules per step, {steps} steps"},
             "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -512,19 +514,23 @@ def main():
                          f"scaled by the row fraction ({frac:.4f})"}
 
     if rank == 0:
-        traffic = None
+        # DRAM bytes per launch from the committed ncu captures (profiles/)
+        traffic = traffic_pf = None
         tr_path = os.path.join(ROOT, "profiles", "traffic.json")
         if os.path.exists(tr_path):
             try:
-                traffic = json.load(open(tr_path)).get("corrected_gemv_kernel<1> qkv T=1")
+                tr = json.load(open(tr_path))
+                traffic = tr.get("decode qkv T=1 group call", {}).get("bytes")
+                traffic_pf = tr.get("prefill gate_up T=2048 corrected_gemm", {}).get("bytes")
             except Exception:
-                traffic = None
+                traffic = traffic_pf = None
+        if prefill is not None:
+            prefill["roofline"]["traffic"] = traffic_pf
         line = {
             "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16 x int4 -> fp32 acc", "data": "synthetic",
-            "config": {"workload": "LLaMA-2-7B attention linears, decode T=1: Q/K/V group (3x4096x4096) + "
-                                   "o_proj solo (4096x4096), INT4 g128 asym, r=64 fp16 factors",
+            "config": {"workload": DECODE_WORKLOAD,
                        "tokens": T, "replicas": args.replicas,
                        "l2": f"inputs larger than L2: {args.replicas} weight replicas rotated "
                              f"({args.replicas * 38.4:.0f} MB)",
