@@ -42,34 +42,51 @@ namespace glowq {
 
 // ---------------------------------------------------------------------------
 // R = X B^T for T <= 16 in one launch.  A cluster of kRcCtas CTAs splits d
-// (CTA c takes the c-th slice of the 32-wide k steps).  Inside a CTA, warp w
-// takes B rows 16*(w % nrb) .. +15 (nrb = ceil(r/16) row blocks) and every kl-th
-// k step of the slice (kl = 16 / nrb k-lanes), with four steps' loads in flight.
-// Partial sums meet in a fixed order: k-lanes in shared memory, then the CTAs
-// of the cluster through distributed shared memory (ascending rank), so R does
-// not depend on timing.  R is rounded to fp16 once.
+// (CTA c takes the c-th slice of the 32-wide k steps).  Inside a CTA the work
+// items (B row block of 16 rows, k-lane) are spread over the warps; a k-lane
+// takes every kl-th k step of the slice, two steps' loads in flight.  Partial
+// sums meet in a fixed order: k-lanes in shared memory, then the CTAs of the
+// cluster through distributed shared memory (ascending rank), so R does not
+// depend on timing.  R is rounded to fp16 once.
+// The CTA is small enough to be resident next to a GEMV CTA, so it starts
+// while the preceding GEMV still runs: B is static, so its slice is copied
+// into shared memory (or, when it does not fit, pulled into L2) before the
+// wait on the preceding kernel; after the wait only X is read from memory.
 // ---------------------------------------------------------------------------
 constexpr int kRcCtas = 8;
-constexpr int kRcWarps = 16;
+constexpr int kRcWarps = 8;
+constexpr int kRcStageB = 72 * 1024;         // largest B slice staged in shared memory
 
 __host__ __device__ inline int rc_row_blocks(int r) { return (r + 15) / 16; }
-// shared memory: per-k-lane partials [kl][8*NT][r] + the CTA partial [8*NT][r] (fp32)
-__host__ __device__ inline int rc_smem_bytes(int r, int nt) {
-    const int nrb = rc_row_blocks(r), kl = kRcWarps / nrb;
-    return (kl + 1) * 8 * nt * r * 4;
+__host__ __device__ inline int rc_klanes(int r) {
+    const int kl = kRcWarps / rc_row_blocks(r);
+    return kl > 0 ? kl : 1;
+}
+// B slice of one CTA: r rows x (steps of 32 k), row pitch padded by 16 B
+__host__ __device__ inline int rc_b_pitch(int d) {
+    const int nsteps = d / 32;
+    return ((nsteps + kRcCtas - 1) / kRcCtas) * 64 + 16;
+}
+__host__ __device__ inline bool rc_stage_b(int r, int d) { return r * rc_b_pitch(d) <= kRcStageB; }
+// shared memory: per-k-lane partials [kl][8*NT][r] + the CTA partial [8*NT][r]
+// (fp32), the CTA's X slice [T][slice] (fp16), then the staged B slice and its
+// mbarrier
+__host__ __device__ inline int rc_part_bytes(int r, int nt) { return (rc_klanes(r) + 1) * 8 * nt * r * 4; }
+__host__ __device__ inline int rc_x_bytes(int d, int nt) { return 8 * nt * (rc_b_pitch(d) - 16); }
+__host__ __device__ inline int rc_smem_bytes(int r, int d, int nt) {
+    const int p = (rc_part_bytes(r, nt) + 15) / 16 * 16 + rc_x_bytes(d, nt);
+    return rc_stage_b(r, d) ? p + r * rc_b_pitch(d) + 16 : p;
 }
 
 template <int NT>
-__global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32)
+__global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32, 4)
     rproj_cluster_kernel(const __half* __restrict__ X, const __half* __restrict__ B, int T, int d, int r,
-                         __half* __restrict__ R) {
+                         __half* __restrict__ R, unsigned int* status) {
     pdl_launch_dependents();    // the GEMV may start streaming weights now
-    pdl_wait();                 // X may come from the previous kernel in the stream
     extern __shared__ __align__(16) float rc_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const int nrb = rc_row_blocks(r), kl = kRcWarps / nrb;
-    const int rb = warp % nrb, kq = warp / nrb;
+    const int nrb = rc_row_blocks(r), kl = rc_klanes(r);
     const int TP = 8 * NT;                       // padded token count
     float* part = rc_smem;                       // [kl][TP][r]
     float* cpart = rc_smem + kl * TP * r;        // [TP][r]
@@ -77,15 +94,51 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32)
     asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
     const int nsteps = d / 32;
     const int s0 = (int)((int64_t)crank * nsteps / kRcCtas), s1 = (int)((int64_t)(crank + 1) * nsteps / kRcCtas);
-    if (kq < kl) {
+    const bool staged = rc_stage_b(r, d);
+    const int pitch = rc_b_pitch(d);
+    unsigned char* xsl = reinterpret_cast<unsigned char*>(rc_smem) + (rc_part_bytes(r, NT) + 15) / 16 * 16;
+    const int xpitch = pitch - 16;               // bytes of one token's slice
+    unsigned char* bs = xsl + rc_x_bytes(d, NT);
+    uint64_t* bbar = reinterpret_cast<uint64_t*>(bs + r * pitch);
+    // B is static: stage (or prefetch) this CTA's slice before the wait
+    if (staged) {
+        if (threadIdx.x == 0) {
+            mbar_init(bbar, 1);
+            fence_mbar_init();
+            mbar_arrive_expect_tx(bbar, (uint32_t)(r * (s1 - s0) * 64));
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < r; j += blockDim.x)
+            bulk_g2s(smem_u32(bs + j * pitch), B + (int64_t)j * d + s0 * 32, (uint32_t)((s1 - s0) * 64), bbar);
+    } else {
+        for (int j = threadIdx.x; j < r; j += blockDim.x)
+            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
+                         ::"l"(B + (int64_t)j * d + s0 * 32), "r"((uint32_t)((s1 - s0) * 64))
+                         : "memory");
+    }
+    pdl_wait();                 // X may come from the previous kernel in the stream
+    // the CTA's slice of X in one round trip (16-byte chunks), padding tokens 0
+    {
+        const int chunks = xpitch / 16, n = TP * chunks;
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            const int tok = i / chunks, c = i - tok * chunks;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (tok < T && s0 * 32 + c * 8 < s1 * 32) v = ldg_128(X + (int64_t)tok * d + s0 * 32 + c * 8);
+            *reinterpret_cast<uint4*>(xsl + tok * xpitch + c * 16) = v;
+        }
+    }
+    if (staged) mbar_wait(bbar, 0, status);
+    __syncthreads();
+    const uint4 zero4 = make_uint4(0, 0, 0, 0);
+    for (int item = warp; item < nrb * kl; item += kRcWarps) {
+        const int rb = item % nrb, kq = item / nrb;
         const int j0 = rb * 16 + g, j1 = j0 + 8;
         float acc[NT][4];
 #pragma unroll
         for (int n = 0; n < NT; ++n)
 #pragma unroll
             for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-        const uint4 zero4 = make_uint4(0, 0, 0, 0);
-        constexpr int U = 4;   // k steps per iteration, all loads issued before the MMAs
+        constexpr int U = 2;   // k steps per iteration, all loads issued before the MMAs
         for (int st = s0 + kq; st < s1; st += U * kl) {
             uint4 blo[U], bhi[U], xv[U][NT];
 #pragma unroll
@@ -93,13 +146,18 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32)
                 const int su = st + u * kl;
                 const bool in = su < s1;
                 const int k = su * 32 + 8 * t;
-                blo[u] = (in && j0 < r) ? ldg_128(B + (int64_t)j0 * d + k) : zero4;
-                bhi[u] = (in && j1 < r) ? ldg_128(B + (int64_t)j1 * d + k) : zero4;
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const int tok = n * 8 + g;
-                    xv[u][n] = (in && tok < T) ? ldg_128(X + (int64_t)tok * d + k) : zero4;
+                if (staged) {
+                    const int off = (su - s0) * 64 + 16 * t;
+                    blo[u] = (in && j0 < r) ? *reinterpret_cast<const uint4*>(bs + j0 * pitch + off) : zero4;
+                    bhi[u] = (in && j1 < r) ? *reinterpret_cast<const uint4*>(bs + j1 * pitch + off) : zero4;
+                } else {
+                    blo[u] = (in && j0 < r) ? ldg_128(B + (int64_t)j0 * d + k) : zero4;
+                    bhi[u] = (in && j1 < r) ? ldg_128(B + (int64_t)j1 * d + k) : zero4;
                 }
+#pragma unroll
+                for (int n = 0; n < NT; ++n)
+                    xv[u][n] = in ? *reinterpret_cast<const uint4*>(xsl + (n * 8 + g) * xpitch + (su - s0) * 64 + 16 * t)
+                                  : zero4;
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -187,7 +245,7 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32)
 //   red  [nslots][NT*4][32] f32      partial sums sent to the finalising warp
 //   as   [fin_slots][16][r+8] f16    A rows of the tiles this CTA finalises
 // ---------------------------------------------------------------------------
-constexpr int kMaxWarps = 8;
+constexpr int kMaxWarps = 12;   // 12 x 32 x 128 registers leave room for an R CTA on the SM
 // Pipeline stages per warp (one 2-D TMA box of 16 rows x 2 groups of 128,
 // 2 KB) are a template parameter S in {4, 8}: the host trades ring depth
 // against resident warps.
@@ -227,7 +285,7 @@ struct GemvLayout {    // byte offsets into dynamic shared memory
 // Launch-time constants computed on the host (no divisions in the kernel).
 struct GemvPlan {
     GemvLayout L;
-    int gsplit[9];     // group boundaries of split j = crank * kw + ks, j in [0, kc * kw]
+    int gsplit[17];    // group boundaries of split j = crank * kw + ks, j in [0, kc * kw] (kc * kw <= 16)
 };
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -289,7 +347,9 @@ __device__ __forceinline__ void unpack_even_odd(uint32_t w, uint32_t ev[2], uint
 }
 
 template <int NT, int S>
-__global__ void __launch_bounds__(kMaxWarps * 32, 2) corrected_gemv_kernel(const __grid_constant__ GemvArgs args,
+// (the bound of 512 threads caps registers at 128 per thread; launches use at
+// most kMaxWarps warps)
+__global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_constant__ GemvArgs args,
                                                                            const __grid_constant__ GemvPlan plan) {
     pdl_launch_dependents();
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -661,9 +721,17 @@ cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int
     const __half* Xh = reinterpret_cast<const __half*>(X);
     const __half* Bh = reinterpret_cast<const __half*>(B);
     __half* Rh = reinterpret_cast<__half*>(R);
-    void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&Rh};
+    unsigned int* status = device_status_ptr();
+    void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&Rh, (void*)&status};
     const void* fn = (nt == 1) ? (const void*)rproj_cluster_kernel<1> : (const void*)rproj_cluster_kernel<2>;
-    return launch_ex(fn, dim3(kRcCtas), dim3(kRcWarps * 32), (size_t)rc_smem_bytes(r, nt), st, true, a1);
+    const size_t smem = (size_t)rc_smem_bytes(r, d, nt);
+    static bool opted[2] = {false, false};
+    if (smem > 48 * 1024 && !opted[nt - 1]) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRcStageB + 32 * 1024);
+        if (e != cudaSuccess) return e;
+        opted[nt - 1] = true;
+    }
+    return launch_ex(fn, dim3(kRcCtas), dim3(kRcWarps * 32), smem, st, true, a1);
 }
 
 
@@ -721,8 +789,17 @@ static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sm
     const int ngroups = d / 128;
     GemvShape best = {0, 0, 0, 0, 0};
     double best_key[5] = {1e30, 1e30, 1e30, 1e30, 1e30};
+    // Cost model: the busiest SM sets the time.  CTAs of a cluster launch are
+    // packed onto SMs up to their residency (observed: two 8-warp CTAs per SM
+    // while other SMs idle), other launches are spread; the busiest SM's load
+    // is its CTAs x row tiles x 128-groups per CTA.  Ties prefer more warps on
+    // that SM (latency hiding), more bytes in flight, then fewer splits.
+    // A shape may also request more shared memory than it uses (kSpreadSmem),
+    // which leaves room for one CTA per SM: the launch is then spread.
+    constexpr size_t kSpreadSmem = 116 * 1024;
+    for (int pad = 0; pad <= 1; ++pad)
     for (int stages = 4; stages <= 8; stages *= 2)
-        for (int rt = 1; rt <= kMaxWarps; rt *= 2)
+        for (int rt = 1; rt <= kMaxWarps; ++rt)
             for (int kw = 1; rt * kw <= kMaxWarps; ++kw)
                 for (int kc = 1; kc <= 8; ++kc) {
                     if (kc > 1 && kw > 1) break;
@@ -730,23 +807,26 @@ static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sm
                     const int warps = rt * kw;
                     const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, nt, stages);
                     if (L.total > 220 * 1024) continue;
+                    if (pad && (size_t)L.total >= kSpreadSmem) continue;
+                    const size_t smem = pad ? kSpreadSmem : (size_t)L.total;
                     const void* fn = gemv_fn(nt, stages);
-                    const int res = resident_ctas(fn, warps, kc, (size_t)L.total, num_sms);
+                    const int res = resident_ctas(fn, warps, kc, smem, num_sms);
                     if (res <= 0) continue;
                     const long ctas = (long)ceil_div(tiles, rt) * kc;
                     const double waves = (double)ctas / res;
-                    const long sms = ctas < num_sms ? ctas : num_sms;
-                    const double warps_sm = (double)(ctas * warps) / sms;
-                    // bytes a warp can have in flight: its ring, or its whole slice if smaller
+                    const int res_sm = res / num_sms > 0 ? res / num_sms : 1;
+                    long per_sm = (kc > 1) ? (ctas < res_sm ? ctas : res_sm) : (long)ceil_div((int)ctas, num_sms);
+                    if (per_sm > res_sm) per_sm = res_sm;
+                    const double load = (double)per_sm * rt * ceil_div(ngroups, kc);
+                    const double warps_sm = (double)per_sm * warps;
                     const int groups_warp = ceil_div(ceil_div(ngroups, kc), kw);
-                    const double inflight_warp = 1024.0 * (groups_warp < 2 * stages ? groups_warp : 2 * stages);
-                    const double inflight_sm = inflight_warp * warps_sm;
+                    const double inflight_sm = 1024.0 * (groups_warp < 2 * stages ? groups_warp : 2 * stages) * warps_sm;
                     double key[5];
                     key[0] = waves <= 1.0 ? 0.0 : waves;
-                    key[1] = -(double)sms;
+                    key[1] = load;
                     key[2] = -(warps_sm < 16.0 ? warps_sm : 16.0);
                     key[3] = -(inflight_sm < 131072.0 ? inflight_sm : 131072.0);
-                    key[4] = kw * kc + 0.1 * stages - 0.01 * rt;
+                    key[4] = kw * kc + 0.1 * stages - 0.01 * rt + 0.001 * pad;
                     bool better = false;
                     for (int j = 0; j < 5; ++j) {
                         if (key[j] < best_key[j] - 1e-9) { better = true; break; }
@@ -754,7 +834,7 @@ static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sm
                     }
                     if (better) {
                         for (int j = 0; j < 5; ++j) best_key[j] = key[j];
-                        best = {rt, kw, kc, stages, (size_t)L.total};
+                        best = {rt, kw, kc, stages, smem};
                     }
                 }
     if (used < 128 && best.rt > 0) memo[used++] = {tiles, d, T, r, nt, best};
@@ -800,7 +880,7 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     if (const char* env = std::getenv("GLOWQ_DECODE_SHAPE")) {
         int v[4] = {0, 0, 0, 0};
         if (std::sscanf(env, "%d,%d,%d,%d", &v[0], &v[1], &v[2], &v[3]) == 4 && v[0] >= 1 && v[1] >= 1 &&
-            v[2] >= 1 && v[2] <= 8 && (v[0] & (v[0] - 1)) == 0 && v[0] * v[1] <= kMaxWarps && (v[2] == 1 || v[1] == 1) &&
+            v[2] >= 1 && v[2] <= 8 && v[0] * v[1] <= kMaxWarps && (v[2] == 1 || v[1] == 1) &&
             (v[3] == 4 || v[3] == 8) && v[2] <= d / 128 && (d / 128) / v[2] >= v[1]) {
             const GemvLayout L = gemv_layout(T, d, r, v[0], v[1], v[2], nt, v[3]);
             if (L.total <= 220 * 1024) sh = {v[0], v[1], v[2], v[3], (size_t)L.total};
