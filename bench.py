@@ -188,8 +188,9 @@ def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
     with torch.cuda.graph(g, stream=stream):
         for i in range(steps):
             run_step(reps[i % n_rep], io)
-    g.replay()
-    stream.synchronize()
+    with torch.cuda.stream(stream):
+        g.replay()                     # warm replay on the same stream as the timed one
+    torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(gpu_index) if want_clocks else None
@@ -218,11 +219,12 @@ def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
             mo, Bo = rep["o_proj"]
             glowq.solo_forward(mo[0], Bo, io["X2"], Y=io["Yo"], workspace=io["ws"])
             evs[i][2].record()
-    gi.replay()
-    stream.synchronize()
     with torch.cuda.stream(stream):
-        gi.replay()
-    stream.synchronize()
+        gi.replay()                    # warm replay
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        gi.replay()                    # the replay whose event nodes are read
+    torch.cuda.synchronize()
     qkv_ms = [evs[i][0].elapsed_time(evs[i][1]) for i in range(steps)]
     o_ms = [evs[i][1].elapsed_time(evs[i][2]) for i in range(steps)]
     del gi
@@ -313,9 +315,28 @@ def time_prefill(T, steps, warmup, device, n_rep=2, seed=0, eager_steps=None):
         for i in range(max(warmup, 3)):
             step(i)
     stream.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    # timed graph: all steps back to back, no event nodes inside (they would
+    # break the programmatic-dependent-launch overlap between calls)
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            step(i)
+    with torch.cuda.stream(stream):
+        g.replay()                     # warm replay on the same stream as the timed one
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record()
+        g.replay()
+        t1.record()
+    torch.cuda.synchronize()
+    total_ms = t0.elapsed_time(t1)
+    del g
+    # per-call durations (roofline): a second graph with event nodes around each call
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(steps)]
+    gi = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gi, stream=stream):
         for i in range(steps):
             gu, Bg, dn, Bd = reps[i % n_rep]
             evs[i][0].record()
@@ -323,19 +344,15 @@ def time_prefill(T, steps, warmup, device, n_rep=2, seed=0, eager_steps=None):
             evs[i][1].record()
             glowq.solo_forward(dn, Bd, Xd, Y=Yd, workspace=ws)
             evs[i][2].record()
-    g.replay()
-    stream.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        t0.record()
-        g.replay()
-        t1.record()
-    stream.synchronize()
-    total_ms = t0.elapsed_time(t1)
+        gi.replay()                    # warm replay
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        gi.replay()                    # the replay whose event nodes are read
+    torch.cuda.synchronize()
     gu_ms = statistics.mean(evs[i][0].elapsed_time(evs[i][1]) for i in range(steps))
     dn_ms = statistics.mean(evs[i][1].elapsed_time(evs[i][2]) for i in range(steps))
-    del g
+    del gi
     return dict(total_ms=total_ms, gu_ms=gu_ms, dn_ms=dn_ms)
 
 
@@ -393,6 +410,131 @@ def run_reference(args, rank, world):
     return 0
 
 
+# ------------------------------------------- 40-layer LLaMA-2-13B linear stack
+
+S13_D, S13_FFN, S13_LAYERS = 5120, 13824, 40
+# (unit, output features of its modules, input dimension, activation alpha)
+S13_UNITS = [("qkv", [5120, 5120, 5120], 5120, "qkv"), ("o_proj", [5120], 5120, "qkv"),
+             ("gate_up", [13824, 13824], 5120, "mlp"), ("down_proj", [5120], 13824, "mlp")]
+# The pages' Table 3 (LLaMA-2-7B time to first batch on their RTX 4090), context only.
+PAGES_TABLE3_TTFB_MS = {"layerwise": 88.45, "glowq": 82.66, "glowq_s": 66.68}
+
+
+def build_stack13b(device, layers=S13_LAYERS, seed=0):
+    """Random-init INT4 g128 weights of a LLaMA-2-13B linear stack, r = 64 factors:
+    a shared B per unit (GlowQ) and an own B_i per module (layerwise), device
+    error norms and the GlowQ-S top-50% mask by g_ner."""
+    import numpy as np
+    import torch
+    from rank_error_correction_b200 import glowq, synth
+    units, e2, w2, layer_idx, kind = [], [], [], [], []
+    for l in range(layers):
+        for k, (name, outs, d, _) in enumerate(S13_UNITS):
+            mods, e_u, w_u = [], 0.0, 0.0
+            for i, O in enumerate(outs):
+                W = synth.device_weights(O, d, seed, sub=100000 + 100 * l + 10 * k + i, device=device)
+                q, s, z = glowq.pack_int4(W)
+                en = glowq.error_norms(W, q, s, z).sum(dim=0)
+                e_u, w_u = e_u + en[0], w_u + en[1]
+                del W
+                mods.append((q, s, z))
+            As, B = synth.device_factors(outs, d, R_RANK, seed, sub=200000 + 10 * l + k, device=device)
+            own = [synth.device_factors([O], d, R_RANK, seed, sub=300000 + 100 * l + 10 * k + i, device=device)
+                   for i, O in enumerate(outs)]
+            units.append(dict(name=name, d=d, outs=outs, packed=mods, As=As, B=B,
+                              own=[(a[0], b) for a, b in own]))
+            e2.append(e_u)
+            w2.append(w_u)
+            layer_idx.append(l)
+            kind.append(k)
+    torch.cuda.synchronize()
+    e2 = np.array([float(x) for x in e2])
+    w2 = np.array([float(x) for x in w2])
+    mask, _, _ = glowq.select_restore(e2, w2, np.array(layer_idx, np.int32), np.array(kind, np.int32),
+                                      len(units) // 2)
+    for u, m in zip(units, mask):
+        u["restore"] = bool(m)
+    return units
+
+
+def time_stack13b(units, T, steps, warmup, device, mode, seed=0):
+    """One token batch through every linear of the stack, captured in one CUDA
+    graph.  mode: 'layerwise' (every module its own R_i = X B_i^T), 'glowq'
+    (R shared per group, all units corrected) or 'glowq_s' (only the restored
+    units corrected).  Every unit reads a fixed synthetic input of its width
+    (the stack's data flow between layers is not modelled; the inputs are the
+    timing-only device draws of synth.device_activations).  Returns ms/batch."""
+    import torch
+    from rank_error_correction_b200 import glowq, synth
+    # timing-only inputs (iid, unit power per coordinate): one per unit kind
+    Xs = {n: synth.device_activations(T, d, seed, sub=500 + k, device=device)
+          for k, (n, _, d, _) in enumerate(S13_UNITS)}
+    Ys = {n: [torch.empty((T, O), dtype=torch.float16, device=device) for O in outs]
+          for n, outs, _, _ in S13_UNITS}
+    ws = glowq.alloc_workspace(T, R_RANK, device)
+    calls = []
+    for u in units:
+        a = u["name"]
+        X = Xs[a]
+        if mode == "layerwise":
+            for (q, s, z), (A, B), Y in zip(u["packed"], u["own"], Ys[a]):
+                calls.append(("solo", glowq.QModule(q, s, z, A), B, X, Y))
+        else:
+            on = mode == "glowq" or u["restore"]
+            mods = [glowq.QModule(q, s, z, A if on else None) for (q, s, z), A in zip(u["packed"], u["As"])]
+            B = u["B"] if on else None
+            if len(mods) > 1:
+                calls.append(("group", mods, B, X, Ys[a]))
+            else:
+                calls.append(("solo", mods[0], B, X, Ys[a][0]))
+    R = torch.empty((T, R_RANK), dtype=torch.float16, device=device)
+
+    def one():
+        for kindc, m, B, X, Y in calls:
+            if kindc == "group":
+                glowq.group_forward(m, B, X, Ys=Y, R_out=R if B is not None else None, workspace=ws)
+            else:
+                glowq.solo_forward(m, B, X, Y=Y, workspace=ws)
+
+    stream = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(max(warmup, 1)):
+            one()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(steps):
+            one()
+    with torch.cuda.stream(stream):
+        g.replay()                     # warm replay on the same stream as the timed one
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record()
+        g.replay()
+        t1.record()
+    stream.synchronize()
+    ms = t0.elapsed_time(t1) / steps
+    del g
+    return ms
+
+
+def stack13b_line(device, warmup):
+    units = build_stack13b(device)
+    out = {"workload": "LLaMA-2-13B-shaped linear stack, 40 layers x (Q/K/V group 3x5120x5120, o_proj 5120x5120, "
+                       "gate/up group 2x13824x5120, down_proj 5120x13824), INT4 g128 asym, r=64, random-init "
+                       "weights, GlowQ-S restoring the top 50% of units by g_ner",
+           "units": len(units), "restored_units": sum(u["restore"] for u in units),
+           "context_pages_table3_ttfb_ms_llama2_7b": PAGES_TABLE3_TTFB_MS}
+    for T, steps in ((1, 10), (2048, 2)):
+        ms = {mode: time_stack13b(units, T, steps, warmup, device, mode) for mode in ("layerwise", "glowq", "glowq_s")}
+        out[f"T{T}"] = {"ms_per_batch": ms, "tok_s": {k: T / (v * 1e-3) for k, v in ms.items()},
+                        "speedup_vs_layerwise": {k: ms["layerwise"] / v for k, v in ms.items()}}
+    del units
+    return out
+
+
 # ------------------------------------------------------------ profile cases
 
 def profile_case(case, device, steps=4):
@@ -427,6 +569,7 @@ def main():
     ap.add_argument("--no-extra", action="store_true", help="skip the T=4/16 decode lines")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill line")
+    ap.add_argument("--no-stack", action="store_true", help="skip the 40-layer LLaMA-2-13B stack line")
     ap.add_argument("--profile-case", choices=["decode", "prefill"],
                     help="run a few untimed steps of one workload and exit (for ncu captures)")
     args = ap.parse_args()
@@ -501,6 +644,10 @@ def main():
                                 "frac": tf_gu / tf_peak, "down_proj_TFLOPs": tf_dn,
                                 "algorithmic_flops": group_flops([MLP_FFN] * 2, MLP_D, R_RANK, Tp)}}
 
+    stack = None
+    if not args.no_stack:
+        stack = stack13b_line(device, args.warmup)
+
     cpu = None
     if rank == 0 and not args.no_cpu:
         times, frac = [], None
@@ -549,6 +696,7 @@ def main():
             "cpu_baseline": cpu,
             "extra": extra,
             "prefill": prefill,
+            "stack13b": stack,
         }
         print(json.dumps(line), flush=True)
     if pg is not None:

@@ -218,3 +218,15 @@ def device_factors(out_features: List[int], d: int, r: int, seed: int, sub: int,
     g.manual_seed(_torch_seed(seed, S_B, sub))
     B = (torch.randn((r, d), generator=g, device=device) * b_std).half()
     return As, B
+
+
+def device_activations(T: int, d: int, seed: int, sub: int, device="cuda"):
+    """Timing-only stand-in for X on the device: iid N(0, 1) rounded to fp16, the
+    same mean power per coordinate as the unit-mean power-law inputs (their
+    correlation structure matters for the solve and the parity tests, not for
+    the kernels' speed)."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(_torch_seed(seed, S_X, sub))
+    return torch.randn((T, d), generator=g, device=device, dtype=torch.float32).half()
+
