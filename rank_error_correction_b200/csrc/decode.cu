@@ -390,6 +390,28 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     const bool finaliser = ks == 0 && owner == crank;
     const bool has_corr = r > 0 && M.A != nullptr;
 
+    // 0) this warp's scales and zeros are the longest-latency reads of the
+    //    prologue (scattered, cold): a split of at most 32 groups is loaded in
+    //    one batch before the weight stream is started, and staged below
+    const int sz_stride = L.nsub_max + 1;
+    float2* my_sz = szs + warp * 16 * sz_stride;
+    const int rr = lane & 15;   // lane -> row (lane & 15) and every other group starting at lane >> 4
+    const int64_t sz_base = (int64_t)(tile_row + rr) * ngroups + G0;
+    const int nsub0 = G1 - G0;
+    const bool one_batch = active && nsub0 <= 32;
+    unsigned short sv[16];
+    unsigned char zv[16];
+    if (one_batch) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int gg = (lane >> 4) + 2 * j;
+            if (gg < nsub0) {
+                sv[j] = __half_as_ushort(M.s[sz_base + gg]);
+                zv[j] = M.z[sz_base + gg];
+            }
+        }
+    }
+
     // 1) start the weight stream: per warp, S mbarriers; lane 0 issues one 2-D
     //    TMA box (16 rows x 2 groups) per stage
     constexpr int kStages = S;
@@ -421,23 +443,23 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     }
     cp_async_commit();
 
-    // 2) this warp's (s, 64 + z): rows of its tile x groups [G0, G1); loads in
-    //    batches of 16 per lane, all issued before any is used
-    const int sz_stride = L.nsub_max + 1;
-    float2* my_sz = szs + warp * 16 * sz_stride;
-    if (active) {
-        // lane -> row (lane & 15) and every other group starting at lane >> 4
-        const int rr = lane & 15;
-        const int64_t obase = (int64_t)(tile_row + rr) * ngroups + G0;
+    // 2) stage (s, 64 + z) of the warp's rows x groups [G0, G1); longer splits
+    //    load in batches of 16 per lane, all issued before any is used
+    if (one_batch) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            const int gg = (lane >> 4) + 2 * j;
+            if (gg < nsub)
+                my_sz[rr * sz_stride + gg] = make_float2(__half2float(__ushort_as_half(sv[j])), 64.0f + (float)zv[j]);
+        }
+    } else if (active) {
         for (int g0 = lane >> 4; g0 < nsub; g0 += 32) {
-            unsigned short sv[16];
-            unsigned char zv[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int gg = g0 + 2 * j;
                 if (gg < nsub) {
-                    sv[j] = __half_as_ushort(M.s[obase + gg]);
-                    zv[j] = M.z[obase + gg];
+                    sv[j] = __half_as_ushort(M.s[sz_base + gg]);
+                    zv[j] = M.z[sz_base + gg];
                 }
             }
 #pragma unroll

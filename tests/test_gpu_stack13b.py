@@ -142,3 +142,26 @@ def test_stack_forward_matches_oracle(stack, T):
             assert np.all(np.isfinite(got))
             err = normwise(got, ref)
             assert err < TOL, (u["name"], u["layer"], bool(restore), T, err)
+
+
+@pytest.mark.parametrize("T", [1, 64])
+def test_layerwise_mode_matches_oracle(stack, T):
+    """Layerwise baseline: every module of the layer-0 Q/K/V group with its own
+    factors (A_i, B_i) through the solo path, R_i = X B_i^T per module."""
+    import torch
+    u = stack[0]
+    X = _activations(T, u["d"], u["alpha"], u["layer"])
+    Xd = torch.from_numpy(X).cuda()
+    Xb = synth.bits(X)
+    g = np.random.default_rng(100 + T)
+    for i, ((qh, sh, zh), m) in enumerate(zip(u["host"], u["dev"])):
+        As, B = synth.device_factors([qh.shape[0]], u["d"], R, SEED, sub=900 + i)
+        m.A = As[0]
+        Y = glowq.solo_forward(m, B, Xd)
+        torch.cuda.synchronize()
+        n = 512
+        ti, oi = g.integers(0, T, n), g.integers(0, qh.shape[0], n)
+        ref = oracle.module_forward_sampled(qh, sh, zh, synth.bits(As[0].cpu().numpy()), synth.bits(B.cpu().numpy()),
+                                            Xb, ti, oi)
+        err = normwise(Y.cpu().numpy()[ti, oi].astype(np.float64), ref)
+        assert err < TOL, (i, T, err)
