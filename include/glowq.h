@@ -215,6 +215,17 @@ GLOWQ_API glowq_status glowq_error_norms(const float* W, const uint32_t* qweight
    synchronises `stream` first. */
 GLOWQ_API glowq_status glowq_get_device_status(void* stream);
 
+/*
+ * Self-test of the failure path (no counterpart on the pages): enqueues one
+ * single-thread kernel that waits on a shared-memory barrier nobody arrives
+ * on, with the same bounded wait the forward kernels use, limited to `polls`
+ * polls (1..65536).  The wait runs out, the kernel records GLOWQ_ERR_TIMEOUT
+ * in the device status word and returns; the context stays usable.  Returns
+ * GLOWQ_ERR_ARG for polls outside the range, GLOWQ_ERR_CUDA if the launch
+ * fails, else GLOWQ_OK (read the outcome with glowq_get_device_status).
+ */
+GLOWQ_API glowq_status glowq_selftest_wait_timeout(uint32_t polls, void* stream);
+
 /* Static description of a status code. */
 GLOWQ_API const char* glowq_status_string(glowq_status s);
 

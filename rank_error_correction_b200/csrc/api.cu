@@ -11,6 +11,17 @@ namespace glowq {
 
 __device__ unsigned int g_device_status = 0;
 
+// Failure-path self-test: one thread waits, bounded, on a barrier that never
+// completes (its only expected arrival never comes).
+__global__ void selftest_wait_kernel(uint32_t polls, unsigned int* status) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_wait(&bar, 0, status, polls);
+    }
+}
+
 unsigned int* device_status_ptr() {
     static unsigned int* cached[64] = {};
     int dev = 0;
@@ -192,6 +203,14 @@ glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16
         R = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(workspace) + workspace_partial_bytes(T, r));
     }
     return forward_impl(mod, 1, d, B, r, X, T, R, workspace, workspace_bytes, (cudaStream_t)stream);
+}
+
+glowq_status glowq_selftest_wait_timeout(uint32_t polls, void* stream) {
+    if (polls < 1 || polls > 65536) return GLOWQ_ERR_ARG;
+    unsigned int* status = device_status_ptr();
+    if (!status) return GLOWQ_ERR_CUDA;
+    selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(polls, status);
+    return cudaGetLastError() == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
 }
 
 glowq_status glowq_get_device_status(void* stream) {

@@ -60,12 +60,14 @@ def lib() -> C.CDLL:
         L.glowq_select_restore.argtypes = [p, p, p, p, i32, i32, p, p, p]
         L.glowq_error_norms.argtypes = [p, p, p, p, i64, i64, p, p]
         L.glowq_get_device_status.argtypes = [p]
+        L.glowq_selftest_wait_timeout.argtypes = [C.c_uint32, p]
         L.glowq_status_string.argtypes = [st]
         L.glowq_status_string.restype = C.c_char_p
         L.glowq_version.restype = C.c_char_p
         for f in ("glowq_pack_int4", "glowq_dequant_int4", "glowq_group_forward", "glowq_solo_forward",
                   "glowq_solo_forward_noalloc",
-                  "glowq_select_restore", "glowq_error_norms", "glowq_get_device_status"):
+                  "glowq_select_restore", "glowq_error_norms", "glowq_get_device_status",
+                  "glowq_selftest_wait_timeout"):
             getattr(L, f).restype = st
         _lib = L
     return _lib
@@ -260,6 +262,11 @@ def noalloc_scratch_bytes() -> int:
 def device_status(stream=None) -> int:
     """Reads and clears the device status word (0 = ok, 5 = a bounded wait ran out)."""
     return int(lib().glowq_get_device_status(_stream(stream)))
+
+
+def selftest_wait_timeout(polls: int = 4096, stream=None) -> None:
+    """Enqueues the failure-path self-test (a bounded wait that must run out)."""
+    _check(lib().glowq_selftest_wait_timeout(int(polls), _stream(stream)), "glowq_selftest_wait_timeout")
 
 
 # ---------------------------------------------------------------- GlowQ-S ----
