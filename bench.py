@@ -119,6 +119,41 @@ class ClockSampler:
                 "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
 
 
+# ------------------------------------------------------------ replica ranks
+
+class Ranks:
+    """Cross-rank plumbing of a replica run (one process per GPU, no data-path
+    collective): a barrier before every timed region, the max over ranks of
+    every timed figure, and the whole-job rate from the max."""
+
+    def __init__(self, dist=None, device=None):
+        self.dist = dist
+        self.device = device
+
+    @property
+    def world(self) -> int:
+        return self.dist.get_world_size() if self.dist is not None else 1
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, *vals):
+        """Max over ranks of each value (every rank calls this in the same order)."""
+        if self.dist is None:
+            out = [float(v) for v in vals]
+        else:
+            import torch
+            t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=self.device)
+            self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+            out = [float(x) for x in t.tolist()]
+        return out if len(out) > 1 else out[0]
+
+    def rate(self, units_per_rank: float, max_ms: float) -> float:
+        """Whole-job units per second: every rank's units over the slowest rank's time."""
+        return self.world * units_per_rank / (max_ms * 1e-3)
+
+
 # ------------------------------------------------------------------ workload
 
 def build_replicas(n_rep, T, device, seed=0):
@@ -167,7 +202,7 @@ def run_step(rep, io, stream=None):
     glowq.solo_forward(mo[0], Bo, io["X2"], Y=io["Yo"], workspace=io["ws"], stream=stream)
 
 
-def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
+def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True, ranks=None):
     """Time exactly `steps` decode steps replayed from one CUDA graph (value),
     then replay an instrumented copy with event nodes around each call to get
     the per-call durations used for the roofline (event nodes break the
@@ -197,6 +232,8 @@ def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
     if sampler:
         sampler.__enter__()
     torch.cuda.synchronize()
+    if ranks is not None:
+        ranks.barrier()
     with torch.cuda.stream(stream):
         t0.record()
         g.replay()
@@ -233,7 +270,7 @@ def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True):
                 reps=reps, io=io)
 
 
-def time_e2e(T, steps, device, reps, io):
+def time_e2e(T, steps, device, reps, io, ranks=None):
     """Public-API steps with host<->device copies of the step's activations/outputs."""
     import torch
     Xh = io["X"].cpu().pin_memory()
@@ -252,6 +289,8 @@ def time_e2e(T, steps, device, reps, io):
     for i in range(3):
         one(i)
     torch.cuda.synchronize()
+    if ranks is not None:
+        ranks.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record()
@@ -270,7 +309,7 @@ def time_e2e(T, steps, device, reps, io):
 MLP_D, MLP_FFN = 4096, 11008
 
 
-def time_prefill(T, steps, warmup, device, n_rep=2, seed=0, eager_steps=None):
+def time_prefill(T, steps, warmup, device, n_rep=2, seed=0, eager_steps=None, ranks=None):
     """LLaMA-2-7B MLP linears at T tokens: gate/up group + down_proj solo (tcgen05 path).
     With `eager_steps`, run that many plain steps and return None (profiling)."""
     import torch
@@ -324,6 +363,8 @@ def time_prefill(T, steps, warmup, device, n_rep=2, seed=0, eager_steps=None):
     with torch.cuda.stream(stream):
         g.replay()                     # warm replay on the same stream as the timed one
     torch.cuda.synchronize()
+    if ranks is not None:
+        ranks.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -457,7 +498,7 @@ def build_stack13b(device, layers=S13_LAYERS, seed=0):
     return units
 
 
-def time_stack13b(units, T, steps, warmup, device, mode, seed=0):
+def time_stack13b(units, T, steps, warmup, device, mode, seed=0, ranks=None):
     """One token batch through every linear of the stack, captured in one CUDA
     graph.  mode: 'layerwise' (every module its own R_i = X B_i^T), 'glowq'
     (R shared per group, all units corrected) or 'glowq_s' (only the restored
@@ -508,19 +549,21 @@ def time_stack13b(units, T, steps, warmup, device, mode, seed=0):
     with torch.cuda.stream(stream):
         g.replay()                     # warm replay on the same stream as the timed one
     torch.cuda.synchronize()
+    if ranks is not None:
+        ranks.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         t0.record()
         g.replay()
         t1.record()
-    stream.synchronize()
+    torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / steps
     del g
-    return ms
+    return ranks.max(ms) if ranks is not None else ms
 
 
-def stack13b_line(device, warmup):
+def stack13b_line(device, warmup, ranks=None):
     units = build_stack13b(device)
     out = {"workload": "LLaMA-2-13B-shaped linear stack, 40 layers x (Q/K/V group 3x5120x5120, o_proj 5120x5120, "
                        "gate/up group 2x13824x5120, down_proj 5120x13824), INT4 g128 asym, r=64, random-init "
@@ -528,8 +571,10 @@ def stack13b_line(device, warmup):
            "units": len(units), "restored_units": sum(u["restore"] for u in units),
            "context_pages_table3_ttfb_ms_llama2_7b": PAGES_TABLE3_TTFB_MS}
     for T, steps in ((1, 10), (2048, 2)):
-        ms = {mode: time_stack13b(units, T, steps, warmup, device, mode) for mode in ("layerwise", "glowq", "glowq_s")}
-        out[f"T{T}"] = {"ms_per_batch": ms, "tok_s": {k: T / (v * 1e-3) for k, v in ms.items()},
+        ms = {mode: time_stack13b(units, T, steps, warmup, device, mode, ranks=ranks)
+              for mode in ("layerwise", "glowq", "glowq_s")}
+        world = ranks.world if ranks is not None else 1
+        out[f"T{T}"] = {"ms_per_batch": ms, "tok_s": {k: world * T / (v * 1e-3) for k, v in ms.items()},
                         "speedup_vs_layerwise": {k: ms["layerwise"] / v for k, v in ms.items()}}
     del units
     return out
@@ -589,13 +634,13 @@ def main():
     device = torch.device("cuda", local)
     if rank == 0 or not os.path.exists(glowq.LIB_PATH):
         build.build()
-    pg = None
+    ranks = Ranks()
     if world > 1:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=device)
-        pg = dist
-        dist.barrier()
+        ranks = Ranks(dist, device)
+        ranks.barrier()
     glowq.lib()
 
     if args.profile_case:
@@ -603,40 +648,41 @@ def main():
 
     hbm_peak, tf_peak, tf_sust, peak_src = _peaks()
     T = 1
-    res = time_decode(T, args.steps, args.warmup, device, args.replicas, local, want_clocks=(rank == 0))
-    total_ms = res["total_ms"]
-    if pg is not None:
-        t = torch.tensor([total_ms], device=device, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        total_ms = float(t.item())
+    res = time_decode(T, args.steps, args.warmup, device, args.replicas, local, want_clocks=(rank == 0),
+                      ranks=ranks)
+    total_ms, qkv_ms, o_ms = ranks.max(res["total_ms"], res["qkv_ms"], res["o_ms"])
     ms_step = total_ms / args.steps
-    value = world * T * args.steps / (total_ms / 1e3)
+    value = ranks.rate(T * args.steps, total_ms)
     qkv_bytes = group_bytes(QKV_OUTS, D, R_RANK, T)
-    achieved = qkv_bytes / (res["qkv_ms"] * 1e-3) / 1e9
+    achieved = qkv_bytes / (qkv_ms * 1e-3) / 1e9
     launches_per_step = 2 + 2          # (rproj_cluster, corrected_gemv) x 2 calls
-    e2e_ms, h2d, d2h, _ = time_e2e(T, args.steps, device, res["reps"], res["io"])
+    e2e_ms, h2d, d2h, _ = time_e2e(T, args.steps, device, res["reps"], res["io"], ranks=ranks)
+    e2e_ms = ranks.max(e2e_ms)
 
     extra = []
     if not args.no_extra:
         for Tx in (4, 16):
-            r2 = time_decode(Tx, min(args.steps, 100), args.warmup, device, args.replicas, local, want_clocks=False)
+            r2 = time_decode(Tx, min(args.steps, 100), args.warmup, device, args.replicas, local, want_clocks=False,
+                             ranks=ranks)
+            tot2, q2, o2 = ranks.max(r2["total_ms"], r2["qkv_ms"], r2["o_ms"])
             b = group_bytes(QKV_OUTS, D, R_RANK, Tx)
-            extra.append({"tokens": Tx, "tok_s": Tx * min(args.steps, 100) / (r2["total_ms"] / 1e3),
-                          "ms_per_step": r2["total_ms"] / min(args.steps, 100),
-                          "qkv_group_us": r2["qkv_ms"] * 1e3, "o_proj_us": r2["o_ms"] * 1e3,
-                          "qkv_group_GBps": b / (r2["qkv_ms"] * 1e-3) / 1e9,
-                          "qkv_group_hbm_frac": b / (r2["qkv_ms"] * 1e-3) / 1e9 / hbm_peak})
+            extra.append({"tokens": Tx, "tok_s": ranks.rate(Tx * min(args.steps, 100), tot2),
+                          "ms_per_step": tot2 / min(args.steps, 100),
+                          "qkv_group_us": q2 * 1e3, "o_proj_us": o2 * 1e3,
+                          "qkv_group_GBps": b / (q2 * 1e-3) / 1e9,
+                          "qkv_group_hbm_frac": b / (q2 * 1e-3) / 1e9 / hbm_peak})
             del r2
 
     prefill = None
     if not args.no_prefill:
         Tp, sp = 2048, min(args.steps, 20)
-        pr = time_prefill(Tp, sp, args.warmup, device)
+        pr = time_prefill(Tp, sp, args.warmup, device, ranks=ranks)
+        pr["total_ms"], pr["gu_ms"], pr["dn_ms"] = ranks.max(pr["total_ms"], pr["gu_ms"], pr["dn_ms"])
         tf_gu = group_flops([MLP_FFN] * 2, MLP_D, R_RANK, Tp) / (pr["gu_ms"] * 1e-3) / 1e12
         tf_dn = group_flops([MLP_D], MLP_FFN, R_RANK, Tp) / (pr["dn_ms"] * 1e-3) / 1e12
         prefill = {"workload": "LLaMA-2-7B MLP linears, prefill T=2048: gate/up group (2x11008x4096) + "
                                "down_proj solo (4096x11008), INT4 g128, r=64",
-                   "tokens": Tp, "steps": sp, "tok_s": world * Tp * sp / (pr["total_ms"] / 1e3),
+                   "tokens": Tp, "steps": sp, "tok_s": ranks.rate(Tp * sp, pr["total_ms"]),
                    "ms_per_step": pr["total_ms"] / sp,
                    "gate_up_us": pr["gu_ms"] * 1e3, "down_us": pr["dn_ms"] * 1e3,
                    "roofline": {"bound": "tensor", "kernel": "glowq_group_forward (gate/up, T=2048)",
@@ -646,7 +692,7 @@ def main():
 
     stack = None
     if not args.no_stack:
-        stack = stack13b_line(device, args.warmup)
+        stack = stack13b_line(device, args.warmup, ranks=ranks)
 
     cpu = None
     if rank == 0 and not args.no_cpu:
@@ -687,9 +733,9 @@ def main():
             "roofline": {"bound": "hbm", "kernel": "glowq_group_forward (Q/K/V, T=1)", "achieved": achieved,
                          "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s", "frac": achieved / hbm_peak,
                          "traffic": traffic, "algorithmic_bytes": qkv_bytes,
-                         "us_per_launch": res["qkv_ms"] * 1e3},
-            "o_proj_us": res["o_ms"] * 1e3,
-            "e2e": {"value": T / (e2e_ms * 1e-3) * world, "unit": "tok/s", "h2d_bytes_per_step": h2d,
+                         "us_per_launch": qkv_ms * 1e3},
+            "o_proj_us": o_ms * 1e3,
+            "e2e": {"value": ranks.rate(T, e2e_ms), "unit": "tok/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": res["clocks"],
@@ -699,9 +745,9 @@ def main():
             "stack13b": stack,
         }
         print(json.dumps(line), flush=True)
-    if pg is not None:
-        pg.barrier()
-        pg.destroy_process_group()
+    if ranks.dist is not None:
+        ranks.barrier()
+        ranks.dist.destroy_process_group()
     return 0
 
 
