@@ -73,8 +73,10 @@ __host__ __device__ inline bool rc_stage_b(int r, int d) { return r * rc_b_pitch
 // mbarrier
 __host__ __device__ inline int rc_part_bytes(int r, int nt) { return (rc_klanes(r) + 1) * 8 * nt * r * 4; }
 __host__ __device__ inline int rc_x_bytes(int d, int nt) { return 8 * nt * (rc_b_pitch(d) - 16); }
+// the X slice is staged when it fits in 32 KB (wider inputs read X in the loop)
+__host__ __device__ inline bool rc_stage_x(int d, int nt) { return rc_x_bytes(d, nt) <= 32 * 1024; }
 __host__ __device__ inline int rc_smem_bytes(int r, int d, int nt) {
-    const int p = (rc_part_bytes(r, nt) + 15) / 16 * 16 + rc_x_bytes(d, nt);
+    const int p = (rc_part_bytes(r, nt) + 15) / 16 * 16 + (rc_stage_x(d, nt) ? rc_x_bytes(d, nt) : 0);
     return rc_stage_b(r, d) ? p + r * rc_b_pitch(d) + 16 : p;
 }
 
@@ -96,9 +98,10 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
     const int s0 = (int)((int64_t)crank * nsteps / kRcCtas), s1 = (int)((int64_t)(crank + 1) * nsteps / kRcCtas);
     const bool staged = rc_stage_b(r, d);
     const int pitch = rc_b_pitch(d);
+    const bool staged_x = rc_stage_x(d, NT);
     unsigned char* xsl = reinterpret_cast<unsigned char*>(rc_smem) + (rc_part_bytes(r, NT) + 15) / 16 * 16;
     const int xpitch = pitch - 16;               // bytes of one token's slice
-    unsigned char* bs = xsl + rc_x_bytes(d, NT);
+    unsigned char* bs = xsl + (staged_x ? rc_x_bytes(d, NT) : 0);
     uint64_t* bbar = reinterpret_cast<uint64_t*>(bs + r * pitch);
     // B is static: stage (or prefetch) this CTA's slice before the wait
     if (staged) {
@@ -118,7 +121,7 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
     }
     pdl_wait();                 // X may come from the previous kernel in the stream
     // the CTA's slice of X in one round trip (16-byte chunks), padding tokens 0
-    {
+    if (staged_x) {
         const int chunks = xpitch / 16, n = TP * chunks;
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             const int tok = i / chunks, c = i - tok * chunks;
@@ -155,9 +158,14 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
                     bhi[u] = (in && j1 < r) ? ldg_128(B + (int64_t)j1 * d + k) : zero4;
                 }
 #pragma unroll
-                for (int n = 0; n < NT; ++n)
-                    xv[u][n] = in ? *reinterpret_cast<const uint4*>(xsl + (n * 8 + g) * xpitch + (su - s0) * 64 + 16 * t)
-                                  : zero4;
+                for (int n = 0; n < NT; ++n) {
+                    const int tok = n * 8 + g;
+                    if (staged_x)
+                        xv[u][n] = in ? *reinterpret_cast<const uint4*>(xsl + tok * xpitch + (su - s0) * 64 + 16 * t)
+                                      : zero4;
+                    else
+                        xv[u][n] = (in && tok < T) ? ldg_128(X + (int64_t)tok * d + k) : zero4;
+                }
             }
 #pragma unroll
             for (int u = 0; u < U; ++u) {
@@ -747,11 +755,13 @@ cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int
     void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&Rh, (void*)&status};
     const void* fn = (nt == 1) ? (const void*)rproj_cluster_kernel<1> : (const void*)rproj_cluster_kernel<2>;
     const size_t smem = (size_t)rc_smem_bytes(r, d, nt);
-    static bool opted[2] = {false, false};
-    if (smem > 48 * 1024 && !opted[nt - 1]) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRcStageB + 32 * 1024);
+    // opt in to the largest dynamic shared memory requested so far (at most
+    // the staged B slice, the partials of r <= 256 and a 16-token X slice)
+    static size_t opted[2] = {48 * 1024, 48 * 1024};
+    if (smem > opted[nt - 1]) {
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        opted[nt - 1] = true;
+        opted[nt - 1] = smem;
     }
     return launch_ex(fn, dim3(kRcCtas), dim3(kRcWarps * 32), smem, st, true, a1);
 }

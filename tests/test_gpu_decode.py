@@ -245,3 +245,35 @@ def test_llama31_8b_layer_decode_t1():
     ref = oracle.solo_forward(down[0].q, down[0].s, down[0].z, synth.bits(down[0].A), synth.bits(Bd),
                               synth.bits(Xd))
     assert normwise(Y.astype(np.float64), ref) < TOL
+
+
+@pytest.mark.parametrize("T", [1, 16])
+@pytest.mark.parametrize("r", [8, 256])
+def test_decode_rank_extremes_and_eight_modules(T, r):
+    """Smallest and largest rank with the largest group (8 modules, 16..128 rows)."""
+    import torch
+    d = 1024
+    outs = [16, 32, 48, 64, 80, 96, 112, 128]
+    mods = make_modules(d, outs, seed=60 + r + T)
+    B = attach_random_factors(mods, d, r, seed=60 + r + T)
+    X = synth.activations(T, d, synth.ALPHA_QKV, seed=60 + T)
+    Ys, R = glowq.group_forward(to_dev(mods), torch.from_numpy(B).cuda(), torch.from_numpy(X).cuda())
+    torch.cuda.synchronize()
+    Rr = oracle.anchor_project(synth.bits(X), synth.bits(B))
+    assert normwise(R.cpu().numpy().astype(np.float64), Rr) < 1e-3
+    for m, Y in zip(mods, Ys):
+        ref = oracle.module_forward(m.q, m.s, m.z, synth.bits(m.A), Rr, synth.bits(X))
+        assert normwise(Y.cpu().numpy().astype(np.float64), ref) < TOL
+
+
+def test_decode_wide_input_solo():
+    """LLaMA-3.1-8B down_proj shape at T=1: 4096 x 14336 (R's B slice too wide to stage)."""
+    import torch
+    d, O, r, T = 14336, 4096, 64, 1
+    mods = make_modules(d, [O], seed=65)
+    B = attach_random_factors(mods, d, r, seed=65)
+    X = synth.activations(T, d, synth.ALPHA_MLP, seed=65)
+    Y = glowq.solo_forward(to_dev(mods)[0], torch.from_numpy(B).cuda(), torch.from_numpy(X).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.solo_forward(mods[0].q, mods[0].s, mods[0].z, synth.bits(mods[0].A), synth.bits(B), synth.bits(X))
+    assert normwise(Y.cpu().numpy().astype(np.float64), ref) < TOL
