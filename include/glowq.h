@@ -110,12 +110,20 @@ GLOWQ_API glowq_status glowq_dequant_int4(const uint32_t* qweight, const uint16_
                                 int32_t group_size, uint16_t* W_deq, void* stream);
 
 /*
- * Bytes of device scratch the forward calls need for T tokens at rank r: for
- * T > 16 the fp32 partial sums of R = X B^T split along d into up to 8 slices
- * (added in a fixed order, so R does not depend on timing), plus the solo
- * call's R.  0 when r == 0.  The caller allocates it once and may reuse it
- * across calls issued in order on one stream; calls that may overlap need
- * separate workspaces.
+ * Bytes of device scratch the forward calls need for T tokens at rank r:
+ *   - 256 bytes of hand-off flags at offset 0, through which the decode GEMV
+ *     (T <= 16) learns, while it already streams weights, that the kernel
+ *     computing R = X B^T has seen X final and has stored R;
+ *   - for T > 16, the fp32 partial sums of R split along d into up to 8 slices
+ *     (added in a fixed order, so R does not depend on timing);
+ *   - the solo call's R.
+ * 0 when r == 0 or T == 0.  The caller allocates it once and may reuse it
+ * across calls issued in order on one stream (any T); calls that may overlap
+ * need separate workspaces.  Ownership: caller's device memory, 16-byte
+ * aligned.  The first 256 bytes must be zero before the first call that uses
+ * the workspace; every call that completes leaves them zero.  After a call
+ * returned GLOWQ_ERR_CUDA, or glowq_get_device_status reported
+ * GLOWQ_ERR_TIMEOUT, zero them again.
  */
 GLOWQ_API size_t glowq_workspace_bytes(int64_t T, int32_t r);
 

@@ -44,6 +44,11 @@ static int device_sm_count() {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Workspace layout (r > 0): [hand-off flags, 256 B][prefill partials][solo R].
+// The flags are the decode kernels' (R kernel -> GEMV) and sit at offset 0 for
+// every T, so a prefill call sharing the workspace never overwrites them.
+static size_t workspace_flag_bytes(int32_t r) { return r > 0 ? 256 : 0; }
+
 // fp32 partial sums of R = X B^T for T > 16 (split along d into up to 8
 // slices when the token tiles alone would not fill the GPU); the decode path
 // reduces its partial sums on chip.
@@ -93,16 +98,19 @@ static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d,
     }
     const bool use_r = r > 0;
     if (T <= kDecodeMaxTokens) {
+        unsigned int* flags = use_r ? reinterpret_cast<unsigned int*>(workspace) : nullptr;
         if (use_r) {
-            cudaError_t e = launch_rproj_decode(X, B, (int)T, (int)d, r, R, st);
+            cudaError_t e = launch_rproj_decode(X, B, (int)T, (int)d, r, R, flags, st);
             if (e != cudaSuccess) return GLOWQ_ERR_CUDA;
         }
-        cudaError_t e = launch_gemv_decode(hm, m, (int)d, (int)T, use_r ? r : 0, X, R, use_r, device_sm_count(), st);
+        cudaError_t e = launch_gemv_decode(hm, m, (int)d, (int)T, use_r ? r : 0, X, R, flags, device_sm_count(), st);
         return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
     }
     (void)any_A;
-    float* partial = (use_r && workspace && ws_bytes >= workspace_partial_bytes(T, r))
-                         ? reinterpret_cast<float*>(workspace) : nullptr;
+    (void)ws_bytes;
+    float* partial = (use_r && workspace_partial_bytes(T, r) > 0)
+                         ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + workspace_flag_bytes(r))
+                         : nullptr;
     return prefill_group_forward(hm, m, (int)d, use_r ? B : nullptr, use_r ? r : 0, X, T, R, partial,
                                  device_sm_count(), st);
 }
@@ -170,8 +178,8 @@ glowq_status glowq_error_norms(const float* W, const uint32_t* qweight, const ui
 }
 
 size_t glowq_workspace_bytes(int64_t T, int32_t r) {
-    if (T < 0 || r < 0) return 0;
-    return workspace_partial_bytes(T, r) + workspace_solo_R_bytes(T, r);
+    if (T <= 0 || r <= 0) return 0;
+    return workspace_flag_bytes(r) + workspace_partial_bytes(T, r) + workspace_solo_R_bytes(T, r);
 }
 
 glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
@@ -183,9 +191,9 @@ glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d,
     if (r > 0) {
         if (!R_out) return GLOWQ_ERR_ARG;
         if (!aligned16(R_out)) return GLOWQ_ERR_ALIGN;
-        const size_t need = workspace_partial_bytes(T, r);
-        if (need > 0 && (!workspace || workspace_bytes < need)) return GLOWQ_ERR_ARG;
-        if (workspace && !aligned16(workspace)) return GLOWQ_ERR_ALIGN;
+        const size_t need = workspace_flag_bytes(r) + workspace_partial_bytes(T, r);
+        if (!workspace || workspace_bytes < need) return GLOWQ_ERR_ARG;
+        if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
     }
     return forward_impl(mods, m, d, B, r, X, T, R_out, workspace, workspace_bytes, (cudaStream_t)stream);
 }
@@ -200,7 +208,8 @@ glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16
         const size_t need = glowq_workspace_bytes(T, r);
         if (!workspace || workspace_bytes < need) return GLOWQ_ERR_ARG;
         if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
-        R = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(workspace) + workspace_partial_bytes(T, r));
+        R = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(workspace) + workspace_flag_bytes(r) +
+                                        workspace_partial_bytes(T, r));
     }
     return forward_impl(mod, 1, d, B, r, X, T, R, workspace, workspace_bytes, (cudaStream_t)stream);
 }

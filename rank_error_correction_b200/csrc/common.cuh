@@ -40,6 +40,45 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
 __device__ __forceinline__ uint4 ldg_128(const void* p) {
     return __ldg(reinterpret_cast<const uint4*>(p));
 }
+// Loads served by L2 (never by a possibly stale L1 line) for data that a kernel
+// overlapping this one may have written: activations produced before a
+// programmatic launch, R produced by a concurrently running kernel.
+__device__ __forceinline__ uint4 ldcg_128(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ uint2 ldcg_64(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
+    return v;
+}
+
+// ---- flags in global memory between concurrently running kernels ----------
+// Release: this thread's earlier writes (and those it has observed) become
+// visible to any thread that acquires the incremented value.
+__device__ __forceinline__ void flag_release_add(unsigned int* f, unsigned int v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(f), "r"(v) : "memory");
+}
+__device__ __forceinline__ unsigned int flag_acquire_load(const unsigned int* f) {
+    unsigned int v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(f) : "memory");
+    return v;
+}
+// Bounded wait until *f >= target.  Returns false (and records
+// GLOWQ_ERR_TIMEOUT) if the value was not reached within `limit` polls.
+__device__ __forceinline__ bool flag_wait_geq(const unsigned int* f, unsigned int target, unsigned int* status,
+                                              uint32_t limit = (1u << 22)) {
+    for (uint32_t it = 0; it < limit; ++it) {
+        if (flag_acquire_load(f) >= target) return true;
+        if (it >= 64) __nanosleep(64);
+    }
+    record_status(status, GLOWQ_ERR_TIMEOUT);
+    return false;
+}
 
 // ---- mbarriers and bulk (TMA) copies --------------------------------------
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -55,6 +94,10 @@ __device__ __forceinline__ void fence_mbar_init() {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
+}
+// Arrive (release, CTA scope) on an mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 // Bounded wait for the phase with the given parity to complete.  Returns false
 // (and records GLOWQ_ERR_TIMEOUT) if it did not complete within `limit` polls.
@@ -88,6 +131,22 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, uint6
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// L2 policy for data read exactly once per call (decode weight streams): its
+// lines are the first evicted, so activations, flags and R stay resident.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+// 2-D tiled TMA load with an L2 cache policy.
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const void* map, uint64_t* bar, int x, int y,
+                                                 uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
 }
 // Order this thread's earlier generic-proxy shared-memory accesses before

@@ -52,6 +52,16 @@ namespace glowq {
 // while the preceding GEMV still runs: B is static, so its slice is copied
 // into shared memory (or, when it does not fit, pulled into L2) before the
 // wait on the preceding kernel; after the wait only X is read from memory.
+//
+// Hand-off to the GEMV that follows (flags = three zeroed words):
+//   flags[0]  each CTA adds 1 once its wait has returned (X is final), and only
+//             then allows the GEMV to launch, so the GEMV streams weights and
+//             runs its main loop while R is still being computed;
+//   flags[1]  each CTA adds 1 after its part of R is stored; the GEMV reads R
+//             in its epilogue only after seeing kRcCtas here;
+//   flags[2]  counts GEMV CTAs past both waits; the last one zeroes all three.
+// A GEMV launched without the programmatic attribute starts after this kernel
+// has completed and finds both counts already reached.
 // ---------------------------------------------------------------------------
 constexpr int kRcCtas = 8;
 constexpr int kRcWarps = 8;
@@ -83,8 +93,7 @@ __host__ __device__ inline int rc_smem_bytes(int r, int d, int nt) {
 template <int NT>
 __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32, 4)
     rproj_cluster_kernel(const __half* __restrict__ X, const __half* __restrict__ B, int T, int d, int r,
-                         __half* __restrict__ R, unsigned int* status) {
-    pdl_launch_dependents();    // the GEMV may start streaming weights now
+                         __half* __restrict__ R, unsigned int* flags, unsigned int* status) {
     extern __shared__ __align__(16) float rc_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
@@ -120,13 +129,15 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
                          : "memory");
     }
     pdl_wait();                 // X may come from the previous kernel in the stream
+    if (flags && threadIdx.x == 0) flag_release_add(flags + 0, 1u);
+    pdl_launch_dependents();    // the GEMV may start streaming weights now
     // the CTA's slice of X in one round trip (16-byte chunks), padding tokens 0
     if (staged_x) {
         const int chunks = xpitch / 16, n = TP * chunks;
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             const int tok = i / chunks, c = i - tok * chunks;
             uint4 v = make_uint4(0, 0, 0, 0);
-            if (tok < T && s0 * 32 + c * 8 < s1 * 32) v = ldg_128(X + (int64_t)tok * d + s0 * 32 + c * 8);
+            if (tok < T && s0 * 32 + c * 8 < s1 * 32) v = ldcg_128(X + (int64_t)tok * d + s0 * 32 + c * 8);
             *reinterpret_cast<uint4*>(xsl + tok * xpitch + c * 16) = v;
         }
     }
@@ -164,7 +175,7 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
                         xv[u][n] = in ? *reinterpret_cast<const uint4*>(xsl + tok * xpitch + (su - s0) * 64 + 16 * t)
                                       : zero4;
                     else
-                        xv[u][n] = (in && tok < T) ? ldg_128(X + (int64_t)tok * d + k) : zero4;
+                        xv[u][n] = (in && tok < T) ? ldcg_128(X + (int64_t)tok * d + k) : zero4;
                 }
             }
 #pragma unroll
@@ -218,6 +229,8 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
     }
     // no CTA leaves while another may still read its shared memory
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    // this CTA's stores of R (ordered before thread 0 by the barrier) are published
+    if (flags && threadIdx.x == 0) flag_release_add(flags + 1, 1u);
 }
 
 // ---------------------------------------------------------------------------
@@ -246,14 +259,24 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
 //   xs   [T+1][wpt_max] uint4        the CTA's activation slice (row T all zero,
 //                                    read by the lanes of padding tokens); each
 //                                    8-element word stored as the half2 pairs
-//                                    (x0,x4) (x1,x5) (x2,x6) (x3,x7) of the MMA B
+//                                    (x0,x4) (x2,x6) (x1,x5) (x3,x7) of the MMA B
 //                                    fragment, word index XOR-swizzled
 //   xsum [ncta_max][8*NT] f32        per-group activation sums S (0 for padding)
 //   sz   [warps][16][nsub_max+1] f32x2  (s, 64 + z) of the warp's rows and groups
 //   red  [nslots][NT*4][32] f32      partial sums sent to the finalising warp
 //   as   [fin_slots][16][r+8] f16    A rows of the tiles this CTA finalises
+//   rs   [8*NT][r+8] f16             R of the call (rows of padding tokens zero)
+//   rbar u64                         completes when rs holds R
+//
+// Besides its rt * kw compute warps a CTA has one control warp.  It waits until
+// X is final (the R kernel's flags[0], or the preceding grid), then, while the
+// compute warps run the main loop, until R is stored (flags[1]); it copies R
+// into shared memory for the epilogue and, as the last CTA to get there,
+// returns the flags to zero.  The hand-off latency thus stays off the weight
+// stream and out of the epilogue.
 // ---------------------------------------------------------------------------
-constexpr int kMaxWarps = 12;   // 12 x 32 x 128 registers leave room for an R CTA on the SM
+constexpr int kMaxWarps = 11;   // compute warps; with the control warp 12 x 32 x 128 registers
+                                // leave room for an R CTA on the SM
 // Pipeline stages per warp (one 2-D TMA box of 16 rows x 2 groups of 128,
 // 2 KB) are a template parameter S in {4, 8}: the host trades ring depth
 // against resident warps.
@@ -282,11 +305,13 @@ struct GemvArgs {
     int kc;            // CTAs per cluster splitting d (kw == 1 when kc > 1)
     const __half* X;   // T x d
     const __half* R;   // T x r (read after the wait)
+    unsigned int* flags;    // hand-off words of the R kernel (nullptr: wait for the preceding grid)
+    int nflag;              // count each flag reaches (CTAs of the R kernel)
     unsigned int* status;   // device status word (bounded-wait timeouts)
 };
 
 struct GemvLayout {    // byte offsets into dynamic shared memory
-    int xs, xsum, sz, red, as, total;
+    int xs, xsum, sz, red, as, rs, rbar, total;
     int wpt_max, ncta_max, nsub_max, fin_slots;
 };
 
@@ -321,7 +346,13 @@ __host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, i
     off += nslots * nt * 4 * 32 * 4;
     L.as = off;
     off += (r > 0) ? L.fin_slots * 16 * (r + 8) * 2 : 0;
-    L.total = (off + 15) / 16 * 16;
+    off = (off + 15) / 16 * 16;
+    L.rs = off;
+    off += (r > 0) ? 8 * nt * (r + 8) * 2 : 0;
+    off = (off + 15) / 16 * 16;
+    L.rbar = off;
+    off += 16;
+    L.total = off;
     return L;
 }
 
@@ -354,14 +385,18 @@ __device__ __forceinline__ void unpack_even_odd(uint32_t w, uint32_t ev[2], uint
     od[1] = (w8 & 0x00F000F0u) | 0x54005400u;
 }
 
-template <int NT, int S>
+template <int NT, int S, bool ONE>
 // (the bound of 512 threads caps registers at 128 per thread; launches use at
-// most kMaxWarps warps)
+// most kMaxWarps compute warps and the control warp).  ONE: T == 1, so only the
+// first column of each MMA tile (lanes t == 0, elements 0 and 2) is finished.
 __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_constant__ GemvArgs args,
                                                                            const __grid_constant__ GemvPlan plan) {
     pdl_launch_dependents();
     extern __shared__ __align__(1024) unsigned char smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the weight streams' TMA descriptors into the descriptor cache
+    if (threadIdx.x < GLOWQ_MAX_MODULES && (int)threadIdx.x < args.m)
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&args.tmq[threadIdx.x])) : "memory");
     const int g = lane >> 2, t = lane & 3;
     const int rt = args.rt, kw = args.kw, kc = args.kc;
     const int warps = rt * kw;
@@ -375,6 +410,9 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     float2* szs = reinterpret_cast<float2*>(smem + L.sz);
     float* red = reinterpret_cast<float*>(smem + L.red);
     __half* as = reinterpret_cast<__half*>(smem + L.as);
+    __half* rs = reinterpret_cast<__half*>(smem + L.rs);
+    uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + L.rbar);
+    const bool control = warp == warps;         // the last warp: hand-off with the R kernel
 
     const int crank = blockIdx.x % kc;          // rank in the cluster (cluster dims (kc,1,1))
     const int block = blockIdx.x / kc;
@@ -382,25 +420,57 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     const int ncta = C1 - C0;
     const int wpt = ncta * 16;                  // 8-element words per token in the CTA's slice
     const int tl = warp % rt, ks = warp / rt;   // tile within the CTA, split index
-    const int G0 = plan.gsplit[crank * kw + ks];
-    const int G1 = plan.gsplit[crank * kw + ks + 1];
+    const int G0 = control ? 0 : plan.gsplit[crank * kw + ks];
+    const int G1 = control ? 0 : plan.gsplit[crank * kw + ks + 1];
     const int tile = block * rt + tl;
-    const bool active = tile < args.num_tiles;
-    int mi = 0;
-    for (int i = 1; i < args.m; ++i)
-        if (tile >= args.mod[i].tile_begin) mi = i;
+    const bool active = !control && tile < args.num_tiles;
+    // The module of this warp's tile.  Kernel parameters are read through the
+    // constant cache, cold at every launch: the lookup reads every module's
+    // first tile and scale / zero pointers unconditionally (independent loads,
+    // one round of misses) rather than a chain of dependent reads.
+    int mi = 0, tb = 0;
+    const __half* Ms = args.mod[0].s;
+    const uint8_t* Mz = args.mod[0].z;
+#pragma unroll
+    for (int i = 1; i < GLOWQ_MAX_MODULES; ++i) {
+        const int b = args.mod[i].tile_begin;
+        const __half* si = args.mod[i].s;
+        const uint8_t* zi = args.mod[i].z;
+        if (i < args.m && tile >= b) {
+            mi = i;
+            tb = b;
+            Ms = si;
+            Mz = zi;
+        }
+    }
     const GemvModule& M = args.mod[mi];
-    const int tile_row = (tile - M.tile_begin) * 16;
+    const int tile_row = (tile - tb) * 16;
     const int row_lo = tile_row + g, row_hi = row_lo + 8;
     // the warp that finalises this tile: split 0 of the owner CTA of the cluster
     const int owner = (kc > 1) ? tl % kc : 0;
     const int fslot = (kc > 1) ? tl / kc : tl;
-    const bool finaliser = ks == 0 && owner == crank;
+    const bool finaliser = !control && ks == 0 && owner == crank;
     const bool has_corr = r > 0 && M.A != nullptr;
 
+    // 1) start the weight stream first: per warp, S mbarriers; lane 0 issues
+    //    one 2-D TMA box (16 rows x 2 groups) per stage
+    constexpr int kStages = S;
+    uint64_t* my_bars = bars + warp * kStages;
+    unsigned char* my_ring = ring + warp * kStages * 2048;
+    const uint32_t ring_smem = smem_u32(my_ring);
+    const CUtensorMap* tmq = &args.tmq[mi];
+    const int nsub = G1 - G0;
+    const int npairs = (nsub + 1) / 2;
+    // the barriers are initialised and fenced while this thread has no memory
+    // operation outstanding (the release fence would wait for it)
+    if (active && lane == 0) {
+        for (int i = 0; i < kStages; ++i) mbar_init(my_bars + i, 1);
+        fence_mbar_init();
+    }
     // 0) this warp's scales and zeros are the longest-latency reads of the
     //    prologue (scattered, cold): a split of at most 32 groups is loaded in
-    //    one batch before the weight stream is started, and staged below
+    //    one batch ahead of the weight stream (behind it, they would queue
+    //    after every stage in flight), and staged below
     const int sz_stride = L.nsub_max + 1;
     float2* my_sz = szs + warp * 16 * sz_stride;
     const int rr = lane & 15;   // lane -> row (lane & 15) and every other group starting at lane >> 4
@@ -414,28 +484,19 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         for (int j = 0; j < 16; ++j) {
             const int gg = (lane >> 4) + 2 * j;
             if (gg < nsub0) {
-                sv[j] = __half_as_ushort(M.s[sz_base + gg]);
-                zv[j] = M.z[sz_base + gg];
+                sv[j] = __half_as_ushort(Ms[sz_base + gg]);
+                zv[j] = Mz[sz_base + gg];
             }
         }
     }
 
-    // 1) start the weight stream: per warp, S mbarriers; lane 0 issues one 2-D
-    //    TMA box (16 rows x 2 groups) per stage
-    constexpr int kStages = S;
-    uint64_t* my_bars = bars + warp * kStages;
-    unsigned char* my_ring = ring + warp * kStages * 2048;
-    const uint32_t ring_smem = smem_u32(my_ring);
-    const CUtensorMap* tmq = &args.tmq[mi];
-    const int nsub = G1 - G0;
-    const int npairs = (nsub + 1) / 2;
+    // 1') start the weight stream (read once per call: evict-first in L2)
+    const uint64_t wpol = l2_policy_evict_first();
     if (active) {
         if (lane == 0) {
-            for (int i = 0; i < kStages; ++i) mbar_init(my_bars + i, 1);
-            fence_mbar_init();
             for (int i = 0; i < kStages && i < npairs; ++i) {
                 mbar_arrive_expect_tx(my_bars + i, 2048u);
-                tma_load_2d(ring_smem + i * 2048, tmq, my_bars + i, (G0 + 2 * i) * 16, tile_row);
+                tma_load_2d_hint(ring_smem + i * 2048, tmq, my_bars + i, (G0 + 2 * i) * 16, tile_row, wpol);
             }
         }
         __syncwarp();
@@ -466,8 +527,8 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
             for (int j = 0; j < 16; ++j) {
                 const int gg = g0 + 2 * j;
                 if (gg < nsub) {
-                    sv[j] = __half_as_ushort(M.s[sz_base + gg]);
-                    zv[j] = M.z[sz_base + gg];
+                    sv[j] = __half_as_ushort(Ms[sz_base + gg]);
+                    zv[j] = Mz[sz_base + gg];
                 }
             }
 #pragma unroll
@@ -479,61 +540,105 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         }
     }
     // Everything above reads only static weight data; activations (and R) may
-    // be produced by the preceding kernels, so wait for them here (a no-op when
-    // launched without programmatic serialization).
-    pdl_wait();
-    // 3) the CTA's activation slice, paired and swizzled (all loads of a batch first)
-    const int stride = warps * 32;
+    // be produced by the preceding kernels.  After an R kernel, X is final once
+    // every R CTA has passed its own wait (flags[0]), which the control warp
+    // awaits meanwhile; R itself is awaited only during the main loop.  Without
+    // flags, wait for the preceding grid (a no-op when launched without
+    // programmatic serialization).
+    if (control && lane == 0) {
+        mbar_init(rbar, 1);
+        if (args.flags) flag_wait_geq(args.flags + 0, (unsigned)args.nflag, args.status);
+    }
+    if (!args.flags) pdl_wait();
+    __syncthreads();   // X is final; rbar is initialised
+    // 3) the CTA's activation slice, paired and swizzled (all loads of a batch
+    //    first); every thread of the CTA, the control warp included, takes part
+    const int stride = (int)blockDim.x;
     {
         const int items = T * wpt;
-        for (int base = threadIdx.x; base < items; base += 4 * stride) {
+        // warp-uniform trip count: every lane reaches the shuffles below
+        for (int b0 = (int)threadIdx.x - lane; b0 < items; b0 += 4 * stride) {
+            const int base = b0 + lane;
             uint4 v[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int i = base + j * stride;
                 if (i < items) {
                     const int tok = i / wpt, wd = i - tok * wpt;
-                    v[j] = ldg_128(args.X + (int64_t)tok * d + (int64_t)C0 * 128 + wd * 8);
+                    v[j] = ldcg_128(args.X + (int64_t)tok * d + (int64_t)C0 * 128 + wd * 8);
                 }
             }
+            // 4) with each word, its even / odd activation sums; the 16 words of
+            //    a (token, group) are held by 16 consecutive lanes (stride and
+            //    wpt are multiples of 16), which add them in a fixed butterfly
+            //    order into S_E and S_O: xsum[(2 * group + e)][token]
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int i = base + j * stride;
+                float se = 0.f, so = 0.f;
                 if (i < items) {
                     const int tok = i / wpt, wd = i - tok * wpt;
                     uint4 p;
                     p.x = pair_lo(v[j].x, v[j].z);   // (x0,x4)
-                    p.y = pair_hi(v[j].x, v[j].z);   // (x1,x5)
-                    p.z = pair_lo(v[j].y, v[j].w);   // (x2,x6)
+                    p.y = pair_lo(v[j].y, v[j].w);   // (x2,x6)
+                    p.z = pair_hi(v[j].x, v[j].z);   // (x1,x5)
                     p.w = pair_hi(v[j].y, v[j].w);   // (x3,x7)
                     // swizzle: XOR the two low bits of the word with (bit 3, token parity)
                     xs[tok * wpt + (wd ^ (((wd >> 3) & 1) | ((tok & 1) << 1)))] = p;
+                    const float2 f0 = __half22float2(u32_as_h2(p.x)), f2 = __half22float2(u32_as_h2(p.y));
+                    const float2 f1 = __half22float2(u32_as_h2(p.z)), f3 = __half22float2(u32_as_h2(p.w));
+                    se = (f0.x + f0.y) + (f2.x + f2.y);
+                    so = (f1.x + f1.y) + (f3.x + f3.y);
+                }
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1) {
+                    se += __shfl_xor_sync(0xffffffffu, se, o);
+                    so += __shfl_xor_sync(0xffffffffu, so, o);
+                }
+                if (i < items && (lane & 15) == 0) {
+                    const int tok = i / wpt, gc = (i - tok * wpt) >> 4;
+                    xsum[(2 * gc) * 8 * NT + tok] = se;
+                    xsum[(2 * gc + 1) * 8 * NT + tok] = so;
                 }
             }
         }
         for (int i = threadIdx.x; i < wpt; i += stride) xs[T * wpt + i] = make_uint4(0, 0, 0, 0);
-    }
-    __syncthreads();
-    // 4) per-group activation sums over even and odd k, S_E and S_O (fixed
-    //    summation order; 0 for padding tokens): xsum[(2 * group + e)][token]
-    for (int i = threadIdx.x; i < ncta * 8 * NT; i += stride) {
-        const int gc = i / (8 * NT), tok = i - gc * (8 * NT);
-        float se = 0.f, so = 0.f;
-        if (tok < T) {
-            const uint4* src = xs + tok * wpt + gc * 16;
-#pragma unroll 4
-            for (int wd = 0; wd < 16; ++wd) {
-                const uint4 v = src[wd];   // (x0,x4) (x1,x5) (x2,x6) (x3,x7)
-                const float2 f0 = __half22float2(u32_as_h2(v.x)), f1 = __half22float2(u32_as_h2(v.y));
-                const float2 f2 = __half22float2(u32_as_h2(v.z)), f3 = __half22float2(u32_as_h2(v.w));
-                se += (f0.x + f0.y) + (f2.x + f2.y);
-                so += (f1.x + f1.y) + (f3.x + f3.y);
-            }
+        // padding tokens: zero sums
+        for (int i = threadIdx.x; i < ncta * (8 * NT - T); i += stride) {
+            const int gc = i / (8 * NT - T), tok = T + (i - gc * (8 * NT - T));
+            xsum[(2 * gc) * 8 * NT + tok] = 0.f;
+            xsum[(2 * gc + 1) * 8 * NT + tok] = 0.f;
         }
-        xsum[(2 * gc) * 8 * NT + tok] = se;
-        xsum[(2 * gc + 1) * 8 * NT + tok] = so;
     }
     __syncthreads();
+
+    // 5a) the control warp: once R is stored, copy it into rs (padding tokens
+    //     zero) and complete rbar; the last CTA here zeroes the flags, which the
+    //     next call's R kernel writes only after this grid has completed
+    if (control && r > 0) {
+        if (args.flags && lane == 0) flag_wait_geq(args.flags + 1, (unsigned)args.nflag, args.status);
+        __syncwarp();
+        const int cpr = r / 8;   // 16-byte chunks per row
+        for (int c = lane; c < 8 * NT * cpr; c += 32) {
+            const int tok = c / cpr, cc = c - tok * cpr;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (tok < T) v = ldcg_128(args.R + (int64_t)tok * r + cc * 8);
+            *reinterpret_cast<uint4*>(rs + tok * (r + 8) + cc * 8) = v;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            if (args.flags) {
+                unsigned int prev;
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(args.flags + 2) : "memory");
+                if (prev == gridDim.x - 1) {
+                    args.flags[0] = 0u;
+                    args.flags[1] = 0u;
+                    args.flags[2] = 0u;
+                }
+            }
+            mbar_arrive(rbar);
+        }
+    }
 
     // 5) main loop: two independent MMA chains per 128-group on (64 + q) x,
     //    then s * (D - (64 + z) S) in fp32
@@ -576,7 +681,8 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                         __syncwarp();
                         if (lane == 0) {
                             mbar_arrive_expect_tx(my_bars + i, 2048u);
-                            tma_load_2d(ring_smem + i * 2048, tmq, my_bars + i, (G0 + 2 * (p + kStages)) * 16, tile_row);
+                            tma_load_2d_hint(ring_smem + i * 2048, tmq, my_bars + i, (G0 + 2 * (p + kStages)) * 16,
+                                             tile_row, wpol);
                         }
                     }
                     const bool two = 2 * p + 1 < nsub;    // warp-uniform
@@ -598,8 +704,8 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
 #pragma unroll
                             for (int n = 0; n < NT; ++n) {
                                 const uint4 x = xrow[n][gl * 16 + ((4 * t + w) ^ xsw)];
-                                const uint32_t be[2] = {x.x, x.z};   // (x0,x4) (x2,x6)
-                                const uint32_t bo[2] = {x.y, x.w};   // (x1,x5) (x3,x7)
+                                const uint32_t be[2] = {x.x, x.y};   // (x0,x4) (x2,x6)
+                                const uint32_t bo[2] = {x.z, x.w};   // (x1,x5) (x3,x7)
                                 if (w == 0) {
                                     mma_16816_zc(te[n], ae, be);
                                     mma_16816_zc(to[n], ao, bo);
@@ -616,6 +722,15 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                         for (int n = 0; n < NT; ++n) {
                             const float2 se = *reinterpret_cast<const float2*>(xsum_w + (2 * gl) * 8 * NT + n * 8);
                             const float2 so = *reinterpret_cast<const float2*>(xsum_w + (2 * gl + 1) * 8 * NT + n * 8);
+                            if (ONE) {
+                                float v0 = fmaf(64.0f, te[n][0], to[n][0]);
+                                float v2 = fmaf(64.0f, te[n][2], to[n][2]);
+                                v0 = fmaf(-zl.y, so.x, fmaf(-cel, se.x, v0));
+                                v2 = fmaf(-zh.y, so.x, fmaf(-ceh, se.x, v2));
+                                acc[n][0] = fmaf(zl.x, v0, acc[n][0]);
+                                acc[n][2] = fmaf(zh.x, v2, acc[n][2]);
+                                continue;
+                            }
                             float v0 = fmaf(64.0f, te[n][0], to[n][0]);
                             float v1 = fmaf(64.0f, te[n][1], to[n][1]);
                             float v2 = fmaf(64.0f, te[n][2], to[n][2]);
@@ -637,11 +752,14 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     cp_async_wait<0>();
     __syncwarp();   // A rows copied by other lanes of this warp are visible
 
+
     // 6) split-d reduction in a fixed order, into the finalising warp
     if (kc > 1) {
         // cluster: partials of tile tl go to rank tl % kc, slot [crank][tl / kc]
         const int idx0 = (crank * L.fin_slots + fslot) * NT * 4 * 32 + lane;
-        if (owner != crank) {
+        if (control) {
+            // no partial sums; only the cluster barrier below
+        } else if (owner != crank) {
             const uint32_t local = (uint32_t)__cvta_generic_to_shared(red);
             uint32_t remote;
             asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(owner));
@@ -670,10 +788,12 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
             }
     } else if (kw > 1) {
         // in-CTA: partials of tile tl from split ks at slot [ks][tl]
+        if (!control) {
 #pragma unroll
-        for (int n = 0; n < NT; ++n)
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) red[((ks * rt + tl) * NT * 4 + n * 4 + i) * 32 + lane] = acc[n][i];
+                for (int i = 0; i < 4; ++i) red[((ks * rt + tl) * NT * 4 + n * 4 + i) * 32 + lane] = acc[n][i];
+        }
         __syncthreads();
         if (!finaliser) return;
 #pragma unroll
@@ -688,7 +808,9 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     if (!active) return;
 
     // 7) rank-r correction A_i R^T, accumulated into the same fp32 registers
+    //    (R from shared memory, staged by the control warp)
     if (has_corr) {
+        mbar_wait(rbar, 0u, args.status);
         const __half* a_lo = as + (fslot * 16 + g) * (r + 8);
         const __half* a_hi = a_lo + 8 * (r + 8);
         for (int kb = 0; kb < r; kb += 16) {
@@ -702,9 +824,9 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
             const uint32_t a[4] = {al.x, ah.x, al.y, ah.y};
 #pragma unroll
             for (int n = 0; n < NT; ++n) {
-                const int tok = n * 8 + g;
+                const int tok = n * 8 + g;   // rows of padding tokens are zero in rs
                 uint2 rv = make_uint2(0, 0);
-                if (kval && tok < T) rv = __ldg(reinterpret_cast<const uint2*>(args.R + (int64_t)tok * r + k));
+                if (kval) rv = *reinterpret_cast<const uint2*>(rs + tok * (r + 8) + k);
                 const uint32_t b[2] = {rv.x, rv.y};
                 mma_16816(acc[n], a, b);
             }
@@ -746,13 +868,13 @@ static cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem,
 
 // R = X B^T into R (fp16) with one cluster of kRcCtas CTAs.
 cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, uint16_t* R,
-                                cudaStream_t st) {
+                                unsigned int* flags, cudaStream_t st) {
     const int nt = (T <= 8) ? 1 : 2;
     const __half* Xh = reinterpret_cast<const __half*>(X);
     const __half* Bh = reinterpret_cast<const __half*>(B);
     __half* Rh = reinterpret_cast<__half*>(R);
     unsigned int* status = device_status_ptr();
-    void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&Rh, (void*)&status};
+    void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&Rh, (void*)&flags, (void*)&status};
     const void* fn = (nt == 1) ? (const void*)rproj_cluster_kernel<1> : (const void*)rproj_cluster_kernel<2>;
     const size_t smem = (size_t)rc_smem_bytes(r, d, nt);
     // opt in to the largest dynamic shared memory requested so far (at most
@@ -802,9 +924,15 @@ static int resident_ctas(const void* fn, int warps, int kc, size_t smem, int num
 
 struct GemvShape { int rt, kw, kc, stages; size_t smem; };
 
-static const void* gemv_fn(int nt, int stages) {
-    if (nt == 1) return stages == 8 ? (const void*)corrected_gemv_kernel<1, 8> : (const void*)corrected_gemv_kernel<1, 4>;
-    return stages == 8 ? (const void*)corrected_gemv_kernel<2, 8> : (const void*)corrected_gemv_kernel<2, 4>;
+// one: T == 1 (a single token: only one output column is finished)
+static const void* gemv_fn(int nt, int stages, bool one = false) {
+    if (nt == 1) {
+        if (one)
+            return stages == 8 ? (const void*)corrected_gemv_kernel<1, 8, true>
+                               : (const void*)corrected_gemv_kernel<1, 4, true>;
+        return stages == 8 ? (const void*)corrected_gemv_kernel<1, 8, false> : (const void*)corrected_gemv_kernel<1, 4, false>;
+    }
+    return stages == 8 ? (const void*)corrected_gemv_kernel<2, 8, false> : (const void*)corrected_gemv_kernel<2, 4, false>;
 }
 
 // Pick (rt, kw, kc, stages): all CTAs resident in one wave; then as many SMs
@@ -836,13 +964,13 @@ static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sm
                 for (int kc = 1; kc <= 8; ++kc) {
                     if (kc > 1 && kw > 1) break;
                     if (kc > ngroups || ngroups / kc < kw) continue;
-                    const int warps = rt * kw;
+                    const int warps = rt * kw;   // compute warps (+1 control warp per CTA)
                     const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, nt, stages);
                     if (L.total > 220 * 1024) continue;
                     if (pad && (size_t)L.total >= kSpreadSmem) continue;
                     const size_t smem = pad ? kSpreadSmem : (size_t)L.total;
                     const void* fn = gemv_fn(nt, stages);
-                    const int res = resident_ctas(fn, warps, kc, smem, num_sms);
+                    const int res = resident_ctas(fn, warps + 1, kc, smem, num_sms);
                     if (res <= 0) continue;
                     const long ctas = (long)ceil_div(tiles, rt) * kc;
                     const double waves = (double)ctas / res;
@@ -879,7 +1007,7 @@ static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sm
 }
 
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
-                               const uint16_t* R, bool after_rproj, int num_sms, cudaStream_t st) {
+                               const uint16_t* R, unsigned int* flags, int num_sms, cudaStream_t st) {
     GemvArgs a = {};
     int tiles = 0;
     for (int i = 0; i < m; ++i) {
@@ -901,10 +1029,12 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     static bool opted = false;
     if (!opted) {
         for (int n = 1; n <= 2; ++n)
-            for (int sg = 4; sg <= 8; sg *= 2) {
-                cudaError_t e = cudaFuncSetAttribute(gemv_fn(n, sg), cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
-                if (e != cudaSuccess) return e;
-            }
+            for (int sg = 4; sg <= 8; sg *= 2)
+                for (int one = 0; one <= (n == 1 ? 1 : 0); ++one) {
+                    cudaError_t e = cudaFuncSetAttribute(gemv_fn(n, sg, one != 0),
+                                                         cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
+                    if (e != cudaSuccess) return e;
+                }
         opted = true;
     }
     GemvShape sh = choose_shape(tiles, d, T, r, nt, num_sms);
@@ -934,13 +1064,14 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     a.rt = sh.rt;
     a.kw = sh.kw;
     a.kc = sh.kc;
-    (void)after_rproj;   // the kernel always waits for its predecessors before reading X and R
+    a.flags = (r > 0) ? flags : nullptr;
+    a.nflag = kRcCtas;
     a.X = reinterpret_cast<const __half*>(X);
     a.R = reinterpret_cast<const __half*>(R);
     a.status = device_status_ptr();
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(ceil_div(tiles, sh.rt) * sh.kc);
-    cfg.blockDim = dim3(sh.rt * sh.kw * 32);
+    cfg.blockDim = dim3((sh.rt * sh.kw + 1) * 32);   // compute warps + the control warp
     cfg.dynamicSmemBytes = sh.smem;
     cfg.stream = st;
     cudaLaunchAttribute attr[2];
@@ -957,7 +1088,7 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     cfg.attrs = attr;
     cfg.numAttrs = na;
     void* args[] = {(void*)&a, (void*)&plan};
-    return cudaLaunchKernelExC(&cfg, gemv_fn(nt, sh.stages), args);
+    return cudaLaunchKernelExC(&cfg, gemv_fn(nt, sh.stages, T == 1), args);
 }
 
 }  // namespace glowq

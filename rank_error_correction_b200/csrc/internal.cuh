@@ -28,10 +28,15 @@ unsigned int* device_status_ptr();
 
 // decode.cu
 // R = X B^T (T <= 16) by one thread-block cluster, written to R in fp16.
+// flags: three zeroed words through which the GEMV that follows learns that X
+// is final and that R is stored (the GEMV zeroes them again).
+constexpr int kDecodeFlagWords = 3;
 cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, uint16_t* R,
-                                cudaStream_t st);
+                                unsigned int* flags, cudaStream_t st);
+// Corrected GEMV over the stacked rows; with flags (after launch_rproj_decode
+// with the same flags) it waits on them instead of on the R kernel's completion.
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
-                               const uint16_t* R, bool after_rproj, int num_sms, cudaStream_t st);
+                               const uint16_t* R, unsigned int* flags, int num_sms, cudaStream_t st);
 // pack.cu
 cudaError_t launch_pack_int4(const float* W, int64_t O, int64_t d, uint32_t* q, uint16_t* s, uint8_t* z,
                              cudaStream_t st);

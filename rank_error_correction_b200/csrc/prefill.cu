@@ -45,10 +45,6 @@ namespace glowq {
 // ---------------------------------------------------------------------------
 // tcgen05 / TMA device helpers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // Shared-memory matrix descriptor: K-major operand in the canonical 128-byte
 // swizzled layout (rows of 128 B, 8-row atoms of 1024 B, atoms 1024 B apart).
 __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
@@ -725,9 +721,12 @@ __global__ void __launch_bounds__(256) rproj_sum_kernel(const float4* __restrict
     pdl_wait();                 // partial sums complete
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n4) return;
-    float4 acc = partial[i];
+    // L2 loads: the partial sums were written while this grid was already resident
+    const uint4 a0 = ldcg_128(partial + i);
+    float4 acc = make_float4(__uint_as_float(a0.x), __uint_as_float(a0.y), __uint_as_float(a0.z), __uint_as_float(a0.w));
     for (int y = 1; y < chunks; ++y) {
-        const float4 v = partial[(int64_t)y * n4 + i];
+        const uint4 u = ldcg_128(partial + (int64_t)y * n4 + i);
+        const float4 v = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
         acc.x += v.x;
         acc.y += v.y;
         acc.z += v.z;

@@ -175,9 +175,11 @@ def workspace_bytes(T: int, r: int) -> int:
 
 
 def alloc_workspace(T: int, r: int, device="cuda"):
+    # zero-filled: the first 256 bytes are the decode kernels' hand-off flags,
+    # which must start at zero (every call leaves them zero)
     import torch
     n = max(workspace_bytes(T, r), 16)
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def _module_structs(mods: Sequence[QModule], Ys, use_A: bool):

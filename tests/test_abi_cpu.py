@@ -42,9 +42,10 @@ def test_workspace_bytes(L):
     assert glowq.workspace_bytes(0, 64) == 0
     assert glowq.workspace_bytes(16, 0) == 0
     small = glowq.workspace_bytes(16, 64)
-    assert small >= 16 * 64 * 2                          # solo R (decode reduces R on chip)
+    assert small == 256 + 16 * 64 * 2                    # hand-off flags + solo R (decode reduces R on chip)
+    assert glowq.workspace_bytes(1, 64) == 256 + 256     # solo R rounded up to 256 B
     big = glowq.workspace_bytes(2048, 64)
-    assert big >= 8 * 2048 * 64 * 4 + 2048 * 64 * 2      # split-d fp32 partials of R + solo R
+    assert big >= 256 + 8 * 2048 * 64 * 4 + 2048 * 64 * 2   # flags + split-d fp32 partials of R + solo R
     assert small % 256 == 0 and big % 256 == 0
 
 
@@ -74,6 +75,9 @@ def test_host_validation_errors(L):
     assert _gf(L, _mods(1), B=None) == 1                # r > 0 needs B
     assert _gf(L, _mods(1), R=None) == 1                # ... and R_out
     assert _gf(L, _mods(1), T=64, wsb=16) == 1          # workspace too small (T > 16 splits R)
+    assert _gf(L, _mods(1), T=4, ws=None, wsb=0) == 1   # decode with r > 0 needs the hand-off flags
+    assert _gf(L, _mods(1), T=4, wsb=128) == 1          # ... all 256 bytes of them
+    assert _gf(L, _mods(1), T=4, ws=0x7008) == 3        # misaligned workspace
     assert _gf(L, _mods(1), T=-1) == 1
     assert _gf(L, _mods(1), T=0) == 0                   # empty batch: no-op
     assert L.glowq_solo_forward(_mods(1), 256, 0x4000, 16, 0x5000, 4, None, 0, None) == 1

@@ -150,3 +150,18 @@ def test_llama31_8b_qkv_prefill_t4096_sampled():
     X = synth.activations(T, d, synth.ALPHA_QKV, seed=1)
     Ys, _ = glowq.group_forward(to_dev(qkv), torch.from_numpy(B).cuda(), torch.from_numpy(X).cuda())
     _sampled_check(qkv, B, X, [_np(Y) for Y in Ys])
+
+
+def test_prefill_eight_modules_small_outputs():
+    """Eight modules of 16..128 rows (the peer CTA of a 256-row pair tile holds
+    no valid row), ragged T, r = 64."""
+    d, r, T = 768, 64, 300
+    mods = make_modules(d, [16, 32, 48, 64, 80, 96, 112, 128], seed=88)
+    B = attach_random_factors(mods, d, r, seed=88)
+    X = synth.activations(T, d, synth.ALPHA_QKV, seed=88)
+    ys, R = _run_group(mods, B, X)
+    refs, R_ref = _oracle_group(mods, B, X)
+    assert normwise(R, R_ref) < 1e-3
+    for y, ref in zip(ys, refs):
+        assert y.shape == ref.shape
+        assert normwise(y, ref) < TOL
