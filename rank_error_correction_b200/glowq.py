@@ -160,6 +160,21 @@ class QModule:
     scales: "object"
     zeros: "object"
     A: Optional["object"] = None
+    # validated device pointers (qweight, scales, zeros, A, out_features),
+    # computed on first use and dropped whenever a field is reassigned
+    _ptrs: Optional[tuple] = dataclasses.field(default=None, init=False, repr=False, compare=False)
+
+    def __setattr__(self, name, value):
+        object.__setattr__(self, name, value)
+        if name != "_ptrs":
+            object.__setattr__(self, "_ptrs", None)
+
+    def pointers(self) -> tuple:
+        if self._ptrs is None:
+            _require_cuda(self.qweight, self.scales, self.zeros, self.A)
+            object.__setattr__(self, "_ptrs", (self.qweight.data_ptr(), self.scales.data_ptr(), self.zeros.data_ptr(),
+                                               _ptr(self.A), int(self.qweight.shape[0])))
+        return self._ptrs
 
     @property
     def out_features(self) -> int:
@@ -183,17 +198,11 @@ def alloc_workspace(T: int, r: int, device="cuda"):
 
 
 def _module_structs(mods: Sequence[QModule], Ys, use_A: bool):
-    arr = (_Module * len(mods))()
-    for i, (m, Y) in enumerate(zip(mods, Ys)):
-        _require_cuda(m.qweight, m.scales, m.zeros, m.A)
-        arr[i].qweight = _ptr(m.qweight)
-        arr[i].scales = _ptr(m.scales)
-        arr[i].zeros = _ptr(m.zeros)
-        arr[i].A = _ptr(m.A) if use_A else None
-        arr[i].out_features = m.out_features
-        arr[i].Y = Y.data_ptr()
-        arr[i].ldY = Y.stride(0)
-    return arr
+    items = []
+    for m, Y in zip(mods, Ys):
+        q, s, z, a, o = m.pointers()
+        items.append(_Module(q, s, z, a if use_A else None, o, Y.data_ptr(), Y.stride(0)))
+    return (_Module * len(items))(*items)
 
 
 def group_forward(mods: Sequence[QModule], B, X, Ys=None, R_out=None, workspace=None, stream=None):

@@ -277,3 +277,28 @@ def test_decode_wide_input_solo():
     torch.cuda.synchronize()
     ref = oracle.solo_forward(mods[0].q, mods[0].s, mods[0].z, synth.bits(mods[0].A), synth.bits(B), synth.bits(X))
     assert normwise(Y.cpu().numpy().astype(np.float64), ref) < TOL
+
+
+def test_workspace_flags_shared_by_decode_prefill_and_solo_calls():
+    """One workspace serves decode group, prefill group and decode solo calls in
+    turn (any T, one stream): the decode hand-off flags at offset 0 are zero
+    after every call and the outputs match the oracle throughout."""
+    import torch
+    d, r = 512, 32
+    mods = make_modules(d, [128, 64], seed=91)
+    B = attach_random_factors(mods, d, r, seed=91)
+    dev = to_dev(mods)
+    Bd = torch.from_numpy(B).cuda()
+    ws = glowq.alloc_workspace(64, r)
+    for k, T in enumerate((1, 64, 3, 16, 1)):
+        X = synth.activations(T, d, synth.ALPHA_QKV, seed=92 + k)
+        Xd = torch.from_numpy(X).cuda()
+        Ys, R = glowq.group_forward(dev, Bd, Xd, workspace=ws)
+        Yo = glowq.solo_forward(dev[1], Bd, Xd, workspace=ws)
+        torch.cuda.synchronize()
+        assert int(ws[:12].view(torch.int32).abs().sum()) == 0, (T, ws[:12].tolist())
+        refs, R_ref = _oracle_group(mods, B, X)
+        assert normwise(_np(R).astype(np.float64), R_ref) < 1e-3
+        for y, ref in zip(Ys, refs):
+            assert normwise(_np(y).astype(np.float64), ref) < TOL
+        assert normwise(_np(Yo).astype(np.float64), refs[1]) < TOL
