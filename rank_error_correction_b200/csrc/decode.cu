@@ -659,11 +659,23 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
             xrow[n] = xs + tok * wpt + (G0 - C0) * 16;
         }
         const float* xsum_w = xsum + (G0 - C0) * 2 * 8 * NT + 2 * t;
+        // Running pointers, advanced once per round of kStages stages, so that
+        // every shared-memory read inside the unrolled round is base + constant:
+        // activation fragment w of token block n, scale/zero pair, group sums.
+        const uint4* xw[NT][4];
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) xw[n][w] = xrow[n] + ((4 * t + w) ^ xsw);
+        const float2* szl = sz_lo;
+        const float2* szh = sz_hi;
+        const float* xsp = xsum_w;
         // lane (g, t) reads 16 B of rows g and g+8 per group
         const unsigned char* rd_lo = my_ring + g * 128 + t * 16;
         const unsigned char* rd_hi = rd_lo + 8 * 128;
         bool ok = true;
-        for (int p0 = 0; p0 < npairs; p0 += kStages) {
+        for (int p0 = 0; p0 < npairs; p0 += kStages,
+                 szl += 2 * kStages, szh += 2 * kStages, xsp += 2 * kStages * 2 * 8 * NT) {
 #pragma unroll
             for (int i = 0; i < kStages; ++i) {
                 const int p = p0 + i;
@@ -689,7 +701,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
                         if (h == 1 && !two) break;
-                        const int gl = 2 * p + h;          // group within the warp's split
+                        const int gi = 2 * i + h;          // group within this round (a constant)
                         const uint32_t wl[4] = {w4[h][0].x, w4[h][0].y, w4[h][0].z, w4[h][0].w};
                         const uint32_t wh[4] = {w4[h][1].x, w4[h][1].y, w4[h][1].z, w4[h][1].w};
                         // two MMA chains: even k (A = 16 + q/64) and odd k (A = 64 + q)
@@ -703,7 +715,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                             const uint32_t ao[4] = {ol[0], oh[0], ol[1], oh[1]};
 #pragma unroll
                             for (int n = 0; n < NT; ++n) {
-                                const uint4 x = xrow[n][gl * 16 + ((4 * t + w) ^ xsw)];
+                                const uint4 x = xw[n][w][gi * 16];
                                 const uint32_t be[2] = {x.x, x.y};   // (x0,x4) (x2,x6)
                                 const uint32_t bo[2] = {x.z, x.w};   // (x1,x5) (x3,x7)
                                 if (w == 0) {
@@ -716,12 +728,12 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                             }
                         }
                         // sum_k (q - z) x = 64 D_E + D_O - (1024 + z) S_E - (64 + z) S_O, times s
-                        const float2 zl = sz_lo[gl], zh = sz_hi[gl];   // (s, 64 + z)
+                        const float2 zl = szl[gi], zh = szh[gi];   // (s, 64 + z)
                         const float cel = zl.y + 960.0f, ceh = zh.y + 960.0f;
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
-                            const float2 se = *reinterpret_cast<const float2*>(xsum_w + (2 * gl) * 8 * NT + n * 8);
-                            const float2 so = *reinterpret_cast<const float2*>(xsum_w + (2 * gl + 1) * 8 * NT + n * 8);
+                            const float2 se = *reinterpret_cast<const float2*>(xsp + (2 * gi) * 8 * NT + n * 8);
+                            const float2 so = *reinterpret_cast<const float2*>(xsp + (2 * gi + 1) * 8 * NT + n * 8);
                             if (ONE) {
                                 float v0 = fmaf(64.0f, te[n][0], to[n][0]);
                                 float v2 = fmaf(64.0f, te[n][2], to[n][2]);
@@ -747,6 +759,10 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                     }
                 }
             }
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int w = 0; w < 4; ++w) xw[n][w] += 2 * kStages * 16;
         }
     }
     cp_async_wait<0>();
