@@ -9,12 +9,15 @@
 // One call is two launches chained with programmatic dependent launch:
 //   * rproj_cluster: R = X B^T by one cluster of 8 CTAs splitting d; the
 //     partial sums meet on chip in a fixed order (deterministic), R is rounded
-//     to fp16 once and written to the caller's R buffer.
+//     to fp16 once and written to the caller's R buffer.  It lets the GEMV
+//     launch once X is final and tells it through workspace flags when X is
+//     final and when R is stored.
 //   * corrected_gemv: one launch over the stacked rows of all modules of the
 //     group.  Each warp streams its 16 rows of packed weights with 2-D TMA
-//     boxes into a private ring of mbarrier-tracked stages, issued before the
-//     wait on the preceding kernel (weights and scales are static), so the
-//     stream overlaps the projection.  Nibbles become exact fp16 values
+//     boxes into a private ring of mbarrier-tracked stages; the stream and the
+//     main loop run while the projection is still being computed (R is needed
+//     only by the epilogue, and a control warp per CTA collects it into shared
+//     memory meanwhile).  Nibbles become exact fp16 values
 //     (16 + q/64 for even k, 64 + q for odd k) with one LOP3 per pair; the
 //     multiply-accumulate runs on the tensor cores with register operands
 //     (mma.sync m16n8k16, fp32 accumulate, one chain per parity) and each
@@ -237,7 +240,7 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
 // Corrected GEMV over the stacked rows of a group.
 //
 // Work shape (chosen on the host from the occupancy calculator so that every
-// CTA is resident in one wave with ~16-24 warps per SM):
+// CTA is resident in one wave, with up to kMaxWarps compute warps per CTA):
 //   * a CTA holds `rt` row tiles of 16 rows x `kw` in-CTA splits of its slice
 //     of d (rt * kw warps; warp w owns tile w % rt and split w / rt);
 //   * optionally a thread-block cluster of `kc` CTAs splits d further (then
@@ -250,7 +253,8 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
 //   (two tensor-core chains, fp32 accumulate),  S_E / S_O = sums of x over E / O.
 // Both operand forms are exact fp16 values built without subtracting anything
 // per weight: the nibble lands in mantissa bits 0..3 of 16.0 or 4..7 of 64.0,
-// one shift and four LOP3 per 8 codes.  S_E and S_O are computed once per CTA.
+// one shift and four LOP3 per 8 codes.  S_E and S_O are computed once per CTA,
+// while the activation slice is staged.
 //
 // Shared memory (dynamic), in this order:
 //   ring [warps][S][16][32] u32      packed-weight stream: a stage is one 2-D TMA
