@@ -208,6 +208,22 @@ GLOWQ_API glowq_status glowq_select_restore(const double* err_fro2, const double
                                   int32_t* order, int32_t* used_fallback);
 
 /*
+ * GlowQ-S selective restore by a caller-computed importance score (key
+ * design 4 names two scores; the other one, the covariance-aligned GSVD
+ * energy capture g_ec(u) = sum_{j<=r} sigma_j(M_u)^2 / ||M_u||_F^2, comes out
+ * of the offline solve's core M_u).  Host-only.
+ *   score[u]                 importance of unit u, larger = restore first (host, n_units)
+ *   layer_idx, kind, k, restore_mask, order, used_fallback: as for
+ *   glowq_select_restore, with the same tie-break and weak-signal fallback.
+ * Errors: GLOWQ_ERR_ARG for n_units < 0, k outside 0..n_units, or a NULL
+ * array with n_units > 0.
+ */
+GLOWQ_API glowq_status glowq_select_restore_scores(const double* score, const int32_t* layer_idx,
+                                         const int32_t* kind, int32_t n_units, int32_t k,
+                                         uint8_t* restore_mask, int32_t* order,
+                                         int32_t* used_fallback);
+
+/*
  * Per-row squared norms for g_ner: row_norms[2*o] = ||W[o] - w_hat[o]||^2 and
  * row_norms[2*o+1] = ||W[o]||^2 (fp64, deterministic), from a module's fp32
  * weight and its packed form.  Summing the rows of every module of a unit

@@ -75,10 +75,12 @@ def _declare(L):
     L.ora_rsvd.argtypes = [_p, _i64, _i64, _i32, _i32, _i32, _p, _p, _p, _p]
     L.ora_group_solve.argtypes = [_p, _i64, _i64, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p]
     L.ora_select_restore.argtypes = [_p, _p, _p, _p, _i32, _i32, _p, _p, _p]
+    L.ora_select_by_score.argtypes = [_p, _p, _p, _i32, _i32, _p, _p]
     for name in ("ora_quantize_int4", "ora_unpack_int4", "ora_dequant_int4", "ora_quant_error",
                  "ora_anchor_project", "ora_module_forward", "ora_solo_forward",
                  "ora_module_forward_sampled", "ora_matmul", "ora_householder_qr",
-                 "ora_jacobi_svd", "ora_rsvd", "ora_group_solve", "ora_select_restore"):
+                 "ora_jacobi_svd", "ora_rsvd", "ora_group_solve", "ora_select_restore",
+                 "ora_select_by_score"):
         getattr(L, name).restype = C.c_int
 
 
@@ -279,7 +281,37 @@ def group_solve(E_cat, Sh, Shp, r, p=16, q=2, Omega=None):
     return A, B, sing
 
 
+def energy_capture(E_cat, Sh, r):
+    """GSVD energy-capture score of a unit (GlowQ pages, papernotes.org summary,
+    key design 4): g_ec(u) = sum_{j<=r} sigma_j(M_u)^2 / ||M_u||_F^2, with M_u the
+    covariance-aligned core of the unit's stacked error, M = R_e Sx^{1/2}
+    (R_e from the thin QR of E_cat, key design 3).  Exact singular values of
+    the core (one-sided Jacobi), so for small and mid sizes only; since
+    ||M||_F^2 = sum_j sigma_j^2, 1 - g_ec is the best rank-r fit's relative
+    residual of the covariance-weighted error."""
+    _, Re = householder_qr(E_cat)
+    M = matmul(Re, Sh)
+    _, S, _ = jacobi_svd(M)
+    s2 = S * S
+    tot = float(np.sum(s2))
+    return float(np.sum(s2[:r]) / tot) if tot > 0 else float("nan")
+
+
 # -- GlowQ-S ---------------------------------------------------------------------
+
+def select_by_score(score, layer, kind, k):
+    """Rank units by any importance score (g_ec or g_ner), descending; exact
+    ties and the weak-signal fallback as in select_restore.  Returns
+    (mask, order, used_fallback)."""
+    sc = _c(score, np.float64)
+    la, ki = _c(layer, np.int32), _c(kind, np.int32)
+    n = sc.size
+    mask = np.zeros(n, np.uint8)
+    order = np.zeros(n, np.int32)
+    rc = _check(lib().ora_select_by_score(_ptr(sc), _ptr(la), _ptr(ki), n, k, _ptr(mask), _ptr(order)),
+                "select_by_score")
+    return mask, order, bool(rc == 1)
+
 
 def select_restore(err_fro2, w_fro2, layer, kind, k):
     e, w = _c(err_fro2, np.float64), _c(w_fro2, np.float64)

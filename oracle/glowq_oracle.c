@@ -640,22 +640,24 @@ static int unit_cmp(const void* pa, const void* pb)
     return a < b ? -1 : (a > b);
 }
 
-int ora_select_restore(const double* err_fro2, const double* w_fro2,
-                       const int32_t* layer, const int32_t* kind, int32_t n,
-                       int32_t k, uint8_t* mask, int32_t* order, double* score)
+/*
+ * Rank units by an arbitrary importance score (the pages name two: the GSVD
+ * energy capture g_ec and the normalised error ratio g_ner) with the same
+ * tie-break and weak-signal fallback as above; restore the top k.
+ * Returns 1 when the fallback was taken, 0 otherwise, -1 on bad arguments.
+ */
+int ora_select_by_score(const double* sc, const int32_t* layer, const int32_t* kind,
+                        int32_t n, int32_t k, uint8_t* mask, int32_t* order)
 {
     if (n < 0 || k < 0 || k > n) return -1;
-    double* sc = (double*)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
     int any_nan = 0;
     double mx = -INFINITY, mn = INFINITY;
     for (int32_t u = 0; u < n; ++u) {
-        sc[u] = err_fro2[u] / w_fro2[u];
         if (isnan(sc[u])) any_nan = 1;
         else {
             if (sc[u] > mx) mx = sc[u];
             if (sc[u] < mn) mn = sc[u];
         }
-        if (score) score[u] = sc[u];
     }
     int weak = any_nan || n == 0 || (mx - mn) <= 1e-6 * fmax(fabs(mx), 1e-300);
     for (int32_t u = 0; u < n; ++u) order[u] = u;
@@ -663,6 +665,20 @@ int ora_select_restore(const double* err_fro2, const double* w_fro2,
     qsort(order, (size_t)n, sizeof(int32_t), unit_cmp);
     for (int32_t u = 0; u < n; ++u) mask[u] = 0;
     for (int32_t i = 0; i < k; ++i) mask[order[i]] = 1;
-    free(sc);
     return weak ? 1 : 0;
+}
+
+int ora_select_restore(const double* err_fro2, const double* w_fro2,
+                       const int32_t* layer, const int32_t* kind, int32_t n,
+                       int32_t k, uint8_t* mask, int32_t* order, double* score)
+{
+    if (n < 0 || k < 0 || k > n) return -1;
+    double* sc = (double*)malloc((size_t)(n > 0 ? n : 1) * sizeof(double));
+    for (int32_t u = 0; u < n; ++u) {
+        sc[u] = err_fro2[u] / w_fro2[u];
+        if (score) score[u] = sc[u];
+    }
+    int rc = ora_select_by_score(sc, layer, kind, n, k, mask, order);
+    free(sc);
+    return rc;
 }

@@ -58,6 +58,7 @@ def lib() -> C.CDLL:
         L.glowq_solo_forward_noalloc.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p]
         L.glowq_noalloc_scratch_bytes.restype = C.c_size_t
         L.glowq_select_restore.argtypes = [p, p, p, p, i32, i32, p, p, p]
+        L.glowq_select_restore_scores.argtypes = [p, p, p, i32, i32, p, p, p]
         L.glowq_error_norms.argtypes = [p, p, p, p, i64, i64, p, p]
         L.glowq_get_device_status.argtypes = [p]
         L.glowq_selftest_wait_timeout.argtypes = [C.c_uint32, p]
@@ -66,7 +67,8 @@ def lib() -> C.CDLL:
         L.glowq_version.restype = C.c_char_p
         for f in ("glowq_pack_int4", "glowq_dequant_int4", "glowq_group_forward", "glowq_solo_forward",
                   "glowq_solo_forward_noalloc",
-                  "glowq_select_restore", "glowq_error_norms", "glowq_get_device_status",
+                  "glowq_select_restore", "glowq_select_restore_scores", "glowq_error_norms",
+                  "glowq_get_device_status",
                   "glowq_selftest_wait_timeout"):
             getattr(L, f).restype = st
         _lib = L
@@ -296,4 +298,21 @@ def select_restore(err_fro2, w_fro2, layer_idx, kind, k: int) -> Tuple["object",
     p = lambda a: a.ctypes.data_as(C.c_void_p)
     _check(lib().glowq_select_restore(p(e), p(w), p(la), p(ki), n, int(k), p(mask), p(order), C.byref(fb)),
            "glowq_select_restore")
+    return mask, order, bool(fb.value)
+
+
+def select_restore_scores(score, layer_idx, kind, k: int) -> Tuple["object", "object", bool]:
+    """Host-only ranking by a caller-computed score (e.g. g_ec from the offline
+    solve); returns (mask uint8[n], order int32[n], used_fallback)."""
+    import numpy as np
+    sc = np.ascontiguousarray(score, dtype=np.float64)
+    la = np.ascontiguousarray(layer_idx, dtype=np.int32)
+    ki = np.ascontiguousarray(kind, dtype=np.int32)
+    n = sc.size
+    mask = np.zeros(n, np.uint8)
+    order = np.zeros(n, np.int32)
+    fb = C.c_int32(0)
+    p = lambda a: a.ctypes.data_as(C.c_void_p)
+    _check(lib().glowq_select_restore_scores(p(sc), p(la), p(ki), n, int(k), p(mask), p(order), C.byref(fb)),
+           "glowq_select_restore_scores")
     return mask, order, bool(fb.value)

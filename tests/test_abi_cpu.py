@@ -107,3 +107,29 @@ def test_select_restore_matches_oracle(L):
 def test_select_restore_rejects_bad_k(L):
     with pytest.raises(glowq.GlowQError):
         glowq.select_restore([1.0], [1.0], [0], [0], 2)
+
+
+def test_select_restore_scores_matches_oracle(L):
+    """Host-only ranking by a caller-computed score (e.g. g_ec) against the oracle."""
+    g = np.random.default_rng(5)
+    for trial in range(40):
+        n = int(g.integers(1, 60))
+        sc = np.round(g.random(n) * 4, 1 if trial % 2 else 6)
+        if trial % 7 == 3:
+            sc = np.full(n, 0.25)                                # flat scores -> layer order
+        if trial % 11 == 5:
+            sc[int(g.integers(0, n))] = np.nan                   # NaN -> layer order
+        layer = g.integers(0, 12, n)
+        kind = g.integers(0, 4, n)
+        k = int(g.integers(0, n + 1))
+        m_g, o_g, fb_g = glowq.select_restore_scores(sc, layer, kind, k)
+        m_o, o_o, fb_o = oracle.select_by_score(sc, layer, kind, k)
+        assert fb_g == fb_o
+        assert np.array_equal(m_g, m_o) and np.array_equal(o_g, o_o)
+    # argument errors are reported before anything is written
+    assert L.glowq_select_restore_scores(None, None, None, 3, 1, None, None, None) == 1
+    assert L.glowq_select_restore_scores(None, None, None, 0, 0, None, None, None) == 0
+    x = np.zeros(2)
+    p = lambda a: a.ctypes.data_as(C.c_void_p)
+    assert L.glowq_select_restore_scores(p(x), p(np.zeros(2, np.int32)), p(np.zeros(2, np.int32)), 2, 3,
+                                         p(np.zeros(2, np.uint8)), None, None) == 1     # k > n

@@ -69,3 +69,37 @@ def test_random_tables_against_brute_force():
         assert weak == bw
         assert np.array_equal(order, bo) and np.array_equal(mask, bm)
         assert mask.sum() == k
+
+
+def _brute_scores(sc, layer, kind, k):
+    weak = any(np.isnan(sc)) or (max(sc) - min(sc)) <= 1e-6 * max(abs(max(sc)), 1e-300)
+    if weak:
+        order = sorted(range(len(sc)), key=lambda u: (layer[u], kind[u], u))
+    else:
+        order = sorted(range(len(sc)), key=lambda u: (-sc[u], layer[u], kind[u], u))
+    mask = np.zeros(len(sc), np.uint8)
+    mask[order[:k]] = 1
+    return mask, np.array(order), weak
+
+
+def test_select_by_score_against_brute_force_and_ratio_path():
+    """Ranking by an arbitrary score (e.g. g_ec) follows the same rule, and on
+    score = err / w it is exactly the g_ner selection."""
+    g = np.random.default_rng(3)
+    for trial in range(50):
+        n = int(g.integers(1, 40))
+        sc = list(np.round(g.random(n) * 2, 2 if trial % 2 else 6))
+        if trial % 9 == 4:
+            sc = [0.5] * n                                       # flat: layer order
+        layer = list(g.integers(0, 10, n))
+        kind = list(g.integers(0, 4, n))
+        k = int(g.integers(0, n + 1))
+        mask, order, weak = oracle.select_by_score(sc, layer, kind, k)
+        bm, bo, bw = _brute_scores(sc, layer, kind, k)
+        assert weak == bw
+        assert np.array_equal(order, bo) and np.array_equal(mask, bm)
+        e = np.array(sc) * 3.0
+        w = np.full(n, 3.0)
+        m2, o2, _, w2 = oracle.select_restore(e, w, layer, kind, k)
+        m3, o3, w3 = oracle.select_by_score(e / w, layer, kind, k)
+        assert np.array_equal(o2, o3) and np.array_equal(m2, m3) and w2 == w3

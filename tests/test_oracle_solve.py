@@ -183,3 +183,45 @@ def test_rsvd_solve_close_to_exact_solve():
     assert re <= rr * (1 + 1e-12)
     assert rr <= re * 1.02
     assert np.allclose(sr, se, rtol=2e-2)
+
+
+# -- GSVD energy-capture score g_ec (key design 4) ------------------------------
+
+def test_energy_capture_closed_form_on_known_spectrum():
+    """E = U diag(sv) V^T with known singular values and Sx = I: the core's
+    singular values are sv, so g_ec = sum of the top-r squares / sum of all."""
+    g = np.random.default_rng(20)
+    m, d = 18, 7
+    U, _ = np.linalg.qr(g.standard_normal((m, d)))
+    V, _ = np.linalg.qr(g.standard_normal((d, d)))
+    sv = np.array([5.0, 3.0, 2.0, 1.0, 0.5, 0.25, 0.125])
+    E = U @ np.diag(sv) @ V.T
+    for r in range(1, d + 1):
+        want = np.sum(sv[:r] ** 2) / np.sum(sv ** 2)
+        assert oracle.energy_capture(E, np.eye(d), r) == pytest.approx(want, rel=1e-12)
+
+
+def test_energy_capture_is_the_best_fit_share_of_the_solve():
+    """Eckart-Young-Mirsky tie to the solve: with the exact core SVD,
+    1 - g_ec = ||(E - A B) Sx^{1/2}||_F^2 / ||E Sx^{1/2}||_F^2 at the same rank."""
+    d, r = 32, 6
+    E = _stacked_error(d, [24, 16, 16], seed=21) * 100.0
+    basis = synth.orthogonal_basis(d, seed=21)
+    Sh, Shp = synth.covariance_half(basis, synth.power_law_spectrum(d, 0.77))
+    A, B, _ = oracle.group_solve(E, Sh, Shp, r)          # exact (Jacobi) core SVD
+    resid = np.linalg.norm((E - A @ B) @ Sh) ** 2 / np.linalg.norm(E @ Sh) ** 2
+    assert 1.0 - oracle.energy_capture(E, Sh, r) == pytest.approx(resid, rel=1e-9)
+
+
+def test_energy_capture_invariances_and_range():
+    g = np.random.default_rng(22)
+    m, d = 20, 9
+    E = g.standard_normal((m, d)) * np.linspace(3.0, 0.1, d)
+    Sh = np.diag(np.linspace(1.5, 0.5, d))
+    base = [oracle.energy_capture(E, Sh, r) for r in range(1, d + 1)]
+    assert all(0.0 < v <= 1.0 + 1e-12 for v in base)
+    assert all(b >= a - 1e-12 for a, b in zip(base, base[1:]))    # non-decreasing in r
+    assert base[-1] == pytest.approx(1.0, abs=1e-12)              # r = rank captures everything
+    Q, _ = np.linalg.qr(g.standard_normal((m, m)))                # rows mixed orthogonally
+    assert [oracle.energy_capture(Q @ E, Sh, r) for r in range(1, d + 1)] == pytest.approx(base, rel=1e-10)
+    assert [oracle.energy_capture(7.0 * E, Sh, r) for r in range(1, d + 1)] == pytest.approx(base, rel=1e-10)
