@@ -733,8 +733,11 @@ def main():
         if os.path.exists(tr_path):
             try:
                 tr = json.load(open(tr_path))
-                traffic = tr.get("decode qkv T=1 group call", {}).get("bytes")
-                traffic_pf = tr.get("prefill gate_up T=2048 corrected_gemm", {}).get("bytes")
+                # an entry whose kernel changed after its capture reports null
+                dec = tr.get("decode qkv T=1 group call", {})
+                pf = tr.get("prefill gate_up T=2048 corrected_gemm", {})
+                traffic = None if dec.get("stale") else dec.get("bytes")
+                traffic_pf = None if pf.get("stale") else pf.get("bytes")
             except Exception:
                 traffic = traffic_pf = None
         if prefill is not None:
