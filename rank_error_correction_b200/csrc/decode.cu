@@ -456,8 +456,10 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     const bool finaliser = !control && ks == 0 && owner == crank;
     const bool has_corr = r > 0 && M.A != nullptr;
 
-    // 1) start the weight stream first: per warp, S mbarriers; lane 0 issues
-    //    one 2-D TMA box (16 rows x 2 groups) per stage
+    // Prologue order (from per-CTA timelines of back-to-back calls): barriers,
+    // scale/zero loads, weight stream, A prefetch, scale/zero staging, then X.
+    // 1) the weight stream's ring: per warp, S mbarriers; lane 0 issues one 2-D
+    //    TMA box (16 rows x 2 groups) per stage
     constexpr int kStages = S;
     uint64_t* my_bars = bars + warp * kStages;
     unsigned char* my_ring = ring + warp * kStages * 2048;
@@ -471,10 +473,10 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         for (int i = 0; i < kStages; ++i) mbar_init(my_bars + i, 1);
         fence_mbar_init();
     }
-    // 0) this warp's scales and zeros are the longest-latency reads of the
+    // 2) this warp's scales and zeros are the longest-latency reads of the
     //    prologue (scattered, cold): a split of at most 32 groups is loaded in
     //    one batch ahead of the weight stream (behind it, they would queue
-    //    after every stage in flight), and staged below
+    //    after every stage in flight), and staged in step 5
     const int sz_stride = L.nsub_max + 1;
     float2* my_sz = szs + warp * 16 * sz_stride;
     const int rr = lane & 15;   // lane -> row (lane & 15) and every other group starting at lane >> 4
@@ -494,7 +496,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         }
     }
 
-    // 1') start the weight stream (read once per call: evict-first in L2)
+    // 3) start the weight stream (read once per call: evict-first in L2)
     const uint64_t wpol = l2_policy_evict_first();
     if (active) {
         if (lane == 0) {
@@ -505,7 +507,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         }
         __syncwarp();
     }
-    // 1b) the finalising warp prefetches its tile's rows of A
+    // 4) the finalising warp prefetches its tile's rows of A
     if (active && has_corr && finaliser) {
         const uint32_t a_base = (uint32_t)__cvta_generic_to_shared(as + fslot * 16 * (r + 8));
         const int cpr = r / 8;   // 16-byte chunks per row
@@ -516,7 +518,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     }
     cp_async_commit();
 
-    // 2) stage (s, 64 + z) of the warp's rows x groups [G0, G1); longer splits
+    // 5) stage (s, 64 + z) of the warp's rows x groups [G0, G1); longer splits
     //    load in batches of 16 per lane, all issued before any is used
     if (one_batch) {
 #pragma unroll
@@ -555,7 +557,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     }
     if (!args.flags) pdl_wait();
     __syncthreads();   // X is final; rbar is initialised
-    // 3) the CTA's activation slice, paired and swizzled (all loads of a batch
+    // 6) the CTA's activation slice, paired and swizzled (all loads of a batch
     //    first); every thread of the CTA, the control warp included, takes part
     const int stride = (int)blockDim.x;
     {
@@ -572,10 +574,10 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                     v[j] = ldcg_128(args.X + (int64_t)tok * d + (int64_t)C0 * 128 + wd * 8);
                 }
             }
-            // 4) with each word, its even / odd activation sums; the 16 words of
-            //    a (token, group) are held by 16 consecutive lanes (stride and
-            //    wpt are multiples of 16), which add them in a fixed butterfly
-            //    order into S_E and S_O: xsum[(2 * group + e)][token]
+            // with each word, its even / odd activation sums; the 16 words of a
+            // (token, group) are held by 16 consecutive lanes (stride and wpt
+            // are multiples of 16), which add them in a fixed butterfly order
+            // into S_E and S_O: xsum[(2 * group + e)][token]
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int i = base + j * stride;
@@ -616,7 +618,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     }
     __syncthreads();
 
-    // 5a) the control warp: once R is stored, copy it into rs (padding tokens
+    // 7) the control warp: once R is stored, copy it into rs (padding tokens
     //     zero) and complete rbar; the last CTA here zeroes the flags, which the
     //     next call's R kernel writes only after this grid has completed
     if (control && r > 0) {
@@ -644,7 +646,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         }
     }
 
-    // 5) main loop: two independent MMA chains per 128-group on (64 + q) x,
+    // 8) main loop: two independent MMA chains per 128-group on (64 + q) x,
     //    then s * (D - (64 + z) S) in fp32
     float acc[NT][4];
 #pragma unroll
@@ -773,7 +775,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     __syncwarp();   // A rows copied by other lanes of this warp are visible
 
 
-    // 6) split-d reduction in a fixed order, into the finalising warp
+    // 9) split-d reduction in a fixed order, into the finalising warp
     if (kc > 1) {
         // cluster: partials of tile tl go to rank tl % kc, slot [crank][tl / kc]
         const int idx0 = (crank * L.fin_slots + fslot) * NT * 4 * 32 + lane;
@@ -827,8 +829,8 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     }
     if (!active) return;
 
-    // 7) rank-r correction A_i R^T, accumulated into the same fp32 registers
-    //    (R from shared memory, staged by the control warp)
+    // 10) rank-r correction A_i R^T, accumulated into the same fp32 registers
+    //     (R from shared memory, staged by the control warp)
     if (has_corr) {
         mbar_wait(rbar, 0u, args.status);
         const __half* a_lo = as + (fslot * 16 + g) * (r + 8);
@@ -853,7 +855,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         }
     }
 
-    // 8) fp16 outputs (round to nearest even)
+    // 11) fp16 outputs (round to nearest even)
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
         const int tk = n * 8 + 2 * t;
