@@ -225,3 +225,22 @@ def test_energy_capture_invariances_and_range():
     Q, _ = np.linalg.qr(g.standard_normal((m, m)))                # rows mixed orthogonally
     assert [oracle.energy_capture(Q @ E, Sh, r) for r in range(1, d + 1)] == pytest.approx(base, rel=1e-10)
     assert [oracle.energy_capture(7.0 * E, Sh, r) for r in range(1, d + 1)] == pytest.approx(base, rel=1e-10)
+
+
+def test_qr_core_is_lossless_and_whitened_split_is_balanced():
+    """Key design 3: the thin QR core keeps the singular values of E Sx^{1/2}
+    (left-orthogonal invariance), and the lifted factors are balanced in the
+    whitened metric: A^T A = (B Sx^{1/2})(B Sx^{1/2})^T = diag(sigma_1..r)."""
+    d, r = 24, 5
+    E = _stacked_error(d, [20, 12, 12], seed=23) * 100.0
+    basis = synth.orthogonal_basis(d, seed=23)
+    Sh, Shp = synth.covariance_half(basis, synth.power_law_spectrum(d, 1.19))
+    _, Re = oracle.householder_qr(E)
+    sv_core = oracle.jacobi_svd(oracle.matmul(Re, Sh))[1]
+    sv_full = np.linalg.svd(E @ Sh, compute_uv=False)
+    assert np.allclose(sv_core, sv_full[:sv_core.size], rtol=1e-11, atol=1e-12 * sv_full[0])
+    A, B, sing = oracle.group_solve(E, Sh, Shp, r)
+    assert np.allclose(sing, sv_full[:r], rtol=1e-11)
+    assert np.allclose(A.T @ A, np.diag(sing), rtol=1e-9, atol=1e-9 * sing[0])
+    BS = B @ Sh
+    assert np.allclose(BS @ BS.T, np.diag(sing), rtol=1e-9, atol=1e-9 * sing[0])
