@@ -76,11 +76,26 @@ def _declare(L):
     L.ora_group_solve.argtypes = [_p, _i64, _i64, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p]
     L.ora_select_restore.argtypes = [_p, _p, _p, _p, _i32, _i32, _p, _p, _p]
     L.ora_select_by_score.argtypes = [_p, _p, _p, _i32, _i32, _p, _p]
+    L.ora_e2m1_decode.argtypes = [C.c_uint8]
+    L.ora_e2m1_decode.restype = C.c_double
+    L.ora_e2m1_encode.argtypes = [C.c_float]
+    L.ora_e2m1_encode.restype = C.c_uint8
+    L.ora_e4m3_decode.argtypes = [C.c_uint8]
+    L.ora_e4m3_decode.restype = C.c_double
+    L.ora_e4m3_encode.argtypes = [C.c_float]
+    L.ora_e4m3_encode.restype = C.c_uint8
+    L.ora_e8m0_decode.argtypes = [C.c_uint8]
+    L.ora_e8m0_decode.restype = C.c_double
+    L.ora_quantize_mxfp4.argtypes = [_p, _i64, _i64, _p, _p]
+    L.ora_dequant_mxfp4.argtypes = [_p, _p, _i64, _i64, _p]
+    L.ora_quantize_nvfp4.argtypes = [_p, _i64, _i64, _p, _p, _p]
+    L.ora_dequant_nvfp4.argtypes = [_p, _p, C.c_float, _i64, _i64, _p]
     for name in ("ora_quantize_int4", "ora_unpack_int4", "ora_dequant_int4", "ora_quant_error",
                  "ora_anchor_project", "ora_module_forward", "ora_solo_forward",
                  "ora_module_forward_sampled", "ora_matmul", "ora_householder_qr",
                  "ora_jacobi_svd", "ora_rsvd", "ora_group_solve", "ora_select_restore",
-                 "ora_select_by_score"):
+                 "ora_select_by_score", "ora_quantize_mxfp4", "ora_dequant_mxfp4", "ora_quantize_nvfp4",
+                 "ora_dequant_nvfp4"):
         getattr(L, name).restype = C.c_int
 
 
@@ -279,6 +294,68 @@ def group_solve(E_cat, Sh, Shp, r, p=16, q=2, Omega=None):
     _check(lib().ora_group_solve(_ptr(E), m, d, _ptr(Sh), _ptr(Shp), r, p, q, _ptr(Om), _ptr(A),
                                  _ptr(B), _ptr(sing)), "group_solve")
     return A, B, sing
+
+
+# -- narrow floating-point base weights (Table 13: MXFP4, NVFP4) ------------------
+
+def e2m1_decode(code: int) -> float:
+    return float(lib().ora_e2m1_decode(int(code)))
+
+
+def e2m1_encode(v: float) -> int:
+    return int(lib().ora_e2m1_encode(float(v)))
+
+
+def e4m3_decode(code: int) -> float:
+    return float(lib().ora_e4m3_decode(int(code)))
+
+
+def e4m3_encode(v: float) -> int:
+    return int(lib().ora_e4m3_encode(float(v)))
+
+
+def e8m0_decode(code: int) -> float:
+    return float(lib().ora_e8m0_decode(int(code)))
+
+
+def quantize_mxfp4(W):
+    """W (O x d fp32, d % 32 == 0) -> (codes uint8 [O, d/2], scales uint8 E8M0 [O, d/32])."""
+    W = _c(W, np.float32)
+    O, d = W.shape
+    codes = np.zeros((O, d // 2), np.uint8)
+    scales = np.zeros((O, d // 32), np.uint8)
+    _check(lib().ora_quantize_mxfp4(_ptr(W), O, d, _ptr(codes), _ptr(scales)), "quantize_mxfp4")
+    return codes, scales
+
+
+def dequant_mxfp4(codes, scales, d):
+    """-> w_hat fp16 bits [O, d] (uint16)."""
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    O = codes.shape[0]
+    out = np.zeros((O, d), np.uint16)
+    _check(lib().ora_dequant_mxfp4(_ptr(codes), _ptr(scales), O, d, _ptr(out)), "dequant_mxfp4")
+    return out
+
+
+def quantize_nvfp4(W):
+    """W (O x d fp32, d % 16 == 0) -> (codes uint8 [O, d/2], scales uint8 E4M3 [O, d/16], tensor scale)."""
+    W = _c(W, np.float32)
+    O, d = W.shape
+    codes = np.zeros((O, d // 2), np.uint8)
+    scales = np.zeros((O, d // 16), np.uint8)
+    ts = np.zeros(1, np.float32)
+    _check(lib().ora_quantize_nvfp4(_ptr(W), O, d, _ptr(codes), _ptr(scales), _ptr(ts)), "quantize_nvfp4")
+    return codes, scales, float(ts[0])
+
+
+def dequant_nvfp4(codes, scales, tensor_scale, d):
+    """-> w_hat fp16 bits [O, d] (uint16)."""
+    codes, scales = _c(codes, np.uint8), _c(scales, np.uint8)
+    O = codes.shape[0]
+    out = np.zeros((O, d), np.uint16)
+    _check(lib().ora_dequant_nvfp4(_ptr(codes), _ptr(scales), C.c_float(tensor_scale), O, d, _ptr(out)),
+           "dequant_nvfp4")
+    return out
 
 
 def energy_capture(E_cat, Sh, r):

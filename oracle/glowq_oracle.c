@@ -682,3 +682,185 @@ int ora_select_restore(const double* err_fro2, const double* w_fro2,
     free(sc);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Narrow floating-point base weights (thelatestinai.com GlowQ page, Table  */
+/* 13: MXFP4 and NVFP4 as alternative base datatypes under GlowQ).          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * The pages report only perplexities for these datatypes; the formats are
+ * taken from their public definitions, and every choice below is a reading:
+ *   - E2M1 element (4 bits): sign bit 3, exponent bits 2..1 with bias 1,
+ *     mantissa bit 0; exponent 0 is subnormal (value m * 0.5).  Magnitudes
+ *     0, 0.5, 1, 1.5, 2, 3, 4, 6.  Encoding: nearest magnitude, ties to the
+ *     code whose mantissa bit is 0, saturation to 6; zero and NaN give code 0.
+ *   - E4M3 (FN) scale: sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+ *     infinity, largest finite 448; round to nearest even, saturating at 448
+ *     (a reading: some converters return NaN on overflow instead).
+ *   - E8M0 scale: value 2^(e - 127) for e in 0..254.
+ *   - MXFP4: blocks of 32 consecutive k of one row; shared scale
+ *     X = 2^(floor(log2(amax)) - 2) (2 = the largest E2M1 exponent), E8M0
+ *     code clamped to 0..254, X = 2^-127 for an all-zero block; elements
+ *     E2M1(w / X) (so |w / X| in [6, 8) saturates to 6).
+ *   - NVFP4: blocks of 16; one fp32 tensor scale
+ *     s_t = amax_tensor / (6 * 448) (1 for an all-zero tensor); block scale
+ *     S = E4M3(amax_block / (6 * s_t)); elements E2M1(w / (dec(S) * s_t)),
+ *     zero when dec(S) == 0.  Scale arithmetic in IEEE fp32, no fused
+ *     multiply-add, like the INT4 quantiser.
+ *   - packing: two codes per byte, even k in the low nibble; one scale byte
+ *     per block, row-major [O][d / block].
+ *   - the W4A16 operand is w_hat = fp16_RN(exact dequantised value), one
+ *     rounding, as for INT4.
+ */
+
+double ora_e2m1_decode(uint8_t c)
+{
+    int s = (c >> 3) & 1, e = (c >> 1) & 3, m = c & 1;
+    double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return s ? -mag : mag;
+}
+
+uint8_t ora_e2m1_encode(float v)
+{
+    if (!(v == v) || v == 0.0f) return 0;
+    double a = fabs((double)v);
+    int best = 0;
+    double bestd = INFINITY;
+    for (int c = 0; c < 8; ++c) {                     /* non-negative codes */
+        double dlt = fabs(a - ora_e2m1_decode((uint8_t)c));
+        if (dlt < bestd || (dlt == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+            bestd = dlt;
+            best = c;
+        }
+    }
+    if (a > 6.0) best = 7;                            /* saturate */
+    if (best == 0) return 0;
+    return (uint8_t)(best | (v < 0.0f ? 8 : 0));
+}
+
+double ora_e4m3_decode(uint8_t c)
+{
+    int s = (c >> 7) & 1, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+uint8_t ora_e4m3_encode(float v)
+{
+    if (!(v == v)) return 0x7f;
+    double a = fabs((double)v);
+    int sign = v < 0.0f ? 0x80 : 0;
+    if (a >= 448.0) return (uint8_t)(sign | 0x7e);     /* saturate to 448 */
+    /* nearest of the 127 finite non-negative codes, ties to even mantissa */
+    int best = 0;
+    double bestd = INFINITY;
+    for (int c = 0; c < 0x7f; ++c) {
+        double dlt = fabs(a - ora_e4m3_decode((uint8_t)c));
+        if (dlt < bestd || (dlt == bestd && (c & 1) == 0 && (best & 1) == 1)) {
+            bestd = dlt;
+            best = c;
+        }
+    }
+    return (uint8_t)(best == 0 ? 0 : (sign | best));
+}
+
+double ora_e8m0_decode(uint8_t e) { return e == 255 ? NAN : ldexp(1.0, (int)e - 127); }
+
+/* codes [O][d/2] (even k low nibble), scales [O][d/32] E8M0.  Returns 0 or -1. */
+int ora_quantize_mxfp4(const float* W, int64_t O, int64_t d, uint8_t* codes, uint8_t* scales)
+{
+    if (O < 0 || d < 0 || d % 32 != 0) return -1;
+    memset(codes, 0, (size_t)(O * (d / 2)));
+    for (int64_t o = 0; o < O; ++o)
+        for (int64_t b = 0; b < d / 32; ++b) {
+            const float* w = W + o * d + b * 32;
+            float amax = 0.0f;
+            for (int k = 0; k < 32; ++k)
+                if (fabsf(w[k]) > amax) amax = fabsf(w[k]);   /* NaN never compares greater */
+            int e = 0;                                          /* E8M0 code */
+            if (amax > 0.0f) {
+                int ex;
+                frexpf(amax, &ex);                               /* amax = f * 2^ex, f in [0.5, 1) */
+                e = (ex - 1) - 2 + 127;                          /* floor(log2 amax) - 2, biased */
+                if (e < 0) e = 0;
+                if (e > 254) e = 254;
+            }
+            scales[o * (d / 32) + b] = (uint8_t)e;
+            const float X = (float)ora_e8m0_decode((uint8_t)e);
+            for (int k = 0; k < 32; ++k) {
+                volatile float t = w[k] / X;
+                uint8_t c = ora_e2m1_encode(t);
+                int64_t col = b * 32 + k;
+                codes[o * (d / 2) + col / 2] |= (uint8_t)(c << (4 * (col % 2)));
+            }
+        }
+    return 0;
+}
+
+static inline uint8_t fp4_at(const uint8_t* codes, int64_t d, int64_t o, int64_t k)
+{
+    return (uint8_t)((codes[o * (d / 2) + k / 2] >> (4 * (k % 2))) & 0xfu);
+}
+
+/* w_hat = fp16_RN(e2m1 * 2^(e - 127)): out [O][d] fp16 bits. */
+int ora_dequant_mxfp4(const uint8_t* codes, const uint8_t* scales, int64_t O, int64_t d, uint16_t* out)
+{
+    if (O < 0 || d < 0 || d % 32 != 0) return -1;
+    for (int64_t o = 0; o < O; ++o)
+        for (int64_t k = 0; k < d; ++k)
+            out[o * d + k] = ora_f64_to_f16(ora_e2m1_decode(fp4_at(codes, d, o, k)) *
+                                            ora_e8m0_decode(scales[o * (d / 32) + k / 32]));
+    return 0;
+}
+
+/* codes [O][d/2], scales [O][d/16] E4M3, *tensor_scale fp32.  Returns 0 or -1. */
+int ora_quantize_nvfp4(const float* W, int64_t O, int64_t d, uint8_t* codes, uint8_t* scales,
+                       float* tensor_scale)
+{
+    if (O < 0 || d < 0 || d % 16 != 0) return -1;
+    memset(codes, 0, (size_t)(O * (d / 2)));
+    float amax_t = 0.0f;
+    for (int64_t i = 0; i < O * d; ++i)
+        if (fabsf(W[i]) > amax_t) amax_t = fabsf(W[i]);
+    volatile float st = amax_t / (6.0f * 448.0f);
+    if (!(st > 0.0f)) st = 1.0f;
+    *tensor_scale = st;
+    for (int64_t o = 0; o < O; ++o)
+        for (int64_t b = 0; b < d / 16; ++b) {
+            const float* w = W + o * d + b * 16;
+            float amax = 0.0f;
+            for (int k = 0; k < 16; ++k)
+                if (fabsf(w[k]) > amax) amax = fabsf(w[k]);
+            volatile float six_st = 6.0f * st;
+            volatile float sb = amax / six_st;
+            uint8_t S = ora_e4m3_encode(sb);
+            scales[o * (d / 16) + b] = S;
+            volatile float dec = (float)ora_e4m3_decode(S);
+            volatile float full = dec * st;
+            for (int k = 0; k < 16; ++k) {
+                uint8_t c = 0;
+                if (full > 0.0f) {
+                    volatile float t = w[k] / full;
+                    c = ora_e2m1_encode(t);
+                }
+                int64_t col = b * 16 + k;
+                codes[o * (d / 2) + col / 2] |= (uint8_t)(c << (4 * (col % 2)));
+            }
+        }
+    return 0;
+}
+
+/* w_hat = fp16_RN(e2m1 * e4m3 * s_t), the product taken exactly: out [O][d] fp16 bits. */
+int ora_dequant_nvfp4(const uint8_t* codes, const uint8_t* scales, float tensor_scale, int64_t O, int64_t d,
+                      uint16_t* out)
+{
+    if (O < 0 || d < 0 || d % 16 != 0) return -1;
+    for (int64_t o = 0; o < O; ++o)
+        for (int64_t k = 0; k < d; ++k)
+            out[o * d + k] = ora_f64_to_f16(ora_e2m1_decode(fp4_at(codes, d, o, k)) *
+                                            ora_e4m3_decode(scales[o * (d / 16) + k / 16]) *
+                                            (double)tensor_scale);
+    return 0;
+}
