@@ -90,12 +90,14 @@ def _declare(L):
     L.ora_dequant_mxfp4.argtypes = [_p, _p, _i64, _i64, _p]
     L.ora_quantize_nvfp4.argtypes = [_p, _i64, _i64, _p, _p, _p]
     L.ora_dequant_nvfp4.argtypes = [_p, _p, C.c_float, _i64, _i64, _p]
+    L.ora_quantize_act_e4m3.argtypes = [_p, _i64, _i64, _p, _p]
+    L.ora_dequant_act_e4m3.argtypes = [_p, _p, _i64, _i64, _p]
     for name in ("ora_quantize_int4", "ora_unpack_int4", "ora_dequant_int4", "ora_quant_error",
                  "ora_anchor_project", "ora_module_forward", "ora_solo_forward",
                  "ora_module_forward_sampled", "ora_matmul", "ora_householder_qr",
                  "ora_jacobi_svd", "ora_rsvd", "ora_group_solve", "ora_select_restore",
                  "ora_select_by_score", "ora_quantize_mxfp4", "ora_dequant_mxfp4", "ora_quantize_nvfp4",
-                 "ora_dequant_nvfp4"):
+                 "ora_dequant_nvfp4", "ora_quantize_act_e4m3", "ora_dequant_act_e4m3"):
         getattr(L, name).restype = C.c_int
 
 
@@ -356,6 +358,41 @@ def dequant_nvfp4(codes, scales, tensor_scale, d):
     _check(lib().ora_dequant_nvfp4(_ptr(codes), _ptr(scales), C.c_float(tensor_scale), O, d, _ptr(out)),
            "dequant_nvfp4")
     return out
+
+
+def quantize_act_e4m3(X_bits):
+    """Per-token FP8 E4M3 activations: X (T x d fp16 bits) -> (codes uint8 [T, d], scales fp32 [T])."""
+    X = _c(X_bits, np.uint16)
+    T, d = X.shape
+    codes = np.zeros((T, d), np.uint8)
+    scales = np.zeros(T, np.float32)
+    _check(lib().ora_quantize_act_e4m3(_ptr(X), T, d, _ptr(codes), _ptr(scales)), "quantize_act_e4m3")
+    return codes, scales
+
+
+def dequant_act_e4m3(codes, scales):
+    codes, scales = _c(codes, np.uint8), _c(scales, np.float32)
+    T, d = codes.shape
+    out = np.zeros((T, d), np.float64)
+    _check(lib().ora_dequant_act_e4m3(_ptr(codes), _ptr(scales), T, d, _ptr(out)), "dequant_act_e4m3")
+    return out
+
+
+def w4a8_group_forward(mods, B_bits, X_bits, group_size: int = 128):
+    """W4A8 group forward (reading): the layer consumes the per-token FP8
+    activations X_hat; R = X_hat B^T and Y_i = X_hat w_hat_i^T + R A_i^T, float64.
+    mods: (q, s, z, A_bits or None).  Returns ([Y_i], R, X_hat)."""
+    Xh = dequant_act_e4m3(*quantize_act_e4m3(X_bits))
+    d = Xh.shape[1]
+    R = None if B_bits is None else matmul(Xh, f16_bits_to_f64(B_bits), tb=True)
+    outs = []
+    for (q, s, z, A) in mods:
+        What = f16_bits_to_f64(dequant_int4(q, s, z, d, group_size))
+        Y = matmul(Xh, What, tb=True)
+        if A is not None and R is not None:
+            Y = Y + matmul(R, f16_bits_to_f64(A), tb=True)
+        outs.append(Y)
+    return outs, R, Xh
 
 
 def energy_capture(E_cat, Sh, r):

@@ -864,3 +864,46 @@ int ora_dequant_nvfp4(const uint8_t* codes, const uint8_t* scales, float tensor_
                                             (double)tensor_scale);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* FP8 activations for W4A8 (GlowQ pages: W4A8 alongside W4A16, Tables      */
+/* 14-15 of the thelatestinai.com page; the format is not defined there).    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Readings: each token (row of X) gets one fp32 scale s = amax_row / 448
+ * (1 for an all-zero row); codes = E4M3(x / s) rounded to nearest even and
+ * saturating; the dequantised activation is the exact product dec(code) * s.
+ * The whole layer (base product and the projection R) consumes the
+ * dequantised activations.
+ * X: T x d fp16 bits.  codes: T x d bytes, scales: T floats.
+ */
+int ora_quantize_act_e4m3(const uint16_t* X, int64_t T, int64_t d, uint8_t* codes, float* scales)
+{
+    if (T < 0 || d < 0) return -1;
+    for (int64_t t = 0; t < T; ++t) {
+        float amax = 0.0f;
+        for (int64_t k = 0; k < d; ++k) {
+            float a = fabsf((float)ora_f16_to_f64(X[t * d + k]));
+            if (a > amax) amax = a;
+        }
+        volatile float s = amax / 448.0f;
+        if (!(s > 0.0f)) s = 1.0f;
+        scales[t] = s;
+        for (int64_t k = 0; k < d; ++k) {
+            volatile float q = (float)ora_f16_to_f64(X[t * d + k]) / s;
+            codes[t * d + k] = ora_e4m3_encode(q);
+        }
+    }
+    return 0;
+}
+
+/* out: T x d float64, dec(code) * s exactly. */
+int ora_dequant_act_e4m3(const uint8_t* codes, const float* scales, int64_t T, int64_t d, double* out)
+{
+    if (T < 0 || d < 0) return -1;
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t k = 0; k < d; ++k)
+            out[t * d + k] = ora_e4m3_decode(codes[t * d + k]) * (double)scales[t];
+    return 0;
+}
