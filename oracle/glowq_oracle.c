@@ -20,13 +20,18 @@
  *                 pseudo-inverse;
  *       design 4  R = X B_shared^T computed once per input-sharing group,
  *                 y_i = W_i^(q) X + A_i R; solo modules inline; GlowQ-S top-k
- *                 by g_ner(u) = ||E_u||_F^2 / ||W_u||_F^2 with layer-order
- *                 fallback when the signal is weak;
+ *                 by an importance score (g_ner(u) = ||E_u||_F^2 / ||W_u||_F^2
+ *                 or the GSVD energy capture g_ec, composed in the Python
+ *                 layer from the QR and SVD below) with layer-order fallback
+ *                 when the signal is weak;
  *       set-up    W4A16, INT4 weights with group size 128, fp16 activations,
  *                 rank 64.
  *   - thelatestinai.com, GlowQ page: Table 6 (notation and shapes),
  *     Table 11 caption (exact SVD vs Halko randomised SVD on the core M),
- *     Table 12 (p = 16 with q = 2 as the fixed values of the sweeps).
+ *     Table 12 (p = 16 with q = 2 as the fixed values of the sweeps),
+ *     Table 13 (MXFP4 / NVFP4 base weights) and Tables 14-15 (W4A8): the
+ *     formats are not defined there; the sections at the end of this file
+ *     state the readings taken.
  *
  * Readings where the pages are silent (each also listed in the design notes):
  *   - the INT4 quantiser is asymmetric round-to-nearest per (row, 128-group):
