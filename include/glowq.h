@@ -165,23 +165,29 @@ GLOWQ_API glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, co
  * counterpart: this is a deployment convenience of this library).
  *
  * Same computation and arguments as glowq_solo_forward, minus the workspace:
- * the scratch it needs (R and, for T <= 16, its split-d partial sums) lives
- * in a fixed array compiled into the library, glowq_noalloc_scratch_bytes()
- * (1 MiB) on every device that loads the library, held until process exit.
- * It is meant for callers that cannot allocate device memory when they call
- * -- e.g. a custom op or plugin running inside another runtime's enqueue step,
- * where that runtime owns every device allocation.  The call itself performs
- * no cudaMalloc/cudaFree and no other allocation of device memory.
+ * the scratch it needs (the hand-off flags, R and, for T > 16, the split-d
+ * partial sums of R) lives in a fixed array compiled into the library,
+ * glowq_noalloc_scratch_bytes() (1 MiB) on every device that loads the
+ * library, held until process exit.  It is meant for callers that cannot
+ * allocate device memory when they call -- e.g. a custom op or plugin running
+ * inside another runtime's enqueue step, where that runtime owns every device
+ * allocation.  The call itself performs no cudaMalloc/cudaFree and no other
+ * allocation of device memory.
  *   - Sizes whose scratch need, glowq_workspace_bytes(T, r), exceeds
  *     glowq_noalloc_scratch_bytes() are rejected with GLOWQ_ERR_SHAPE before
- *     anything is enqueued (at r = 64 that is T > 8192).
+ *     anything is enqueued.  At r = 64 the largest accepted T is 481 (for
+ *     T > 16 the split-d partial sums need 8 x T x r x 4 bytes).
  *   - The first call on a device looks up the array's device address (once per
- *     device, with that device current); make that first call before any
+ *     device, with that device current) and keeps it for the life of the CUDA
+ *     context (not across a cudaDeviceReset); make that first call before any
  *     stream capture.
- *   - All calls on a device share the one array: calls that may overlap on the
- *     GPU (different streams without ordering between them) race on it.  The
- *     array keeps the last call's contents; every value a call reads there is
- *     written earlier by the same call, so nothing needs clearing.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents: calls that may overlap on the GPU (different streams without
+ *     ordering between them) race on it.  Each call (r > 0) first clears the
+ *     array's 256 flag bytes on `stream` (cudaMemsetAsync, which allocates
+ *     nothing), so flags left non-zero by a failed or timed-out call never
+ *     reach the next one; every other value a call reads there is written
+ *     earlier by the same call.
  */
 GLOWQ_API glowq_status glowq_solo_forward_noalloc(const glowq_module* mod, int64_t d, const uint16_t* B,
                                                   int32_t r, const uint16_t* X, int64_t T, void* stream);

@@ -85,6 +85,12 @@ static glowq_status validate_forward(const glowq_module* mods, int32_t m, int64_
     return GLOWQ_OK;
 }
 
+// Host-side validation of a solo call (exported to the other translation units).
+glowq_status validate_solo_call(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r, const uint16_t* X,
+                                int64_t T) {
+    return validate_forward(mod, 1, d, B, r, X, T);
+}
+
 static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
                                  const uint16_t* X, int64_t T, uint16_t* R, void* workspace, size_t ws_bytes,
                                  cudaStream_t st) {

@@ -23,6 +23,10 @@ struct ModuleView {
 
 constexpr int kDecodeMaxTokens = 16;
 
+// Argument checks of glowq_solo_forward, without the workspace (api.cu).
+glowq_status validate_solo_call(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r, const uint16_t* X,
+                                int64_t T);
+
 // Device address of this device's status word (bounded-wait timeouts).
 unsigned int* device_status_ptr();
 

@@ -1,19 +1,22 @@
-"""The allocation-free solo forward matches the regular solo forward.
+"""The allocation-free solo forward matches the oracle.
 
 glowq_solo_forward_noalloc is for callers that cannot allocate device memory
 at call time (for example a custom op or plugin inside another runtime's
 enqueue step, where that runtime owns every allocation): it takes no workspace
-and uses a fixed scratch array compiled into the library.  This file runs last
-(pytest collects it after the others) and passes alone or after the suite.
+and uses a fixed scratch array compiled into the library.  Every call shares
+that array, so each test makes two calls in a row with different inputs and
+checks both against the CPU oracle.  This file runs last (pytest collects it
+after the others) and passes alone or after the suite.
 """
 import ctypes as C
 
 import numpy as np
 import pytest
 
+import oracle
 from rank_error_correction_b200 import build, glowq, synth
 
-from helpers import TOL, attach_random_factors, make_modules, normwise, to_dev
+from helpers import check, TOL, attach_random_factors, make_modules, normwise, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -28,28 +31,64 @@ def _lib():
     assert glowq.device_status() == 0
 
 
-@pytest.mark.parametrize("d,O,T", [(1024, 256, 8), (4096, 256, 16), (512, 144, 300)])
-def test_noalloc_matches_solo_forward_twice(d, O, T):
+def _noalloc(m, d, Bt, r, X, O):
+    """One call through the C ABI; returns (status, Y on the host)."""
+    import torch
+    T = X.shape[0]
+    Y = torch.full((T, O), float("nan"), dtype=torch.float16, device="cuda")
+    arr = glowq._module_structs([m], [Y], True)
+    rc = glowq.lib().glowq_solo_forward_noalloc(arr, d, Bt.data_ptr(), r, X.data_ptr(), T,
+                                                 C.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    return rc, Y.cpu().numpy().astype(np.float64)
+
+
+def _largest_T(r):
+    cap = glowq.noalloc_scratch_bytes()
+    T = 1
+    while glowq.workspace_bytes(T + 1, r) <= cap:
+        T += 1
+    return T
+
+
+@pytest.mark.parametrize("d,O,T", [(4096, 256, 1), (4096, 256, 16), (512, 144, 300)])
+def test_noalloc_matches_oracle_twice(d, O, T):
     import torch
     r = 64
     mods = make_modules(d, [O], seed=90 + T)
     B = attach_random_factors(mods, d, r, seed=90 + T)
     m = to_dev(mods)[0]
     Bt = torch.from_numpy(B).cuda()
-    ref = glowq.solo_forward(m, Bt, torch.from_numpy(synth.activations(T, d, synth.ALPHA_QKV, seed=1)).cuda())
-    ref2 = glowq.solo_forward(m, Bt, torch.from_numpy(synth.activations(T, d, synth.ALPHA_QKV, seed=2)).cuda())
-    # two calls in a row through the C ABI, different inputs, shared scratch
-    for seed, want in ((1, ref), (2, ref2)):
-        X = torch.from_numpy(synth.activations(T, d, synth.ALPHA_QKV, seed=seed)).cuda()
-        Y = torch.full((T, O), float("nan"), dtype=torch.float16, device="cuda")
-        arr = glowq._module_structs([m], [Y], True)
-        rc = glowq.lib().glowq_solo_forward_noalloc(arr, d, Bt.data_ptr(), r, X.data_ptr(), T,
-                                                     C.c_void_p(torch.cuda.current_stream().cuda_stream))
+    h = mods[0]
+    # two calls in a row, different inputs, one shared scratch array
+    for seed in (1, 2):
+        X = synth.activations(T, d, synth.ALPHA_QKV, seed=seed)
+        rc, got = _noalloc(m, d, Bt, r, torch.from_numpy(X).cuda(), O)
         assert rc == 0
-        torch.cuda.synchronize()
-        got = Y.cpu().numpy().astype(np.float64)
         assert np.all(np.isfinite(got))
-        assert normwise(got, want.cpu().numpy().astype(np.float64)) < TOL
+        ref = oracle.solo_forward(h.q, h.s, h.z, synth.bits(h.A), synth.bits(B), synth.bits(X))
+        check(got, ref)
+
+
+def test_noalloc_size_boundary():
+    """The largest T whose scratch need fits is accepted and correct; T + 1 is rejected."""
+    import torch
+    r, d, O = 64, 256, 64
+    Tmax = _largest_T(r)
+    assert Tmax == 481                       # 256 + 8*T*r*4 + align256(T*r*2) <= 1 MiB
+    mods = make_modules(d, [O], seed=97)
+    B = attach_random_factors(mods, d, r, seed=97)
+    m = to_dev(mods)[0]
+    Bt = torch.from_numpy(B).cuda()
+    h = mods[0]
+    X = synth.activations(Tmax + 1, d, synth.ALPHA_QKV, seed=97)
+    rc, got = _noalloc(m, d, Bt, r, torch.from_numpy(X[:Tmax]).cuda(), O)
+    assert rc == 0
+    ref = oracle.solo_forward(h.q, h.s, h.z, synth.bits(h.A), synth.bits(B), synth.bits(X[:Tmax]))
+    check(got, ref)
+    rc, got = _noalloc(m, d, Bt, r, torch.from_numpy(X).cuda(), O)
+    assert rc == 2                           # GLOWQ_ERR_SHAPE, nothing enqueued
+    assert np.all(np.isnan(got))             # output untouched
 
 
 def test_noalloc_rejects_oversized_requests():
@@ -67,3 +106,24 @@ def test_noalloc_rejects_oversized_requests():
     arr = glowq._module_structs([m], [Y], True)
     rc = glowq.lib().glowq_solo_forward_noalloc(arr, 256, B.data_ptr(), 64, X.data_ptr(), T, None)
     assert rc == 2                   # GLOWQ_ERR_SHAPE, nothing enqueued
+
+
+def test_noalloc_after_a_timed_out_wait():
+    """A bounded wait that ran out (recorded in the device status word) leaves
+    the next allocation-free decode calls correct: each call clears the flag
+    bytes of the shared array before its kernels."""
+    import torch
+    glowq.selftest_wait_timeout(polls=64)
+    assert glowq.device_status() == 5        # GLOWQ_ERR_TIMEOUT, read and cleared
+    d, O, r = 1024, 128, 32
+    mods = make_modules(d, [O], seed=98)
+    B = attach_random_factors(mods, d, r, seed=98)
+    m = to_dev(mods)[0]
+    Bt = torch.from_numpy(B).cuda()
+    h = mods[0]
+    for T in (1, 16):
+        X = synth.activations(T, d, synth.ALPHA_MLP, seed=98 + T)
+        rc, got = _noalloc(m, d, Bt, r, torch.from_numpy(X).cuda(), O)
+        assert rc == 0
+        ref = oracle.solo_forward(h.q, h.s, h.z, synth.bits(h.A), synth.bits(B), synth.bits(X))
+        check(got, ref)
