@@ -24,7 +24,7 @@ _SRC = os.path.join(_HERE, "glowq_oracle.c")
 _BUILD = os.path.join(_HERE, "_build")
 _LIB = os.path.join(_BUILD, "libglowq_oracle.so")
 
-CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
+CFLAGS = ["-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared"]
 
 
 def build(force: bool = False) -> str:
@@ -76,6 +76,8 @@ def _declare(L):
     L.ora_group_solve.argtypes = [_p, _i64, _i64, _p, _p, _i32, _i32, _i32, _p, _p, _p, _p]
     L.ora_select_restore.argtypes = [_p, _p, _p, _p, _i32, _i32, _p, _p, _p]
     L.ora_select_by_score.argtypes = [_p, _p, _p, _i32, _i32, _p, _p]
+    L.ora_set_threads.argtypes = [_i32]
+    L.ora_set_threads.restype = C.c_int
     L.ora_e2m1_decode.argtypes = [C.c_uint8]
     L.ora_e2m1_decode.restype = C.c_double
     L.ora_e2m1_encode.argtypes = [C.c_float]
@@ -243,6 +245,12 @@ def module_forward_sampled(q, s, z, A_bits, B_bits, X_bits, t_idx, o_idx, group_
 
 
 # -- offline solve -----------------------------------------------------------------
+
+def set_threads(n: int = 0) -> int:
+    """OpenMP threads of the forward loops (n >= 1 sets it; 0 only queries).
+    Results do not depend on it: each output is one sequential sum."""
+    return int(lib().ora_set_threads(int(n)))
+
 
 def matmul(A, B, ta=False, tb=False):
     A, B = _c(A, np.float64), _c(B, np.float64)

@@ -48,9 +48,15 @@
  *
  * Parity pins for every function live in tests/test_oracle_*.py.
  *
- * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared.
+ * Threads: the forward functions split independent outputs (tokens of R,
+ * rows of Y, samples) across OpenMP threads; each output is still one
+ * sequential float64 sum in k order, so the result does not depend on the
+ * thread count.  ora_set_threads() fixes the count (1 = single-threaded).
+ *
+ * Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -fno-fast-math -fPIC -shared.
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -220,6 +226,7 @@ int ora_anchor_project(const uint16_t* X, const uint16_t* B, int64_t T,
                        int64_t d, int32_t r, double* R)
 {
     if (T < 0 || d < 0 || r < 0) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
     for (int64_t t = 0; t < T; ++t)
         for (int32_t j = 0; j < r; ++j) {
             double acc = 0.0;
@@ -242,31 +249,42 @@ int ora_module_forward(const uint32_t* q, const uint16_t* s, const uint8_t* z,
                        double* Y)
 {
     if (O < 0 || d < 0 || T < 0 || gs <= 0 || d % gs != 0) return -1;
-    double* whd = (double*)malloc((size_t)(d > 0 ? d : 1) * sizeof(double));
     double* xd = (double*)malloc((size_t)(T * d > 0 ? T * d : 1) * sizeof(double));
-    if (!whd || !xd) { free(whd); free(xd); return -2; }
+    if (!xd) return -2;
     for (int64_t i = 0; i < T * d; ++i) xd[i] = ora_f16_to_f64(X[i]);
     int64_t ng = d / gs;
-    for (int64_t o = 0; o < O; ++o) {
-        for (int64_t k = 0; k < d; ++k) {
-            int64_t g = k / gs;
-            double prod = (double)(code_at(q, d, o, k) - (int)z[o * ng + g]) *
-                          ora_f16_to_f64(s[o * ng + g]);
-            whd[k] = ora_f16_to_f64(ora_f64_to_f16(prod));
+    int failed = 0;
+#pragma omp parallel
+    {
+        /* one dequantised row per thread */
+        double* whd = (double*)malloc((size_t)(d > 0 ? d : 1) * sizeof(double));
+        if (!whd) {
+#pragma omp atomic write
+            failed = 1;
         }
-        for (int64_t t = 0; t < T; ++t) {
-            double acc = 0.0;
-            for (int64_t k = 0; k < d; ++k)
-                acc += xd[t * d + k] * whd[k];
-            if (A && r > 0 && R)
-                for (int32_t j = 0; j < r; ++j)
-                    acc += R[t * r + j] * ora_f16_to_f64(A[o * r + j]);
-            Y[t * O + o] = acc;
+#pragma omp for schedule(static)
+        for (int64_t o = 0; o < O; ++o) {
+            if (!whd) continue;
+            for (int64_t k = 0; k < d; ++k) {
+                int64_t g = k / gs;
+                double prod = (double)(code_at(q, d, o, k) - (int)z[o * ng + g]) *
+                              ora_f16_to_f64(s[o * ng + g]);
+                whd[k] = ora_f16_to_f64(ora_f64_to_f16(prod));
+            }
+            for (int64_t t = 0; t < T; ++t) {
+                double acc = 0.0;
+                for (int64_t k = 0; k < d; ++k)
+                    acc += xd[t * d + k] * whd[k];
+                if (A && r > 0 && R)
+                    for (int32_t j = 0; j < r; ++j)
+                        acc += R[t * r + j] * ora_f16_to_f64(A[o * r + j]);
+                Y[t * O + o] = acc;
+            }
         }
+        free(whd);
     }
-    free(whd);
     free(xd);
-    return 0;
+    return failed ? -2 : 0;
 }
 
 /* Solo module: its own R = X B^T computed inline, nothing shared. */
@@ -299,9 +317,11 @@ int ora_module_forward_sampled(const uint32_t* q, const uint16_t* s, const uint8
 {
     if (gs <= 0 || d % gs != 0) return -1;
     int64_t ng = d / gs;
+    for (int64_t i = 0; i < n; ++i)
+        if (t_idx[i] < 0 || t_idx[i] >= T || o_idx[i] < 0 || o_idx[i] >= O) return -1;
+#pragma omp parallel for schedule(dynamic, 16)
     for (int64_t i = 0; i < n; ++i) {
         int64_t t = t_idx[i], o = o_idx[i];
-        if (t < 0 || t >= T || o < 0 || o >= O) return -1;
         double acc = 0.0;
         for (int64_t k = 0; k < d; ++k) {
             int64_t g = k / gs;
@@ -320,6 +340,13 @@ int ora_module_forward_sampled(const uint32_t* q, const uint16_t* s, const uint8
         out[i] = acc;
     }
     return 0;
+}
+
+/* Thread count of the OpenMP loops (n >= 1); returns the count in effect. */
+int ora_set_threads(int32_t n)
+{
+    if (n >= 1) omp_set_num_threads(n);
+    return omp_get_max_threads();
 }
 
 /* ------------------------------------------------------------------------ */

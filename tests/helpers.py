@@ -15,6 +15,17 @@ from rank_error_correction_b200 import synth
 # rounding enters only through the ~1-2% correction term.
 TOL = 2e-3
 
+# Per-element bound beside the normwise bar:
+#   |y_gpu - y_ora| <= ELEM_REL * |y_ora| + ELEM_ABS * max|y_ora|
+# ELEM_REL = 2^-10 covers the fp16 rounding of y (2^-11 relative) twice over;
+# ELEM_ABS = 2^-10 of the output's largest magnitude covers what does not scale
+# with the element itself: fp32 accumulation over d <= 14336 terms, the decode
+# kernel's exact (q - z) s weights against the oracle's fp16-rounded w_hat
+# (<= 2^-12 per weight, random in sign), and R rounded to fp16 in the
+# correction term.  Near-zero outputs are held to the absolute part only.
+ELEM_REL = 2.0 ** -10
+ELEM_ABS = 2.0 ** -10
+
 
 @dataclasses.dataclass
 class HostModule:
@@ -61,6 +72,28 @@ def attach_solved_factors(mods: List[HostModule], d: int, r: int, alpha: float, 
 def normwise(y_gpu: np.ndarray, y_ref: np.ndarray) -> float:
     den = np.linalg.norm(y_ref)
     return float(np.linalg.norm(y_gpu.astype(np.float64) - y_ref) / (den if den > 0 else 1.0))
+
+
+def elementwise_excess(y_gpu: np.ndarray, y_ref: np.ndarray, ymax: Optional[float] = None) -> float:
+    """Largest |y_gpu - y_ref| / (ELEM_REL |y_ref| + ELEM_ABS ymax); <= 1 passes."""
+    y_ref = np.asarray(y_ref, dtype=np.float64)
+    if y_ref.size == 0:
+        return 0.0
+    ymax = float(np.max(np.abs(y_ref))) if ymax is None else float(ymax)
+    bound = ELEM_REL * np.abs(y_ref) + ELEM_ABS * max(ymax, 1e-30)
+    return float(np.max(np.abs(np.asarray(y_gpu, dtype=np.float64) - y_ref) / bound))
+
+
+def check(y_gpu: np.ndarray, y_ref: np.ndarray, ymax: Optional[float] = None, tol: float = TOL) -> None:
+    """The parity bar of a module's output: normwise relative error <= tol and
+    every element inside the per-element bound."""
+    y_gpu = np.asarray(y_gpu, dtype=np.float64)
+    assert y_gpu.shape == np.shape(y_ref), (y_gpu.shape, np.shape(y_ref))
+    assert np.all(np.isfinite(y_gpu)), "non-finite output"
+    nw = normwise(y_gpu, y_ref)
+    assert nw < tol, f"normwise {nw:.3e} >= {tol:.1e}"
+    ex = elementwise_excess(y_gpu, y_ref, ymax)
+    assert ex <= 1.0, f"per-element bound exceeded by {ex:.2f}x"
 
 
 def to_dev(mods: List[HostModule], device="cuda", with_A: bool = True):

@@ -2,7 +2,8 @@
 
 Shapes span several 128-row and 256-token tiles with ragged tails in both, the
 r = 0 / disabled-module / multi-slab (r > 64) cases, and the full LLaMA-2-7B
-MLP and LLaMA-3.1-8B prefill shapes checked on sampled outputs.
+MLP and LLaMA-3.1-8B prefill shapes checked on whole output tiles (every
+element of four 256 x 256 tiles per module) and whole tokens.
 Pages: papernotes.org GlowQ summary, key design 4 and the set-up paragraph.
 """
 import numpy as np
@@ -11,7 +12,7 @@ import pytest
 import oracle
 from rank_error_correction_b200 import build, glowq, synth
 
-from helpers import TOL, attach_random_factors, make_modules, normwise, to_dev
+from helpers import check, TOL, attach_random_factors, make_modules, normwise, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -54,7 +55,7 @@ def test_prefill_group_ragged(T, r):
     assert normwise(R, R_ref) < 1e-3
     for y, ref in zip(ys, refs):
         assert y.shape == ref.shape
-        assert normwise(y, ref) < TOL
+        check(y, ref)
 
 
 @pytest.mark.parametrize("r", [0, 128, 200, 256])
@@ -66,7 +67,7 @@ def test_prefill_rank_slabs(r):
     ys, _ = _run_group(mods, B, X)
     refs, _ = _oracle_group(mods, B, X)
     for y, ref in zip(ys, refs):
-        assert normwise(y, ref) < TOL
+        check(y, ref)
 
 
 def test_prefill_disabled_module_and_ldY_views():
@@ -82,8 +83,8 @@ def test_prefill_disabled_module_and_ldY_views():
     glowq.group_forward(to_dev(mods), torch.from_numpy(B).cuda(), torch.from_numpy(X).cuda(), Ys=views)
     host = _np(buf).astype(np.float64)
     refs, _ = _oracle_group(mods, B, X)
-    assert normwise(host[:, :128], refs[0]) < TOL
-    assert normwise(host[:, 128:192], refs[1]) < TOL
+    check(host[:, :128], refs[0])
+    check(host[:, 128:192], refs[1])
     assert np.all(np.isnan(host[:, 192:]))
 
 
@@ -97,7 +98,7 @@ def test_prefill_solo_wide_input():
     Y = _np(glowq.solo_forward(to_dev(mods)[0], torch.from_numpy(B).cuda(), torch.from_numpy(X).cuda()))
     m = mods[0]
     ref = oracle.solo_forward(m.q, m.s, m.z, synth.bits(m.A), synth.bits(B), synth.bits(X))
-    assert normwise(Y.astype(np.float64), ref) < TOL
+    check(Y.astype(np.float64), ref)
 
 
 def test_prefill_deterministic():
@@ -115,41 +116,85 @@ def test_prefill_deterministic():
         assert torch.equal(x, y)
 
 
-def _sampled_check(mods, B, X, Ys, n=1500, seed=0):
-    g = np.random.default_rng(seed)
+# Output tiles of the prefill kernel: 256 W rows x 256 tokens per CTA pair.
+TILE_ROWS, TILE_TOKENS = 256, 256
+
+
+def _tiles(O, T):
+    """(rows, tokens) ranges of the first, the last and two interior output tiles."""
+    nm, nn = -(-O // TILE_ROWS), -(-T // TILE_TOKENS)
+    picks = [(0, 0), (nm - 1, nn - 1), (nm // 3, nn // 2), ((2 * nm) // 3, max(nn // 2 - 1, 0))]
+    return [((bi * TILE_ROWS, min(O, (bi + 1) * TILE_ROWS)), (bj * TILE_TOKENS, min(T, (bj + 1) * TILE_TOKENS)))
+            for bi, bj in picks]
+
+
+def _tile_check(mods, B, X, Ys, whole_tokens=(0, -1)):
+    """Every element of four whole output tiles per module (the first, the last
+    and two interior ones) and every output feature of a few whole tokens,
+    against the oracle evaluated on exactly those rows and tokens."""
     Xb, Bb = synth.bits(X), synth.bits(B)
     for m, Y in zip(mods, Ys):
         T, O = Y.shape
-        ti, oi = g.integers(0, T, n), g.integers(0, O, n)
-        ref = oracle.module_forward_sampled(m.q, m.s, m.z, synth.bits(m.A), Bb, Xb, ti, oi)
-        got = Y[ti, oi].astype(np.float64)
-        assert normwise(got, ref) < TOL
+        Ab = synth.bits(m.A)
+        pairs = []
+        for (r0, r1), (t0, t1) in _tiles(O, T):
+            Xt = Xb[t0:t1]
+            R = oracle.anchor_project(Xt, Bb)
+            ref = oracle.module_forward(m.q[r0:r1], m.s[r0:r1], m.z[r0:r1], Ab[r0:r1], R, Xt)
+            pairs.append((Y[t0:t1, r0:r1], ref))
+        for t in whole_tokens:
+            t = t % T
+            Xt = Xb[t:t + 1]
+            ref = oracle.module_forward(m.q, m.s, m.z, Ab, oracle.anchor_project(Xt, Bb), Xt)
+            pairs.append((Y[t:t + 1], ref))
+        ymax = max(float(np.max(np.abs(ref))) for _, ref in pairs)
+        for got, ref in pairs:
+            check(got.astype(np.float64), ref, ymax)
 
 
-def test_llama2_7b_mlp_prefill_sampled():
-    """gate/up 2 x 11008x4096 group + down_proj 4096x11008 solo, r=64, T=2048 (sampled outputs)."""
+def test_llama2_7b_mlp_prefill_tiles():
+    """gate/up 2 x 11008x4096 group + down_proj 4096x11008 solo, r=64, T=2048 (whole tiles)."""
     import torch
     d, r, T = 4096, 64, 2048
     gu = make_modules(d, [11008, 11008], seed=0, sub0=30)
     Bg = attach_random_factors(gu, d, r, seed=0, sub=30)
     X = synth.activations(T, d, synth.ALPHA_MLP, seed=0)
     Ys, _ = glowq.group_forward(to_dev(gu), torch.from_numpy(Bg).cuda(), torch.from_numpy(X).cuda())
-    _sampled_check(gu, Bg, X, [_np(Y) for Y in Ys])
+    _tile_check(gu, Bg, X, [_np(Y) for Y in Ys])
     down = make_modules(11008, [4096], seed=0, sub0=40)
     Bd = attach_random_factors(down, 11008, r, seed=0, sub=40)
     Xd = synth.activations(T, 11008, synth.ALPHA_MLP, seed=0, sub=1)
     Yd = glowq.solo_forward(to_dev(down)[0], torch.from_numpy(Bd).cuda(), torch.from_numpy(Xd).cuda())
-    _sampled_check(down, Bd, Xd, [_np(Yd)])
+    _tile_check(down, Bd, Xd, [_np(Yd)])
 
 
-def test_llama31_8b_qkv_prefill_t4096_sampled():
+def test_llama31_8b_qkv_prefill_t4096_tiles():
+    """GQA Q/K/V group 4096/1024/1024 x 4096, r=64, T=4096 (whole tiles)."""
     import torch
     d, r, T = 4096, 64, 4096
     qkv = make_modules(d, [4096, 1024, 1024], seed=1, sub0=50)
     B = attach_random_factors(qkv, d, r, seed=1, sub=50)
     X = synth.activations(T, d, synth.ALPHA_QKV, seed=1)
     Ys, _ = glowq.group_forward(to_dev(qkv), torch.from_numpy(B).cuda(), torch.from_numpy(X).cuda())
-    _sampled_check(qkv, B, X, [_np(Y) for Y in Ys])
+    _tile_check(qkv, B, X, [_np(Y) for Y in Ys])
+
+
+def test_llama31_8b_mlp_prefill_t4096_tiles():
+    """gate/up 2 x 14336x4096 group (shared B) and down_proj 4096x14336 solo, r=64,
+    T=4096, alpha=0.77 (whole tiles)."""
+    import torch
+    d, ffn, r, T = 4096, 14336, 64, 4096
+    gu = make_modules(d, [ffn, ffn], seed=1, sub0=60)
+    Bg = attach_random_factors(gu, d, r, seed=1, sub=60)
+    X = synth.activations(T, d, synth.ALPHA_MLP, seed=1, sub=2)
+    Ys, _ = glowq.group_forward(to_dev(gu), torch.from_numpy(Bg).cuda(), torch.from_numpy(X).cuda())
+    _tile_check(gu, Bg, X, [_np(Y) for Y in Ys])
+    del Ys
+    down = make_modules(ffn, [d], seed=1, sub0=70)
+    Bd = attach_random_factors(down, ffn, r, seed=1, sub=70)
+    Xd = synth.activations(T, ffn, synth.ALPHA_MLP, seed=1, sub=3)
+    Yd = glowq.solo_forward(to_dev(down)[0], torch.from_numpy(Bd).cuda(), torch.from_numpy(Xd).cuda())
+    _tile_check(down, Bd, Xd, [_np(Yd)])
 
 
 def test_prefill_eight_modules_small_outputs():
@@ -164,4 +209,4 @@ def test_prefill_eight_modules_small_outputs():
     assert normwise(R, R_ref) < 1e-3
     for y, ref in zip(ys, refs):
         assert y.shape == ref.shape
-        assert normwise(y, ref) < TOL
+        check(y, ref)

@@ -19,7 +19,7 @@ import pytest
 import oracle
 from rank_error_correction_b200 import glowq, synth
 
-from helpers import TOL, normwise
+from helpers import TOL, check, normwise
 
 pytestmark = pytest.mark.gpu
 
@@ -140,8 +140,8 @@ def test_stack_forward_matches_oracle(stack, T):
                                                 u["B_bits"] if restore else None, Xb, ti, oi)
             got = Y.cpu().numpy()[ti, oi].astype(np.float64)
             assert np.all(np.isfinite(got))
-            err = normwise(got, ref)
-            assert err < TOL, (u["name"], u["layer"], bool(restore), T, err)
+            assert normwise(got, ref) < TOL, (u["name"], u["layer"], bool(restore), T)
+            check(got, ref)
 
 
 @pytest.mark.parametrize("T", [1, 64])
@@ -163,5 +163,4 @@ def test_layerwise_mode_matches_oracle(stack, T):
         ti, oi = g.integers(0, T, n), g.integers(0, qh.shape[0], n)
         ref = oracle.module_forward_sampled(qh, sh, zh, synth.bits(As[0].cpu().numpy()), synth.bits(B.cpu().numpy()),
                                             Xb, ti, oi)
-        err = normwise(Y.cpu().numpy()[ti, oi].astype(np.float64), ref)
-        assert err < TOL, (i, T, err)
+        check(Y.cpu().numpy()[ti, oi].astype(np.float64), ref)
