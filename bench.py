@@ -418,53 +418,109 @@ def time_prefill(T, steps, warmup, device, n_rep=2, seed=0, eager_steps=None, ra
 
 # ------------------------------------------------------------ oracle timing
 
-def oracle_sample(T=1, rows_per_module=512, seed=0):
-    """Oracle forward (float64 C, one thread) over a row sample of every module of the step."""
-    import numpy as np
+_ORACLE_STEP = None
+
+
+def oracle_step_inputs(T=1, seed=0):
+    """Host inputs of one whole decode step for the CPU oracle: the Q/K/V group
+    (3 x 4096 x 4096) and the o_proj solo (4096 x 4096), INT4 g128 packed by
+    the oracle's own quantiser, r = 64 stand-in factors of the solve's
+    magnitude, X of T tokens.  Built once per process."""
+    global _ORACLE_STEP
+    if _ORACLE_STEP is None:
+        import numpy as np
+        import oracle
+        from rank_error_correction_b200 import synth
+        X = synth.bits(synth.activations(T, D, synth.ALPHA_QKV, seed=seed))
+        X2 = synth.bits(synth.activations(T, D, synth.ALPHA_QKV, seed=seed, sub=1))
+        units = []
+        for name, outs, sub in (("qkv", QKV_OUTS, 0), ("o_proj", O_OUTS, 10)):
+            mods = []
+            As, B = synth.random_factors(outs, D, R_RANK, seed=seed, sub=sub)
+            for j, O in enumerate(outs):
+                W = synth.weights(O, D, seed=seed, stream_sub=sub + j)
+                q, s, z = oracle.quantize_int4(W)
+                del W
+                mods.append((q, s, z, synth.bits(As[j])))
+            units.append((name, mods, synth.bits(B)))
+        _ORACLE_STEP = (X, X2, units)
+    return _ORACLE_STEP
+
+
+def oracle_step(threads):
+    """One whole decode step through the oracle (float64 C): the Q/K/V group
+    with one shared R, then the o_proj solo with its own R.  Returns seconds."""
     import oracle
-    from rank_error_correction_b200 import synth
-    rows_total = sum(QKV_OUTS) + sum(O_OUTS)
-    X = synth.bits(synth.activations(T, D, synth.ALPHA_QKV, seed=seed))
-    mods = []
-    for j, O in enumerate(QKV_OUTS + O_OUTS):
-        W = synth.weights(rows_per_module, D, seed=seed, stream_sub=900 + j)
-        q, s, z = oracle.quantize_int4(W)
-        A = (np.random.default_rng(j).standard_normal((rows_per_module, R_RANK)) * 0.005).astype(np.float16)
-        mods.append((q, s, z, synth.bits(A)))
-    B = synth.bits((np.random.default_rng(99).standard_normal((R_RANK, D)) * 0.01).astype(np.float16))
+    X, X2, units = oracle_step_inputs()
+    oracle.set_threads(threads)
     t0 = time.perf_counter()
-    # QKV: one shared R; o_proj: its own R
-    oracle.group_forward(mods[:3], B, X)
-    q, s, z, A = mods[3]
-    oracle.solo_forward(q, s, z, A, B, X)
-    dt = time.perf_counter() - t0
-    frac = (4 * rows_per_module) / rows_total
-    return dt, frac
+    (_, mods, B), (_, omods, Bo) = units
+    oracle.group_forward(mods, B, X)
+    q, s, z, A = omods[0]
+    oracle.solo_forward(q, s, z, A, Bo, X2)
+    return time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_figures(budget_s=12.0):
+    """The oracle as it stands on this host's cores: whole decode steps with
+    every core (OpenMP over output rows), and with one thread."""
+    ncores = host_cores()
+    oracle_step(ncores)                     # warm: pages, thread pool
+    t_all, t_start = [], time.perf_counter()
+    while time.perf_counter() - t_start < budget_s * 0.5 and len(t_all) < 50:
+        t_all.append(oracle_step(ncores))
+    t_one, t_start = [], time.perf_counter()
+    while time.perf_counter() - t_start < budget_s * 0.5 and len(t_one) < 5:
+        t_one.append(oracle_step(1))
+    import oracle
+    oracle.set_threads(ncores)
+    all_s, one_s = statistics.median(t_all), statistics.median(t_one)
+    return {"value": 1.0 / all_s, "unit": "tok/s", "cores": ncores, "kind": "oracle",
+            "nproc": os.cpu_count(), "threads": ncores,
+            "single_thread_value": 1.0 / one_s, "ms_per_step_all_cores": all_s * 1e3,
+            "ms_per_step_single_thread": one_s * 1e3,
+            "sample": f"the whole decode step (T=1: Q/K/V group 3x4096x4096 with one shared R + o_proj solo "
+                      f"4096x4096, r=64), float64 C oracle; {len(t_all)} steps on {ncores} threads "
+                      f"(median), {len(t_one)} steps on 1 thread (median)"}
+
+
+def decode_config(replicas, world):
+    """The config dict of the decode line (shared by both arms)."""
+    return {"workload": DECODE_WORKLOAD, "tokens": 1, "replicas": replicas,
+            "l2": f"inputs larger than L2: {replicas} weight replicas rotated ({replicas * 38.4:.0f} MB)",
+            "graph": "one CUDA graph of all timed steps (per-call roofline times from a second, "
+                     "event-instrumented replay)",
+            "parallelism": "replicas" if world > 1 else "single GPU"}
 
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm: every step is the whole decode step
+    (nothing sampled or extrapolated), timed on the host's cores."""
     if rank != 0:
         return 0
     T = 1
-    steps, warmup = args.steps, args.warmup
-    # size each step so the whole run stays within a few minutes
-    rows = 256
-    for _ in range(warmup):
-        oracle_sample(T, rows)
-    times = []
-    frac = None
-    for _ in range(steps):
-        dt, frac = oracle_sample(T, rows)
-        times.append(dt)
-    step_s = sum(times) / len(times) / frac          # scaled to the full step
-    value = T / step_s
-    line = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 1, "steps": steps, "warmup": warmup,
-            "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": DECODE_WORKLOAD, "tokens": T,
-                       "sample": f"{rows} rows per module of 16384; scaled by row fraction"},
-            "cpu_baseline": {"value": value, "unit": "tok/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{rows} of 4096 rows per module x 4 modules per step, {steps} steps"},
+    ncores = host_cores()
+    for _ in range(args.warmup):
+        oracle_step(ncores)
+    times = [oracle_step(ncores) for _ in range(args.steps)]
+    total_s = sum(times)
+    value = T * args.steps / total_s
+    line = {"metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_s / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": decode_config(args.replicas, world),
+            "cpu_baseline": {"value": value, "unit": "tok/s", "cores": ncores, "kind": "oracle",
+                             "nproc": os.cpu_count(),
+                             "sample": f"every step is the whole decode step (Q/K/V group + o_proj, T=1), "
+                                       f"{args.steps} timed steps after {args.warmup} warm-up steps, "
+                                       f"float64 C oracle, OpenMP over output rows on {ncores} threads"},
             "e2e": {"value": value, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -716,15 +772,7 @@ def main():
 
     cpu = None
     if rank == 0 and not args.no_cpu:
-        times, frac = [], None
-        t_start = time.perf_counter()
-        while time.perf_counter() - t_start < 10.0 and len(times) < 20:
-            dt, frac = oracle_sample(1, 512)
-            times.append(dt)
-        step_s = statistics.mean(times) / frac
-        cpu = {"value": 1.0 / step_s, "unit": "tok/s", "cores": 1, "kind": "oracle",
-               "sample": f"T=1, 512 of 4096 rows of each of the 4 modules per sample, {len(times)} samples, "
-                         f"scaled by the row fraction ({frac:.4f})"}
+        cpu = cpu_baseline_figures()
 
     if rank == 0:
         # DRAM bytes per launch from the committed ncu captures (profiles/)
@@ -746,13 +794,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16 x int4 -> fp32 acc", "data": "synthetic",
-            "config": {"workload": DECODE_WORKLOAD,
-                       "tokens": T, "replicas": args.replicas,
-                       "l2": f"inputs larger than L2: {args.replicas} weight replicas rotated "
-                             f"({args.replicas * 38.4:.0f} MB)",
-                       "graph": "one CUDA graph of all timed steps (per-call roofline times from a second, "
-                                "event-instrumented replay)",
-                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "config": decode_config(args.replicas, world),
             "roofline": {"bound": "hbm", "kernel": "glowq_group_forward (Q/K/V, T=1): rproj_cluster + corrected_gemv",
                          "achieved": achieved, "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": traffic, "algorithmic_bytes": qkv_bytes,
