@@ -655,13 +655,119 @@ def stack13b_line(device, warmup, ranks=None):
     return out
 
 
+# ------------------------------------------------ per-unit lines (configs)
+
+# LLaMA-3.1-8B-shaped GQA layer: (unit, module output features, input dim)
+L31_UNITS = [("qkv", [4096, 1024, 1024], 4096), ("o_proj", [4096], 4096),
+             ("gate_up", [14336, 14336], 4096), ("down_proj", [4096], 14336)]
+# LLaMA-2-13B-shaped layer units
+S13_UNIT_SHAPES = [("qkv", [5120, 5120, 5120], 5120), ("o_proj", [5120], 5120),
+                   ("gate_up", [13824, 13824], 5120), ("down_proj", [5120], 13824)]
+L2_BYTES = 126 * 1024 * 1024
+
+
+def build_unit(outs, d, seed, sub, device):
+    """One unit (group or solo) of random-init INT4 g128 modules with r = 64 factors."""
+    from rank_error_correction_b200 import glowq, synth
+    mods = []
+    for j, O in enumerate(outs):
+        W = synth.device_weights(O, d, seed, sub=sub + j, device=device)
+        q, s, z = glowq.pack_int4(W)
+        del W
+        mods.append(glowq.QModule(q, s, z))
+    As, B = synth.device_factors(outs, d, R_RANK, seed, sub=sub, device=device)
+    for m, A in zip(mods, As):
+        m.A = A
+    return mods, B
+
+
+def time_unit_chain(reps, X, T, calls, device, ranks=None):
+    """Average duration of one call of a unit in a CUDA graph of `calls`
+    back-to-back calls over the weight replicas `reps` (CUDA events around the
+    graph on the launching stream).  Returns microseconds per call."""
+    import torch
+    from rank_error_correction_b200 import glowq
+    mods0, _ = reps[0]
+    Ys = [torch.empty((T, m.out_features), dtype=torch.float16, device=device) for m in mods0]
+    R = torch.empty((T, R_RANK), dtype=torch.float16, device=device)
+    ws = glowq.alloc_workspace(T, R_RANK, device)
+
+    def call(i):
+        mods, B = reps[i % len(reps)]
+        if len(mods) > 1:
+            glowq.group_forward(mods, B, X, Ys=Ys, R_out=R, workspace=ws)
+        else:
+            glowq.solo_forward(mods[0], B, X, Y=Ys[0], workspace=ws)
+
+    stream = torch.cuda.Stream(device=device)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            call(i)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(calls):
+            call(i)
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    if ranks is not None:
+        ranks.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record()
+        g.replay()
+        t1.record()
+    torch.cuda.synchronize()
+    us = t0.elapsed_time(t1) * 1e3 / calls
+    del g
+    st = glowq.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} after a timed chain (T={T}, {len(mods0)} modules, "
+                           f"d={mods0[0].in_features})")
+    return ranks.max(us) if ranks is not None else us
+
+
+def unit_lines(shapes, tokens, device, hbm_peak, tf_peak, seed=0, sub0=0, ranks=None):
+    """Per-unit throughput of one layer's linears at each token count: decode
+    counts (T <= 64) rotate enough weight replicas that every call streams its
+    weights from HBM (more than 2x L2 per chain); T >= 512 rotate two."""
+    import torch
+    from rank_error_correction_b200 import synth
+    out = {}
+    for k, (name, outs, d) in enumerate(shapes):
+        ubytes = group_bytes(outs, d, R_RANK, 1)
+        n_dec = max(2, min(8, -(-2 * L2_BYTES // ubytes)))
+        reps = [build_unit(outs, d, seed, sub0 + 1000 * i + 10 * k, device) for i in range(n_dec)]
+        for T in tokens:
+            X = synth.device_activations(T, d, seed, sub=700 + k, device=device)
+            calls = 64 if T <= 64 else 6
+            use = reps if T <= 64 else reps[:2]
+            us = time_unit_chain(use, X, T, calls, device, ranks=ranks)
+            b = group_bytes(outs, d, R_RANK, T)
+            f = group_flops(outs, d, R_RANK, T)
+            e = {"us_per_call": us, "GBps": b / (us * 1e-6) / 1e9, "hbm_frac": b / (us * 1e-6) / 1e9 / hbm_peak,
+                 "TFLOPs": f / (us * 1e-6) / 1e12, "tensor_frac": f / (us * 1e-6) / 1e12 / tf_peak,
+                 "algorithmic_bytes": b, "algorithmic_flops": f, "replicas": len(use)}
+            out.setdefault(f"T{T}", {})[name] = e
+            del X
+        del reps
+        torch.cuda.empty_cache()
+    for key, units in out.items():
+        T = int(key[1:])
+        tot = sum(u["us_per_call"] for u in units.values())
+        units["layer"] = {"us": tot, "tok_s": (ranks.world if ranks is not None else 1) * T / (tot * 1e-6)}
+    return out
+
+
 # ------------------------------------------------------------ profile cases
 
 def profile_case(case, device, steps=4):
     """A few untimed steps of one bench workload (no JSON line): the command
     that the ncu summaries under profiles/ are captured from.  Launch order per
-    step -- decode: rproj_cluster, corrected_gemv (Q/K/V group), rproj_cluster,
-    corrected_gemv (o_proj); prefill: rproj_tc, rproj_sum, corrected_gemm
+    step -- decode: corrected_gemv (Q/K/V group), corrected_gemv (o_proj);
+    prefill: rproj_tc, rproj_sum, corrected_gemm
     (gate/up), rproj_tc, rproj_sum, corrected_gemm (down_proj)."""
     import torch
     from rank_error_correction_b200 import glowq
@@ -690,6 +796,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill line")
     ap.add_argument("--no-stack", action="store_true", help="skip the 40-layer LLaMA-2-13B stack line")
+    ap.add_argument("--no-units", action="store_true",
+                    help="skip the per-unit lines (LLaMA-3.1-8B layer, LLaMA-2-13B decode batches)")
     ap.add_argument("--profile-case", choices=["decode", "prefill"],
                     help="run a few untimed steps of one workload and exit (for ncu captures)")
     args = ap.parse_args()
@@ -731,7 +839,7 @@ def main():
     value = ranks.rate(T * args.steps, total_ms)
     qkv_bytes = group_bytes(QKV_OUTS, D, R_RANK, T)
     achieved = qkv_bytes / (qkv_chain_ms * 1e-3) / 1e9
-    launches_per_step = 2 + 2          # (rproj_cluster, corrected_gemv) x 2 calls
+    launches_per_step = 1 + 1          # one corrected_gemv launch per call (R computed inside it)
     e2e_ms, h2d, d2h, _ = time_e2e(T, args.steps, device, res["reps"], res["io"], ranks=ranks)
     e2e_ms = ranks.max(e2e_ms)
 
@@ -770,6 +878,16 @@ def main():
     if not args.no_stack:
         stack = stack13b_line(device, args.warmup, ranks=ranks)
 
+    l31 = s13b = None
+    if not args.no_units:
+        l31 = unit_lines(L31_UNITS, (1, 4096), device, hbm_peak, tf_peak, sub0=20000, ranks=ranks)
+        l31["workload"] = ("LLaMA-3.1-8B-shaped GQA layer: Q/K/V group 4096/1024/1024 x 4096, o_proj 4096x4096, "
+                           "gate/up group 2x14336x4096, down_proj 4096x14336; INT4 g128, r=64; per unit, "
+                           "CUDA graph of back-to-back calls")
+        s13b = unit_lines(S13_UNIT_SHAPES, (16, 32, 64), device, hbm_peak, tf_peak, sub0=40000, ranks=ranks)
+        s13b["workload"] = ("LLaMA-2-13B-shaped layer units at decode batches 16/32/64 (T <= 16: weight-streaming "
+                            "decode kernel; T > 16: tcgen05 kernel); INT4 g128, r=64; per unit")
+
     cpu = None
     if rank == 0 and not args.no_cpu:
         cpu = cpu_baseline_figures()
@@ -795,7 +913,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp16 x int4 -> fp32 acc", "data": "synthetic",
             "config": decode_config(args.replicas, world),
-            "roofline": {"bound": "hbm", "kernel": "glowq_group_forward (Q/K/V, T=1): rproj_cluster + corrected_gemv",
+            "roofline": {"bound": "hbm", "kernel": "glowq_group_forward (Q/K/V, T=1): corrected_gemv with the anchor projection inside",
                          "achieved": achieved, "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s",
                          "frac": achieved / hbm_peak, "traffic": traffic, "algorithmic_bytes": qkv_bytes,
                          "us_per_launch": qkv_chain_ms * 1e3,
@@ -811,6 +929,8 @@ def main():
             "extra": extra,
             "prefill": prefill,
             "stack13b": stack,
+            "llama31_8b_layer": l31,
+            "llama2_13b_units_decode_batches": s13b,
         }
         print(json.dumps(line), flush=True)
     if ranks.dist is not None:

@@ -110,6 +110,57 @@ GLOWQ_API glowq_status glowq_dequant_int4(const uint32_t* qweight, const uint16_
                                 int32_t group_size, uint16_t* W_deq, void* stream);
 
 /*
+ * Base-weight formats (thelatestinai.com GlowQ page, Table 13: GlowQ's
+ * correction applied on top of INT4, MXFP4 and NVFP4 base weights).  The
+ * pages name MXFP4 and NVFP4 without defining them; their public definitions
+ * are used, each a reading:
+ *   E2M1 element (4 bits): sign bit 3, exponent bits 2..1 (bias 1), mantissa
+ *     bit 0; magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.  Encoding: nearest
+ *     magnitude, ties to the even mantissa, saturating at 6; zero and NaN
+ *     encode as 0 (so a tiny negative value gives +0).
+ *   MXFP4: blocks of 32 consecutive k of a row share an E8M0 scale
+ *     X = 2^(floor(log2 amax) - 2) (code clamped to 0..254; 2^-127 for an
+ *     all-zero block); elements E2M1(w / X) in IEEE fp32.
+ *   NVFP4: one fp32 tensor scale s_t = amax_tensor / (6 * 448) (1 for an
+ *     all-zero tensor); blocks of 16 k share an E4M3 scale
+ *     S = E4M3(amax_block / (6 s_t)) (nearest, ties to even, saturating at
+ *     448); elements E2M1(w / (S s_t)), 0 when S s_t == 0.  All scale
+ *     arithmetic in IEEE fp32 without fused multiply-add.
+ *   Packing: codes [O][d/8] uint32, code k of a row in nibble (k % 8) of word
+ *   k / 8 (as for INT4); scales [O][d/32] (MXFP4, E8M0) or [O][d/16]
+ *   (NVFP4, E4M3) bytes, row-major.
+ *   Dequantised weight: w_hat = fp16_RN(exact e2m1 * scale (* s_t)).
+ */
+typedef enum glowq_format {
+    GLOWQ_FMT_INT4 = 0,
+    GLOWQ_FMT_MXFP4 = 1,
+    GLOWQ_FMT_NVFP4 = 2
+} glowq_format;
+
+/*
+ * MXFP4 or NVFP4 quantisation and packing of W (device, O x d fp32, d % 128
+ * == 0).  Outputs (device, caller-allocated): codes [O][d/8] uint32, scales
+ * [O][d/32] (MXFP4) or [O][d/16] (NVFP4) bytes, and for NVFP4 the tensor
+ * scale s_t in tensor_scale[0] (one float; ignored for MXFP4, may be NULL).
+ * Errors: GLOWQ_ERR_ARG (null pointer, negative size, fmt not MXFP4/NVFP4),
+ * GLOWQ_ERR_SHAPE (d % 128), GLOWQ_ERR_ALIGN (W not 16-byte aligned, codes
+ * not 4-byte aligned, tensor_scale not 4-byte aligned).
+ */
+GLOWQ_API glowq_status glowq_pack_fp4(glowq_format fmt, const float* W, int64_t O, int64_t d, uint32_t* codes,
+                                      uint8_t* scales, float* tensor_scale, void* stream);
+
+/*
+ * Dequantise MXFP4 / NVFP4 codes to fp16 (device, O x d): w_hat =
+ * fp16_RN(e2m1 * 2^(e - 127)) or fp16_RN(e2m1 * e4m3 * s_t), the product
+ * formed exactly.  Arguments as for glowq_pack_fp4; tensor_scale is read on
+ * the device (NVFP4 only).  Used to check the packed formats; the forward
+ * kernels never materialise w_hat in HBM.
+ */
+GLOWQ_API glowq_status glowq_dequant_fp4(glowq_format fmt, const uint32_t* codes, const uint8_t* scales,
+                                         const float* tensor_scale, int64_t O, int64_t d, uint16_t* W_deq,
+                                         void* stream);
+
+/*
  * Bytes of device scratch the forward calls need for T tokens at rank r:
  *   - 256 bytes of hand-off flags at offset 0, through which the decode GEMV
  *     (T <= 16) learns, while it already streams weights, that the kernel
@@ -159,6 +210,47 @@ GLOWQ_API glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, 
 GLOWQ_API glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16_t* B,
                                 int32_t r, const uint16_t* X, int64_t T, void* workspace,
                                 size_t workspace_bytes, void* stream);
+
+/*
+ * One MXFP4 / NVFP4 module of a group (formats and packing as for
+ * glowq_pack_fp4).  Device pointers:
+ *   codes         [O][d/8] uint32 E2M1 codes
+ *   scales        [O][d/32] E8M0 (MXFP4, 4-byte aligned) or [O][d/16] E4M3
+ *                 (NVFP4, 8-byte aligned) bytes
+ *   tensor_scale  NVFP4: one float s_t; ignored (may be NULL) for MXFP4
+ *   A, out_features, Y, ldY  as in glowq_module
+ */
+typedef struct glowq_fp4_module {
+    const uint32_t* codes;
+    const uint8_t* scales;
+    const float* tensor_scale;
+    const uint16_t* A;
+    int64_t out_features;
+    uint16_t* Y;
+    int64_t ldY;
+} glowq_fp4_module;
+
+/*
+ * Group and solo forward with MXFP4 / NVFP4 base weights (thelatestinai.com
+ * GlowQ page, Table 13: the group-shared correction on top of these base
+ * datatypes), W4A16: Y_i = X w_hat_i^T + R A_i^T with R = X B^T computed once
+ * per group, as glowq_group_forward / glowq_solo_forward do for INT4 (same
+ * arguments, workspace and errors; all modules of a call share one format).
+ * The kernels form each weight in fp16 from its exact E2M1 value and block
+ * scale (one conversion per pair of codes, one multiply): MXFP4 as
+ * fp16_RN(e2m1 * 2^(e - 127)), block scales outside [2^-24, 2^15] clamped to
+ * that range (below 2^-24: 0); NVFP4 at T <= 16 as the exact e2m1 * e4m3 with
+ * the tensor scale s_t applied to the fp32 sums, at T > 16 (tensor-core path,
+ * where the correction shares the accumulator) as
+ * fp16_RN(e2m1 * fp16_RN(e4m3 * s_t)).
+ */
+GLOWQ_API glowq_status glowq_group_forward_fp4(glowq_format fmt, const glowq_fp4_module* mods, int32_t m, int64_t d,
+                                               const uint16_t* B, int32_t r, const uint16_t* X, int64_t T,
+                                               uint16_t* R_out, void* workspace, size_t workspace_bytes,
+                                               void* stream);
+GLOWQ_API glowq_status glowq_solo_forward_fp4(glowq_format fmt, const glowq_fp4_module* mod, int64_t d,
+                                              const uint16_t* B, int32_t r, const uint16_t* X, int64_t T,
+                                              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Solo module forward that allocates nothing (the GlowQ pages have no

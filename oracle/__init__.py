@@ -368,6 +368,25 @@ def dequant_nvfp4(codes, scales, tensor_scale, d):
     return out
 
 
+def fp4_group_forward(fmt, mods, B_bits, X_bits):
+    """W4A16 group forward with MXFP4 / NVFP4 base weights, float64: R = X B^T
+    once, Y_i = X w_hat_i^T + R A_i^T with w_hat_i the format's dequantised
+    fp16 weight.  fmt: "mx" or "nv"; mods: (codes uint8 [O, d/2], scales,
+    tensor_scale or None, A_bits or None).  Returns ([Y_i], R)."""
+    X = _c(X_bits, np.uint16)
+    d = X.shape[1]
+    R = None if B_bits is None else anchor_project(X, B_bits)
+    Xd = f16_bits_to_f64(X)
+    outs = []
+    for (codes, scales, ts, A) in mods:
+        Wb = dequant_mxfp4(codes, scales, d) if fmt == "mx" else dequant_nvfp4(codes, scales, ts, d)
+        Y = matmul(Xd, f16_bits_to_f64(Wb), tb=True)
+        if A is not None and R is not None:
+            Y = Y + matmul(R, f16_bits_to_f64(A), tb=True)
+        outs.append(Y)
+    return outs, R
+
+
 def quantize_act_e4m3(X_bits):
     """Per-token FP8 E4M3 activations: X (T x d fp16 bits) -> (codes uint8 [T, d], scales fp32 [T])."""
     X = _c(X_bits, np.uint16)

@@ -44,17 +44,17 @@ static int device_sm_count() {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace layout (r > 0): [hand-off flags, 256 B][prefill partials][solo R].
-// The flags are the decode kernels' (R kernel -> GEMV) and sit at offset 0 for
-// every T, so a prefill call sharing the workspace never overwrites them.
+// Workspace layout (r > 0): [hand-off flags, 256 B][R partials][solo R].
+// The flags are the decode GEMV's (producers of R -> consumers) and sit at
+// offset 0 for every T, so a prefill call sharing the workspace never
+// overwrites them.
 static size_t workspace_flag_bytes(int32_t r) { return r > 0 ? 256 : 0; }
 
-// fp32 partial sums of R = X B^T for T > 16 (split along d into up to 8
-// slices when the token tiles alone would not fill the GPU); the decode path
-// reduces its partial sums on chip.
+// fp32 partial sums of R = X B^T split along d: up to 16 slices for T <= 16
+// (decode), up to 8 when the prefill token tiles alone would not fill the GPU.
 static size_t workspace_partial_bytes(int64_t T, int32_t r) {
-    if (r <= 0 || T <= kDecodeMaxTokens) return 0;
-    return align_up(prefill_partial_bytes(T, r), 256);
+    if (r <= 0 || T <= 0) return 0;
+    return align_up(T <= kDecodeMaxTokens ? decode_partial_bytes(T, r) : prefill_partial_bytes(T, r), 256);
 }
 
 static size_t workspace_solo_R_bytes(int64_t T, int32_t r) {
@@ -91,34 +91,55 @@ glowq_status validate_solo_call(const glowq_module* mod, int64_t d, const uint16
     return validate_forward(mod, 1, d, B, r, X, T);
 }
 
-static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
-                                 const uint16_t* X, int64_t T, uint16_t* R, void* workspace, size_t ws_bytes,
-                                 cudaStream_t st) {
+static glowq_status forward_views(const ModuleView* hm, int32_t m, int64_t d, const uint16_t* B, int32_t r,
+                                  const uint16_t* X, int64_t T, uint16_t* R, void* workspace, cudaStream_t st,
+                                  int fmt) {
     if (T == 0) return GLOWQ_OK;
-    ModuleView hm[GLOWQ_MAX_MODULES];
-    bool any_A = false;
-    for (int i = 0; i < m; ++i) {
-        hm[i] = {mods[i].qweight, mods[i].scales, mods[i].zeros, (r > 0) ? mods[i].A : nullptr,
-                 mods[i].Y, mods[i].ldY, mods[i].out_features};
-        any_A = any_A || hm[i].A != nullptr;
-    }
     const bool use_r = r > 0;
-    if (T <= kDecodeMaxTokens) {
-        unsigned int* flags = use_r ? reinterpret_cast<unsigned int*>(workspace) : nullptr;
-        if (use_r) {
-            cudaError_t e = launch_rproj_decode(X, B, (int)T, (int)d, r, R, flags, st);
-            if (e != cudaSuccess) return GLOWQ_ERR_CUDA;
-        }
-        cudaError_t e = launch_gemv_decode(hm, m, (int)d, (int)T, use_r ? r : 0, X, R, flags, device_sm_count(), st);
-        return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
-    }
-    (void)any_A;
-    (void)ws_bytes;
     float* partial = (use_r && workspace_partial_bytes(T, r) > 0)
                          ? reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + workspace_flag_bytes(r))
                          : nullptr;
+    if (T <= kDecodeMaxTokens) {
+        unsigned int* flags = use_r ? reinterpret_cast<unsigned int*>(workspace) : nullptr;
+        cudaError_t e = launch_gemv_decode(hm, m, (int)d, (int)T, use_r ? r : 0, X, use_r ? B : nullptr, R, flags,
+                                           partial, device_sm_count(), st, fmt);
+        return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
+    }
     return prefill_group_forward(hm, m, (int)d, use_r ? B : nullptr, use_r ? r : 0, X, T, R, partial,
-                                 device_sm_count(), st);
+                                 device_sm_count(), st, fmt);
+}
+
+static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
+                                 const uint16_t* X, int64_t T, uint16_t* R, void* workspace, cudaStream_t st) {
+    ModuleView hm[GLOWQ_MAX_MODULES];
+    for (int i = 0; i < m; ++i)
+        hm[i] = {mods[i].qweight, mods[i].scales, mods[i].zeros, nullptr, (r > 0) ? mods[i].A : nullptr,
+                 mods[i].Y, mods[i].ldY, mods[i].out_features};
+    return forward_views(hm, m, d, B, r, X, T, R, workspace, st, GLOWQ_FMT_INT4);
+}
+
+// Validation of MXFP4 / NVFP4 modules and their conversion to module views.
+static glowq_status fp4_views(glowq_format fmt, const glowq_fp4_module* mods, int32_t m, int64_t d,
+                              const uint16_t* B, int32_t r, const uint16_t* X, int64_t T, ModuleView* hm) {
+    if (fmt != GLOWQ_FMT_MXFP4 && fmt != GLOWQ_FMT_NVFP4) return GLOWQ_ERR_ARG;
+    if (!mods || m < 1 || m > GLOWQ_MAX_MODULES) return GLOWQ_ERR_ARG;
+    glowq_module tmp[GLOWQ_MAX_MODULES];
+    for (int i = 0; i < m; ++i) {
+        const glowq_fp4_module& f = mods[i];
+        if (!f.scales || (fmt == GLOWQ_FMT_NVFP4 && !f.tensor_scale)) return GLOWQ_ERR_ARG;
+        const uintptr_t sa = reinterpret_cast<uintptr_t>(f.scales);
+        if ((fmt == GLOWQ_FMT_MXFP4 && (sa & 3u)) || (fmt == GLOWQ_FMT_NVFP4 && (sa & 7u)) ||
+            (f.tensor_scale && (reinterpret_cast<uintptr_t>(f.tensor_scale) & 3u)))
+            return GLOWQ_ERR_ALIGN;
+        // the shared checks of the INT4 path (zeros are not used: any non-null value)
+        tmp[i] = {f.codes, reinterpret_cast<const uint16_t*>(f.scales), f.scales, f.A, f.out_features, f.Y, f.ldY};
+    }
+    glowq_status v = validate_forward(tmp, m, d, B, r, X, T);
+    if (v != GLOWQ_OK) return v;
+    for (int i = 0; i < m; ++i)
+        hm[i] = {mods[i].codes, mods[i].scales, nullptr, fmt == GLOWQ_FMT_NVFP4 ? mods[i].tensor_scale : nullptr,
+                 (r > 0) ? mods[i].A : nullptr, mods[i].Y, mods[i].ldY, mods[i].out_features};
+    return GLOWQ_OK;
 }
 
 }  // namespace glowq
@@ -183,6 +204,35 @@ glowq_status glowq_error_norms(const float* W, const uint32_t* qweight, const ui
                : GLOWQ_ERR_CUDA;
 }
 
+glowq_status glowq_pack_fp4(glowq_format fmt, const float* W, int64_t O, int64_t d, uint32_t* codes,
+                            uint8_t* scales, float* tensor_scale, void* stream) {
+    if (O < 0 || d < 0) return GLOWQ_ERR_ARG;
+    if (fmt != GLOWQ_FMT_MXFP4 && fmt != GLOWQ_FMT_NVFP4) return GLOWQ_ERR_ARG;
+    if (d % GLOWQ_GROUP_SIZE != 0) return GLOWQ_ERR_SHAPE;
+    if (O == 0 || d == 0) return GLOWQ_OK;
+    if (!W || !codes || !scales || (fmt == GLOWQ_FMT_NVFP4 && !tensor_scale)) return GLOWQ_ERR_ARG;
+    if (!aligned16(W) || (reinterpret_cast<uintptr_t>(codes) & 3u) ||
+        (tensor_scale && (reinterpret_cast<uintptr_t>(tensor_scale) & 3u)))
+        return GLOWQ_ERR_ALIGN;
+    return launch_pack_fp4((int)fmt, W, O, d, codes, scales, tensor_scale, (cudaStream_t)stream) == cudaSuccess
+               ? GLOWQ_OK
+               : GLOWQ_ERR_CUDA;
+}
+
+glowq_status glowq_dequant_fp4(glowq_format fmt, const uint32_t* codes, const uint8_t* scales,
+                               const float* tensor_scale, int64_t O, int64_t d, uint16_t* W_deq, void* stream) {
+    if (O < 0 || d < 0) return GLOWQ_ERR_ARG;
+    if (fmt != GLOWQ_FMT_MXFP4 && fmt != GLOWQ_FMT_NVFP4) return GLOWQ_ERR_ARG;
+    if (d % GLOWQ_GROUP_SIZE != 0) return GLOWQ_ERR_SHAPE;
+    if (O == 0 || d == 0) return GLOWQ_OK;
+    if (!codes || !scales || !W_deq || (fmt == GLOWQ_FMT_NVFP4 && !tensor_scale)) return GLOWQ_ERR_ARG;
+    if (!aligned16(W_deq) || (reinterpret_cast<uintptr_t>(codes) & 3u)) return GLOWQ_ERR_ALIGN;
+    return launch_dequant_fp4((int)fmt, codes, scales, tensor_scale, O, d, W_deq, (cudaStream_t)stream) ==
+                   cudaSuccess
+               ? GLOWQ_OK
+               : GLOWQ_ERR_CUDA;
+}
+
 size_t glowq_workspace_bytes(int64_t T, int32_t r) {
     if (T <= 0 || r <= 0) return 0;
     return workspace_flag_bytes(r) + workspace_partial_bytes(T, r) + workspace_solo_R_bytes(T, r);
@@ -201,7 +251,8 @@ glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d,
         if (!workspace || workspace_bytes < need) return GLOWQ_ERR_ARG;
         if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
     }
-    return forward_impl(mods, m, d, B, r, X, T, R_out, workspace, workspace_bytes, (cudaStream_t)stream);
+    (void)workspace_bytes;
+    return forward_impl(mods, m, d, B, r, X, T, R_out, workspace, (cudaStream_t)stream);
 }
 
 glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r, const uint16_t* X,
@@ -217,7 +268,43 @@ glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16
         R = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(workspace) + workspace_flag_bytes(r) +
                                         workspace_partial_bytes(T, r));
     }
-    return forward_impl(mod, 1, d, B, r, X, T, R, workspace, workspace_bytes, (cudaStream_t)stream);
+    (void)workspace_bytes;
+    return forward_impl(mod, 1, d, B, r, X, T, R, workspace, (cudaStream_t)stream);
+}
+
+glowq_status glowq_group_forward_fp4(glowq_format fmt, const glowq_fp4_module* mods, int32_t m, int64_t d,
+                                     const uint16_t* B, int32_t r, const uint16_t* X, int64_t T, uint16_t* R_out,
+                                     void* workspace, size_t workspace_bytes, void* stream) {
+    ModuleView hm[GLOWQ_MAX_MODULES];
+    glowq_status v = fp4_views(fmt, mods, m, d, B, r, X, T, hm);
+    if (v != GLOWQ_OK) return v;
+    if (T == 0) return GLOWQ_OK;
+    if (r > 0) {
+        if (!R_out) return GLOWQ_ERR_ARG;
+        if (!aligned16(R_out)) return GLOWQ_ERR_ALIGN;
+        const size_t need = workspace_flag_bytes(r) + workspace_partial_bytes(T, r);
+        if (!workspace || workspace_bytes < need) return GLOWQ_ERR_ARG;
+        if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
+    }
+    return forward_views(hm, m, d, B, r, X, T, R_out, workspace, (cudaStream_t)stream, (int)fmt);
+}
+
+glowq_status glowq_solo_forward_fp4(glowq_format fmt, const glowq_fp4_module* mod, int64_t d, const uint16_t* B,
+                                    int32_t r, const uint16_t* X, int64_t T, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+    ModuleView hm[1];
+    glowq_status v = fp4_views(fmt, mod, 1, d, B, r, X, T, hm);
+    if (v != GLOWQ_OK) return v;
+    if (T == 0) return GLOWQ_OK;
+    uint16_t* R = nullptr;
+    if (r > 0) {
+        const size_t need = glowq_workspace_bytes(T, r);
+        if (!workspace || workspace_bytes < need) return GLOWQ_ERR_ARG;
+        if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
+        R = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(workspace) + workspace_flag_bytes(r) +
+                                        workspace_partial_bytes(T, r));
+    }
+    return forward_views(hm, 1, d, B, r, X, T, R, workspace, (cudaStream_t)stream, (int)fmt);
 }
 
 glowq_status glowq_selftest_wait_timeout(uint32_t polls, void* stream) {

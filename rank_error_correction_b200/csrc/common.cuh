@@ -51,6 +51,11 @@ __device__ __forceinline__ uint4 ldcg_128(const void* p) {
                  : "memory");
     return v;
 }
+__device__ __forceinline__ float ldcg_f32(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p) : "memory");
+    return v;
+}
 __device__ __forceinline__ uint2 ldcg_64(const void* p) {
     uint2 v;
     asm volatile("ld.global.cg.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");

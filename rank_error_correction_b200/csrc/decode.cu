@@ -6,18 +6,18 @@
 //
 // At T <= 16 the layer is a weight-streaming GEMV: every INT4 weight byte is
 // read once from HBM and meets at most 16 tokens, so the kernels are HBM-bound.
-// One call is two launches chained with programmatic dependent launch:
-//   * rproj_cluster: R = X B^T by one cluster of 8 CTAs splitting d; the
-//     partial sums meet on chip in a fixed order (deterministic), R is rounded
-//     to fp16 once and written to the caller's R buffer.  It lets the GEMV
-//     launch once X is final and tells it through workspace flags when X is
-//     final and when R is stored.
-//   * corrected_gemv: one launch over the stacked rows of all modules of the
-//     group.  Each warp streams its 16 rows of packed weights with 2-D TMA
-//     boxes into a private ring of mbarrier-tracked stages; the stream and the
-//     main loop run while the projection is still being computed (R is needed
-//     only by the epilogue, and a control warp per CTA collects it into shared
-//     memory meanwhile).  Nibbles become exact fp16 values
+// One call is one launch, corrected_gemv, over the stacked rows of all modules
+// of the group, launched with programmatic dependent launch:
+//   * the anchor projection R = X B^T is computed inside the same launch: the
+//     control warps of the first CTAs compute fp32 partial sums over slices of
+//     d, the last producer of each 16-row block of B adds them in a fixed
+//     order (deterministic), rounds R to fp16 once and writes the caller's R
+//     buffer; every CTA collects R into shared memory for its epilogue.  R is
+//     needed only there, so the projection runs beside the main loop;
+//   * each warp streams its 16 rows of packed weights with 2-D TMA boxes into
+//     a private ring of mbarrier-tracked stages, issued before the wait on the
+//     preceding grid (weights are static), so the stream starts while the
+//     previous kernel in the stream finishes.  Nibbles become exact fp16 values
 //     (16 + q/64 for even k, 64 + q for odd k) with one LOP3 per pair; the
 //     multiply-accumulate runs on the tensor cores with register operands
 //     (mma.sync m16n8k16, fp32 accumulate, one chain per parity) and each
@@ -42,199 +42,6 @@
 namespace glowq {
 
 
-
-// ---------------------------------------------------------------------------
-// R = X B^T for T <= 16 in one launch.  A cluster of kRcCtas CTAs splits d
-// (CTA c takes the c-th slice of the 32-wide k steps).  Inside a CTA the work
-// items (B row block of 16 rows, k-lane) are spread over the warps; a k-lane
-// takes every kl-th k step of the slice, two steps' loads in flight.  Partial
-// sums meet in a fixed order: k-lanes in shared memory, then the CTAs of the
-// cluster through distributed shared memory (ascending rank), so R does not
-// depend on timing.  R is rounded to fp16 once.
-// The CTA is small enough to be resident next to a GEMV CTA, so it starts
-// while the preceding GEMV still runs: B is static, so its slice is copied
-// into shared memory (or, when it does not fit, pulled into L2) before the
-// wait on the preceding kernel; after the wait only X is read from memory.
-//
-// Hand-off to the GEMV that follows (flags = three zeroed words):
-//   flags[0]  each CTA adds 1 once its wait has returned (X is final), and only
-//             then allows the GEMV to launch, so the GEMV streams weights and
-//             runs its main loop while R is still being computed;
-//   flags[1]  each CTA adds 1 after its part of R is stored; the GEMV reads R
-//             in its epilogue only after seeing kRcCtas here;
-//   flags[2]  counts GEMV CTAs past both waits; the last one zeroes all three.
-// A GEMV launched without the programmatic attribute starts after this kernel
-// has completed and finds both counts already reached.
-// ---------------------------------------------------------------------------
-constexpr int kRcCtas = 8;
-constexpr int kRcWarps = 8;
-constexpr int kRcStageB = 72 * 1024;         // largest B slice staged in shared memory
-
-__host__ __device__ inline int rc_row_blocks(int r) { return (r + 15) / 16; }
-__host__ __device__ inline int rc_klanes(int r) {
-    const int kl = kRcWarps / rc_row_blocks(r);
-    return kl > 0 ? kl : 1;
-}
-// B slice of one CTA: r rows x (steps of 32 k), row pitch padded by 16 B
-__host__ __device__ inline int rc_b_pitch(int d) {
-    const int nsteps = d / 32;
-    return ((nsteps + kRcCtas - 1) / kRcCtas) * 64 + 16;
-}
-__host__ __device__ inline bool rc_stage_b(int r, int d) { return r * rc_b_pitch(d) <= kRcStageB; }
-// shared memory: per-k-lane partials [kl][8*NT][r] + the CTA partial [8*NT][r]
-// (fp32), the CTA's X slice [T][slice] (fp16), then the staged B slice and its
-// mbarrier
-__host__ __device__ inline int rc_part_bytes(int r, int nt) { return (rc_klanes(r) + 1) * 8 * nt * r * 4; }
-__host__ __device__ inline int rc_x_bytes(int d, int nt) { return 8 * nt * (rc_b_pitch(d) - 16); }
-// the X slice is staged when it fits in 32 KB (wider inputs read X in the loop)
-__host__ __device__ inline bool rc_stage_x(int d, int nt) { return rc_x_bytes(d, nt) <= 32 * 1024; }
-__host__ __device__ inline int rc_smem_bytes(int r, int d, int nt) {
-    const int p = (rc_part_bytes(r, nt) + 15) / 16 * 16 + (rc_stage_x(d, nt) ? rc_x_bytes(d, nt) : 0);
-    return rc_stage_b(r, d) ? p + r * rc_b_pitch(d) + 16 : p;
-}
-
-template <int NT>
-__global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32, 4)
-    rproj_cluster_kernel(const __half* __restrict__ X, const __half* __restrict__ B, int T, int d, int r,
-                         __half* __restrict__ R, unsigned int* flags, unsigned int* status) {
-    extern __shared__ __align__(16) float rc_smem[];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int nrb = rc_row_blocks(r), kl = rc_klanes(r);
-    const int TP = 8 * NT;                       // padded token count
-    float* part = rc_smem;                       // [kl][TP][r]
-    float* cpart = rc_smem + kl * TP * r;        // [TP][r]
-    uint32_t crank;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
-    const int nsteps = d / 32;
-    const int s0 = (int)((int64_t)crank * nsteps / kRcCtas), s1 = (int)((int64_t)(crank + 1) * nsteps / kRcCtas);
-    const bool staged = rc_stage_b(r, d);
-    const int pitch = rc_b_pitch(d);
-    const bool staged_x = rc_stage_x(d, NT);
-    unsigned char* xsl = reinterpret_cast<unsigned char*>(rc_smem) + (rc_part_bytes(r, NT) + 15) / 16 * 16;
-    const int xpitch = pitch - 16;               // bytes of one token's slice
-    unsigned char* bs = xsl + (staged_x ? rc_x_bytes(d, NT) : 0);
-    uint64_t* bbar = reinterpret_cast<uint64_t*>(bs + r * pitch);
-    // B is static: stage (or prefetch) this CTA's slice before the wait
-    if (staged) {
-        if (threadIdx.x == 0) {
-            mbar_init(bbar, 1);
-            fence_mbar_init();
-            mbar_arrive_expect_tx(bbar, (uint32_t)(r * (s1 - s0) * 64));
-        }
-        __syncthreads();
-        for (int j = threadIdx.x; j < r; j += blockDim.x)
-            bulk_g2s(smem_u32(bs + j * pitch), B + (int64_t)j * d + s0 * 32, (uint32_t)((s1 - s0) * 64), bbar);
-    } else {
-        for (int j = threadIdx.x; j < r; j += blockDim.x)
-            asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;"
-                         ::"l"(B + (int64_t)j * d + s0 * 32), "r"((uint32_t)((s1 - s0) * 64))
-                         : "memory");
-    }
-    pdl_wait();                 // X may come from the previous kernel in the stream
-    if (flags && threadIdx.x == 0) flag_release_add(flags + 0, 1u);
-    pdl_launch_dependents();    // the GEMV may start streaming weights now
-    // the CTA's slice of X in one round trip (16-byte chunks), padding tokens 0
-    if (staged_x) {
-        const int chunks = xpitch / 16, n = TP * chunks;
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            const int tok = i / chunks, c = i - tok * chunks;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (tok < T && s0 * 32 + c * 8 < s1 * 32) v = ldcg_128(X + (int64_t)tok * d + s0 * 32 + c * 8);
-            *reinterpret_cast<uint4*>(xsl + tok * xpitch + c * 16) = v;
-        }
-    }
-    if (staged) mbar_wait(bbar, 0, status);
-    __syncthreads();
-    const uint4 zero4 = make_uint4(0, 0, 0, 0);
-    for (int item = warp; item < nrb * kl; item += kRcWarps) {
-        const int rb = item % nrb, kq = item / nrb;
-        const int j0 = rb * 16 + g, j1 = j0 + 8;
-        float acc[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
-        constexpr int U = 2;   // k steps per iteration, all loads issued before the MMAs
-        for (int st = s0 + kq; st < s1; st += U * kl) {
-            uint4 blo[U], bhi[U], xv[U][NT];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int su = st + u * kl;
-                const bool in = su < s1;
-                const int k = su * 32 + 8 * t;
-                if (staged) {
-                    const int off = (su - s0) * 64 + 16 * t;
-                    blo[u] = (in && j0 < r) ? *reinterpret_cast<const uint4*>(bs + j0 * pitch + off) : zero4;
-                    bhi[u] = (in && j1 < r) ? *reinterpret_cast<const uint4*>(bs + j1 * pitch + off) : zero4;
-                } else {
-                    blo[u] = (in && j0 < r) ? ldg_128(B + (int64_t)j0 * d + k) : zero4;
-                    bhi[u] = (in && j1 < r) ? ldg_128(B + (int64_t)j1 * d + k) : zero4;
-                }
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const int tok = n * 8 + g;
-                    if (staged_x)
-                        xv[u][n] = in ? *reinterpret_cast<const uint4*>(xsl + tok * xpitch + (su - s0) * 64 + 16 * t)
-                                      : zero4;
-                    else
-                        xv[u][n] = (in && tok < T) ? ldcg_128(X + (int64_t)tok * d + k) : zero4;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const uint32_t a0[4] = {blo[u].x, bhi[u].x, blo[u].y, bhi[u].y};
-                const uint32_t a1[4] = {blo[u].z, bhi[u].z, blo[u].w, bhi[u].w};
-#pragma unroll
-                for (int n = 0; n < NT; ++n) {
-                    const uint32_t b0[2] = {xv[u][n].x, xv[u][n].y};
-                    const uint32_t b1[2] = {xv[u][n].z, xv[u][n].w};
-                    mma_16816(acc[n], a0, b0);
-                    mma_16816(acc[n], a1, b1);
-                }
-            }
-        }
-        float* my = part + kq * TP * r;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) {
-            const int tk = n * 8 + 2 * t;
-            if (j0 < r) {
-                my[tk * r + j0] = acc[n][0];
-                my[(tk + 1) * r + j0] = acc[n][1];
-            }
-            if (j1 < r) {
-                my[tk * r + j1] = acc[n][2];
-                my[(tk + 1) * r + j1] = acc[n][3];
-            }
-        }
-    }
-    __syncthreads();
-    // this CTA's partial: k-lanes in ascending order
-    for (int i = threadIdx.x; i < T * r; i += blockDim.x) {
-        float v = part[i];
-        for (int q = 1; q < kl; ++q) v += part[q * TP * r + i];
-        cpart[i] = v;
-    }
-    // all CTAs' partials are complete and visible in the cluster
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    const uint32_t cbase = (uint32_t)__cvta_generic_to_shared(cpart);
-    for (int i = (int)crank * blockDim.x + threadIdx.x; i < T * r; i += kRcCtas * blockDim.x) {
-        float v = 0.f;
-#pragma unroll
-        for (int c = 0; c < kRcCtas; ++c) {
-            uint32_t ra;
-            asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(cbase + 4u * (uint32_t)i), "r"(c));
-            float pv;
-            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(pv) : "r"(ra) : "memory");
-            v = (c == 0) ? pv : v + pv;
-        }
-        R[i] = __float2half_rn(v);
-    }
-    // no CTA leaves while another may still read its shared memory
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-    // this CTA's stores of R (ordered before thread 0 by the barrier) are published
-    if (flags && threadIdx.x == 0) flag_release_add(flags + 1, 1u);
-}
 
 // ---------------------------------------------------------------------------
 // Corrected GEMV over the stacked rows of a group.
@@ -272,23 +79,33 @@ __global__ void __cluster_dims__(kRcCtas, 1, 1) __launch_bounds__(kRcWarps * 32,
 //   rs   [8*NT][r+8] f16             R of the call (rows of padding tokens zero)
 //   rbar u64                         completes when rs holds R
 //
-// Besides its rt * kw compute warps a CTA has one control warp.  It waits until
-// X is final (the R kernel's flags[0], or the preceding grid), then, while the
-// compute warps run the main loop, until R is stored (flags[1]); it copies R
-// into shared memory for the epilogue and, as the last CTA to get there,
-// returns the flags to zero.  The hand-off latency thus stays off the weight
-// stream and out of the epilogue.
+// Besides its rt * kw compute warps a CTA has one control warp.  While the
+// compute warps run the main loop it computes this CTA's items of the anchor
+// projection (see rproj_item), waits until every 16-row block of R is stored,
+// copies R into shared memory for the epilogue and, as the last CTA to get
+// there, returns the hand-off flags to zero.
+//
+// Hand-off flags (workspace words; zero when a call starts, zero when it ends):
+//   [0, 16)   arrivals of the d-slice producers of each 16-row block of B
+//   16        16-row blocks of R stored
+//   17        CTAs that have copied R (the last one zeroes the flags; the next
+//             call reads them only after this grid has completed)
 // ---------------------------------------------------------------------------
-constexpr int kMaxWarps = 11;   // compute warps; with the control warp 12 x 32 x 128 registers
-                                // leave room for an R CTA on the SM
+constexpr int kMaxWarps = 15;   // compute warps; with the control warp 16 x 32 x 128 registers
+constexpr int kFlagReady = 16;
+constexpr int kFlagDone = 17;
+constexpr int kRMaxSlices = 16;  // d-slices of the anchor projection (fp32 partials in the workspace)
+constexpr int kBSliceGroups = 4;                        // 128-groups of B staged per projection item
+constexpr int kBSlicePitch = kBSliceGroups * 256 + 16;  // bytes per staged row of B (padded: no bank conflicts)
 // Pipeline stages per warp (one 2-D TMA box of 16 rows x 2 groups of 128,
 // 2 KB) are a template parameter S in {4, 8}: the host trades ring depth
 // against resident warps.
 
 struct GemvModule {
     const uint32_t* q;
-    const __half* s;
-    const uint8_t* z;
+    const void* s;     // INT4: fp16 scales [O][d/128]; MXFP4 / NVFP4: scale bytes [O][d/32] / [O][d/16]
+    const uint8_t* z;  // INT4 zeros [O][d/128]
+    const float* ts;   // NVFP4 tensor scale (device, one float)
     const __half* A;   // nullptr: correction off for this module
     __half* Y;
     int64_t ldY;
@@ -308,14 +125,18 @@ struct GemvArgs {
     int kw;            // in-CTA splits of d
     int kc;            // CTAs per cluster splitting d (kw == 1 when kc > 1)
     const __half* X;   // T x d
-    const __half* R;   // T x r (read after the wait)
-    unsigned int* flags;    // hand-off words of the R kernel (nullptr: wait for the preceding grid)
-    int nflag;              // count each flag reaches (CTAs of the R kernel)
+    const __half* B;   // r x d shared right factor (r > 0)
+    __half* R;         // T x r: the anchor projection, written by this launch
+    float* part;       // [kc * rsub][T][r] fp32 partial sums of R
+    int rsub;          // sub-slices of each cluster rank's slice of d (kc * rsub <= kRMaxSlices)
+    int rpre;          // 1: R was computed by the preceding launch (rproj_decode_kernel)
+    int stages;        // weight-ring stages per warp (4 or 8)
+    unsigned int* flags;    // hand-off words (r > 0), see above
     unsigned int* status;   // device status word (bounded-wait timeouts)
 };
 
 struct GemvLayout {    // byte offsets into dynamic shared memory
-    int xs, xsum, sz, red, as, rs, rbar, total;
+    int xs, xsum, sz, red, as, rs, rbar, bsl, total;
     int wpt_max, ncta_max, nsub_max, fin_slots;
 };
 
@@ -327,7 +148,9 @@ struct GemvPlan {
 
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
-__host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, int kw, int kc, int nt, int stages) {
+// bstage: reserve the shared-memory copy of the B rows of a projection item
+__host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, int kw, int kc, int nt, int stages,
+                                                  bool bstage = true) {
     GemvLayout L;
     const int warps = rt * kw;
     const int ngroups = d / 128;
@@ -340,7 +163,7 @@ __host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, i
     off += warps * stages * 8;                // mbarriers
     off = (off + 15) / 16 * 16;
     L.xs = off;
-    off += (T + 1) * L.wpt_max * 16;
+    off += (T + 1) * (L.wpt_max + 4) * 16;
     L.xsum = off;
     off += L.ncta_max * 2 * 8 * nt * 4;
     off = (off + 15) / 16 * 16;
@@ -355,7 +178,9 @@ __host__ __device__ inline GemvLayout gemv_layout(int T, int d, int r, int rt, i
     off += (r > 0) ? 8 * nt * (r + 8) * 2 : 0;
     off = (off + 15) / 16 * 16;
     L.rbar = off;
-    off += 16;
+    off += 16;             // rbar, then the staging barrier of the B slice
+    L.bsl = off;
+    off += (r > 0 && bstage) ? 16 * kBSlicePitch : 0;
     L.total = off;
     return L;
 }
@@ -389,7 +214,291 @@ __device__ __forceinline__ void unpack_even_odd(uint32_t w, uint32_t ev[2], uint
     od[1] = (w8 & 0x00F000F0u) | 0x54005400u;
 }
 
-template <int NT, int S, bool ONE>
+// Items of the anchor projection.  Cluster rank c's slice of d (the groups
+// whose activations the CTA has staged) is cut into Sc sub-slices; an item is
+// one 16-row block rb of B times one sub-slice sc, and its fp32 partial sums
+// go to part[c * Sc + sc][t][j] (S = kc * Sc partials per element).  The
+// clusters take the (rb, sc) pairs of their rank round-robin.
+struct RItem { int rb, sc, g0, g1, s; };
+__device__ __forceinline__ RItem ritem(int p, int nrb, int Sc, int crank, int C0, int C1) {
+    RItem it;
+    it.rb = p % nrb;
+    it.sc = p / nrb;
+    it.g0 = C0 + it.sc * (C1 - C0) / Sc;
+    it.g1 = C0 + (it.sc + 1) * (C1 - C0) / Sc;
+    it.s = crank * Sc + it.sc;
+    return it;
+}
+
+// One item, by one warp: R[t][j] partial = sum over the item's k of X[t][k] B[j][k]
+// for the 16 rows j of block rb.  Activations come from the CTA's staged slice
+// xs (pairs (x0,x4) (x2,x6) (x1,x5) (x3,x7) of each 8-element word, word
+// 4t + w of a group at 4w + t, as for the GEMV); B comes from `brow` (row j at brow + (j - 16 rb) * pitch, the item's
+// first k at offset 0: the staged copy in shared memory or B itself), its
+// halves paired the same way, so both MMA operands see one k order.
+// PAIRED: the INT4 kernels stage each 8-element activation word as the pairs
+// (x0,x4) (x2,x6) (x1,x5) (x3,x7); the MXFP4 / NVFP4 kernels keep k order.
+template <int NT, bool PAIRED>
+__device__ __forceinline__ void rproj_item(const GemvArgs& a, const RItem& it, const unsigned char* brow, int64_t pitch,
+                                           const uint4* xs, int xpitch, int C0, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    const int T = a.T, r = a.r;
+    const int j0 = it.rb * 16 + g, j1 = j0 + 8;
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    const unsigned char* b0p = brow + (int64_t)g * pitch + t * 64;
+    const unsigned char* b1p = b0p + 8 * pitch;
+    const uint4* xrow[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int tok = (n * 8 + g < T) ? n * 8 + g : T;   // padding tokens read the zero row
+        xrow[n] = xs + tok * xpitch + (it.g0 - C0) * 16 + t;
+    }
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+    for (int gi = 0; gi < it.g1 - it.g0; ++gi) {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const uint4 bl = (j0 < r) ? *reinterpret_cast<const uint4*>(b0p + gi * 256 + w * 16) : z4;
+            const uint4 bh = (j1 < r) ? *reinterpret_cast<const uint4*>(b1p + gi * 256 + w * 16) : z4;
+            uint32_t ae[4], ao[4];
+            if constexpr (PAIRED) {
+                ae[0] = pair_lo(bl.x, bl.z); ae[1] = pair_lo(bh.x, bh.z); ae[2] = pair_lo(bl.y, bl.w); ae[3] = pair_lo(bh.y, bh.w);
+                ao[0] = pair_hi(bl.x, bl.z); ao[1] = pair_hi(bh.x, bh.z); ao[2] = pair_hi(bl.y, bl.w); ao[3] = pair_hi(bh.y, bh.w);
+            } else {
+                ae[0] = bl.x; ae[1] = bh.x; ae[2] = bl.y; ae[3] = bh.y;
+                ao[0] = bl.z; ao[1] = bh.z; ao[2] = bl.w; ao[3] = bh.w;
+            }
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const uint4 x = xrow[n][gi * 16 + w * 4];
+                const uint32_t xe[2] = {x.x, x.y};
+                const uint32_t xo[2] = {x.z, x.w};
+                mma_16816(acc[n], ae, xe);
+                mma_16816(acc[n], ao, xo);
+            }
+        }
+    }
+    float* P = a.part + (int64_t)it.s * T * r;   // [T][r]
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int tk = n * 8 + 2 * t;
+        if (tk < T) {
+            if (j0 < r) P[tk * r + j0] = acc[n][0];
+            if (j1 < r) P[tk * r + j1] = acc[n][2];
+        }
+        if (tk + 1 < T) {
+            if (j0 < r) P[(tk + 1) * r + j0] = acc[n][1];
+            if (j1 < r) P[(tk + 1) * r + j1] = acc[n][3];
+        }
+    }
+}
+
+// The last producer of block rb: R[t][rb*16 + c] = fp16(sum over s ascending of
+// part[s][t][rb*16 + c]), written to the caller's R.  A lane takes 4 adjacent
+// columns of a token (r % 8 == 0) and issues every slice's load before adding.
+__device__ __forceinline__ void rproj_reduce(const GemvArgs& a, int rb, int S, int lane) {
+    const int T = a.T, r = a.r;
+    const int quads = ((r - rb * 16 < 16) ? r - rb * 16 : 16) / 4;
+    const int64_t stride = (int64_t)T * r;
+    for (int o = lane; o < T * 4; o += 32) {
+        const int tok = o >> 2, qd = o & 3;
+        if (qd >= quads) continue;
+        const float* pp = a.part + (int64_t)tok * r + rb * 16 + qd * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int s0 = 0; s0 < S; s0 += 8) {
+            float4 p8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (s0 + u < S) p8[u] = __ldcg(reinterpret_cast<const float4*>(pp + (s0 + u) * stride));
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (s0 + u < S) {
+                    if (s0 + u == 0) {
+                        v = p8[u];
+                    } else {
+                        v.x += p8[u].x; v.y += p8[u].y; v.z += p8[u].z; v.w += p8[u].w;
+                    }
+                }
+        }
+        __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
+        uint2 pk;
+        pk.x = h2_as_u32(h01);
+        pk.y = h2_as_u32(h23);
+        *reinterpret_cast<uint2*>(a.R + (int64_t)tok * r + rb * 16 + qd * 4) = pk;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Stand-alone anchor projection for GEMV shapes that do not fit in one wave
+// (a CTA of the GEMV must never wait on a producer that is not resident).
+// CTA i computes item (rb = i % nrb, slice s = i / nrb) of R = X B^T over
+// d-slice s: its four warps take a quarter of the slice's groups each, their
+// fp32 sums meet in shared memory in warp order, and the item's partial goes
+// to part[s][t][j]; the last of the S items of a block adds them in ascending
+// s, stores the block of R in fp16 and returns its arrival count to zero.
+// The GEMV launched after it reads R once this grid has completed.
+// ---------------------------------------------------------------------------
+constexpr int kRpWarps = 4;
+
+template <int NT>
+__global__ void __launch_bounds__(kRpWarps * 32) rproj_decode_kernel(const __grid_constant__ GemvArgs args, int S) {
+    __shared__ float red[kRpWarps][NT][4][32];
+    pdl_launch_dependents();    // the GEMV may start streaming its weights
+    pdl_wait();                 // X may come from the preceding kernel
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int d = args.d, T = args.T, r = args.r;
+    const int nrb = (r + 15) / 16, ng = d / 128;
+    const int rb = blockIdx.x % nrb, sl = blockIdx.x / nrb;
+    const int g0 = sl * ng / S, g1 = (sl + 1) * ng / S;
+    const int w0 = g0 + warp * (g1 - g0) / kRpWarps, w1 = g0 + (warp + 1) * (g1 - g0) / kRpWarps;
+    const int j0 = rb * 16 + g, j1 = j0 + 8;
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    const __half* b0p = args.B + (int64_t)(j0 < r ? j0 : 0) * d + 8 * t;
+    const __half* b1p = args.B + (int64_t)(j1 < r ? j1 : 0) * d + 8 * t;
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
+    for (int gg = w0; gg < w1; ++gg) {   // one 128-group: 4 steps of 32 k, loads first
+        uint4 bl[4], bh[4], xv[4][NT];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int kk = gg * 128 + 32 * u;
+            bl[u] = (j0 < r) ? ldg_128(b0p + kk) : z4;
+            bh[u] = (j1 < r) ? ldg_128(b1p + kk) : z4;
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const int tok = n * 8 + g;
+                xv[u][n] = (tok < T) ? ldcg_128(args.X + (int64_t)tok * d + kk + 8 * t) : z4;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint32_t a0[4] = {bl[u].x, bh[u].x, bl[u].y, bh[u].y};
+            const uint32_t a1[4] = {bl[u].z, bh[u].z, bl[u].w, bh[u].w};
+#pragma unroll
+            for (int n = 0; n < NT; ++n) {
+                const uint32_t x0[2] = {xv[u][n].x, xv[u][n].y};
+                const uint32_t x1[2] = {xv[u][n].z, xv[u][n].w};
+                mma_16816(acc[n], a0, x0);
+                mma_16816(acc[n], a1, x1);
+            }
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) red[warp][n][i][lane] = acc[n][i];
+    __syncthreads();
+    if (warp == 0) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float v = red[0][n][i][lane];
+                for (int w = 1; w < kRpWarps; ++w) v += red[w][n][i][lane];
+                acc[n][i] = v;
+            }
+        float* P = args.part + (int64_t)sl * T * r;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int tk = n * 8 + 2 * t;
+            if (tk < T) {
+                if (j0 < r) P[tk * r + j0] = acc[n][0];
+                if (j1 < r) P[tk * r + j1] = acc[n][2];
+            }
+            if (tk + 1 < T) {
+                if (j0 < r) P[(tk + 1) * r + j0] = acc[n][1];
+                if (j1 < r) P[(tk + 1) * r + j1] = acc[n][3];
+            }
+        }
+        __syncwarp();
+        unsigned int prev = 0;
+        if (lane == 0)
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(args.flags + rb) : "memory");
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev == (unsigned)S - 1) {
+            __syncwarp();
+            rproj_reduce(args, rb, S, lane);
+            if (lane == 0) args.flags[rb] = 0u;   // every producer of this block has arrived
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Base-weight formats.  INT4 (the default) is described above.  MXFP4 and
+// NVFP4 codes are E2M1 (thelatestinai.com GlowQ page, Table 13): each byte of
+// a packed word (codes 2j, 2j+1) becomes an fp16 pair of exact E2M1 values in
+// one conversion and is multiplied by its block scale in fp16 (HMUL2): the
+// MXFP4 scale 2^(e - 127) makes the product fp16_RN of the exact weight
+// (scales outside fp16's range are clamped to [2^-24, 2^15], below 2^-24 to
+// 0), the NVFP4 E4M3 scale makes it exact and the fp32 tensor scale s_t is
+// applied to the fp32 sums.  With the scale inside the operand one MMA chain
+// per group accumulates straight into the output sums.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e8m0_to_f16_bits(uint32_t e) {
+    if (e >= 113u && e <= 142u) return (e - 112u) << 10;   // normal fp16 2^(e - 127)
+    if (e > 142u) return 0x7800u;                         // clamped to 2^15
+    if (e >= 103u) return 1u << (e - 103u);               // fp16 subnormal
+    return 0u;                                            // below 2^-24
+}
+
+// Scale data of one (row, 128-group), loaded in the prologue.
+template <int FMT>
+__device__ __forceinline__ void load_group_scales(const void* s, const uint8_t* z, int64_t idx, unsigned short& sv,
+                                                  unsigned char& zv, uint2& fv) {
+    if constexpr (FMT == GLOWQ_FMT_INT4) {
+        sv = __half_as_ushort(static_cast<const __half*>(s)[idx]);
+        zv = z[idx];
+    } else if constexpr (FMT == GLOWQ_FMT_MXFP4) {
+        fv.x = static_cast<const uint32_t*>(s)[idx];   // the group's 4 E8M0 bytes
+    } else {
+        fv = static_cast<const uint2*>(s)[idx];        // the group's 8 E4M3 bytes
+    }
+}
+
+// The 8-byte shared-memory slot of one (row, group): INT4 (s, 64 + z) as
+// fp32; MXFP4 the four block scales as fp16; NVFP4 the eight E4M3 bytes.
+template <int FMT>
+__device__ __forceinline__ float2 stage_group_scales(unsigned short sv, unsigned char zv, uint2 fv) {
+    if constexpr (FMT == GLOWQ_FMT_INT4) {
+        return make_float2(__half2float(__ushort_as_half(sv)), 64.0f + (float)zv);
+    } else if constexpr (FMT == GLOWQ_FMT_MXFP4) {
+        uint2 u;
+        u.x = e8m0_to_f16_bits(fv.x & 0xffu) | (e8m0_to_f16_bits((fv.x >> 8) & 0xffu) << 16);
+        u.y = e8m0_to_f16_bits((fv.x >> 16) & 0xffu) | (e8m0_to_f16_bits(fv.x >> 24) << 16);
+        return *reinterpret_cast<float2*>(&u);
+    } else {
+        return *reinterpret_cast<float2*>(&fv);
+    }
+}
+
+// The four bytes of a packed word (codes 2j, 2j+1 in byte j) as fp16 pairs of
+// exact E2M1 values.
+__device__ __forceinline__ void e2m1_word(uint32_t w, uint32_t p[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3])
+        : "r"(w));
+}
+
+// Two E4M3 bytes (low byte first) as an fp16 pair (exact).
+__device__ __forceinline__ __half2 e4m3x2_to_h2(uint32_t two) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 b;\n\tcvt.u16.u32 b, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, b;\n\t}" : "=r"(r) : "r"(two));
+    return u32_as_h2(r);
+}
+
+template <int NT, bool ONE, int FMT>
 // (the bound of 512 threads caps registers at 128 per thread; launches use at
 // most kMaxWarps compute warps and the control warp).  ONE: T == 1, so only the
 // first column of each MMA tile (lanes t == 0, elements 0 and 2) is finished.
@@ -408,7 +517,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     const int ngroups = d / 128;
     const GemvLayout& L = plan.L;
     unsigned char* ring = smem;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + warps * S * 2048);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + warps * args.stages * 2048);
     uint4* xs = reinterpret_cast<uint4*>(smem + L.xs);
     float* xsum = reinterpret_cast<float*>(smem + L.xsum);
     float2* szs = reinterpret_cast<float2*>(smem + L.sz);
@@ -423,6 +532,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     const int C0 = plan.gsplit[crank * kw], C1 = plan.gsplit[crank * kw + kw];
     const int ncta = C1 - C0;
     const int wpt = ncta * 16;                  // 8-element words per token in the CTA's slice
+    const int xpitch = wpt + 4;                 // row pitch of the staged slice, in 16-byte words
     const int tl = warp % rt, ks = warp / rt;   // tile within the CTA, split index
     const int G0 = control ? 0 : plan.gsplit[crank * kw + ks];
     const int G1 = control ? 0 : plan.gsplit[crank * kw + ks + 1];
@@ -433,12 +543,12 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     // first tile and scale / zero pointers unconditionally (independent loads,
     // one round of misses) rather than a chain of dependent reads.
     int mi = 0, tb = 0;
-    const __half* Ms = args.mod[0].s;
+    const void* Ms = args.mod[0].s;
     const uint8_t* Mz = args.mod[0].z;
 #pragma unroll
     for (int i = 1; i < GLOWQ_MAX_MODULES; ++i) {
         const int b = args.mod[i].tile_begin;
-        const __half* si = args.mod[i].s;
+        const void* si = args.mod[i].s;
         const uint8_t* zi = args.mod[i].z;
         if (i < args.m && tile >= b) {
             mi = i;
@@ -460,7 +570,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     // scale/zero loads, weight stream, A prefetch, scale/zero staging, then X.
     // 1) the weight stream's ring: per warp, S mbarriers; lane 0 issues one 2-D
     //    TMA box (16 rows x 2 groups) per stage
-    constexpr int kStages = S;
+    const int kStages = args.stages;   // ring depth (4 or 8), chosen per launch
     uint64_t* my_bars = bars + warp * kStages;
     unsigned char* my_ring = ring + warp * kStages * 2048;
     const uint32_t ring_smem = smem_u32(my_ring);
@@ -485,17 +595,39 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     const bool one_batch = active && nsub0 <= 32;
     unsigned short sv[16];
     unsigned char zv[16];
+    uint2 fv[16];      // MXFP4: 4 E8M0 bytes of the group; NVFP4: 8 E4M3 bytes
     if (one_batch) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int gg = (lane >> 4) + 2 * j;
-            if (gg < nsub0) {
-                sv[j] = __half_as_ushort(Ms[sz_base + gg]);
-                zv[j] = Mz[sz_base + gg];
-            }
+            if (gg < nsub0) load_group_scales<FMT>(Ms, Mz, sz_base + gg, sv[j], zv[j], fv[j]);
         }
     }
 
+    // 3a) the control warp stages the rows of B that its first projection item
+    //     reads (B is static: the copy runs while the preceding grid finishes;
+    //     issued ahead of the weight stream so that it does not queue behind it)
+    const int nrb = (r + 15) / 16;
+    const int nclusters = (int)gridDim.x / kc;
+    uint64_t* bbar = rbar + 1;
+    unsigned char* bsl = smem + L.bsl;
+    const bool staged_b = control && r > 0 && !args.rpre && L.total > L.bsl && block < nrb * args.rsub &&
+                          [&] { const RItem it = ritem(block, nrb, args.rsub, crank, C0, C1);
+                                return it.g1 - it.g0 <= kBSliceGroups; }();
+    if (staged_b) {
+        const RItem it = ritem(block, nrb, args.rsub, crank, C0, C1);
+        const int rows = (r - it.rb * 16 < 16) ? r - it.rb * 16 : 16;
+        const uint32_t bytes = (uint32_t)(it.g1 - it.g0) * 256u;
+        if (lane == 0) {
+            mbar_init(bbar, 1);
+            fence_mbar_init();
+            mbar_arrive_expect_tx(bbar, bytes * (uint32_t)rows);
+        }
+        __syncwarp();
+        if (lane < rows)
+            bulk_g2s(smem_u32(bsl + lane * kBSlicePitch), args.B + (int64_t)(it.rb * 16 + lane) * d + it.g0 * 128,
+                     bytes, bbar);
+    }
     // 3) start the weight stream (read once per call: evict-first in L2)
     const uint64_t wpol = l2_policy_evict_first();
     if (active) {
@@ -524,38 +656,27 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int gg = (lane >> 4) + 2 * j;
-            if (gg < nsub)
-                my_sz[rr * sz_stride + gg] = make_float2(__half2float(__ushort_as_half(sv[j])), 64.0f + (float)zv[j]);
+            if (gg < nsub) my_sz[rr * sz_stride + gg] = stage_group_scales<FMT>(sv[j], zv[j], fv[j]);
         }
     } else if (active) {
         for (int g0 = lane >> 4; g0 < nsub; g0 += 32) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int gg = g0 + 2 * j;
-                if (gg < nsub) {
-                    sv[j] = __half_as_ushort(Ms[sz_base + gg]);
-                    zv[j] = Mz[sz_base + gg];
-                }
+                if (gg < nsub) load_group_scales<FMT>(Ms, Mz, sz_base + gg, sv[j], zv[j], fv[j]);
             }
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const int gg = g0 + 2 * j;
-                if (gg < nsub)
-                    my_sz[rr * sz_stride + gg] = make_float2(__half2float(__ushort_as_half(sv[j])), 64.0f + (float)zv[j]);
+                if (gg < nsub) my_sz[rr * sz_stride + gg] = stage_group_scales<FMT>(sv[j], zv[j], fv[j]);
             }
         }
     }
-    // Everything above reads only static weight data; activations (and R) may
-    // be produced by the preceding kernels.  After an R kernel, X is final once
-    // every R CTA has passed its own wait (flags[0]), which the control warp
-    // awaits meanwhile; R itself is awaited only during the main loop.  Without
-    // flags, wait for the preceding grid (a no-op when launched without
-    // programmatic serialization).
-    if (control && lane == 0) {
-        mbar_init(rbar, 1);
-        if (args.flags) flag_wait_geq(args.flags + 0, (unsigned)args.nflag, args.status);
-    }
-    if (!args.flags) pdl_wait();
+    // Everything above reads only static weight data.  X may be produced by
+    // the preceding grid, and the hand-off flags are returned to zero by the
+    // preceding call's last CTA: both are final once that grid has completed.
+    if (control && lane == 0) mbar_init(rbar, 1);
+    pdl_wait();
     __syncthreads();   // X is final; rbar is initialised
     // 6) the CTA's activation slice, paired and swizzled (all loads of a batch
     //    first); every thread of the CTA, the control warp included, takes part
@@ -578,6 +699,16 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
             // (token, group) are held by 16 consecutive lanes (stride and wpt
             // are multiples of 16), which add them in a fixed butterfly order
             // into S_E and S_O: xsum[(2 * group + e)][token]
+            if constexpr (FMT != GLOWQ_FMT_INT4) {   // natural k order, no sums
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = base + j * stride;
+                    if (i < items) {
+                        const int tok = i / wpt, wd = i - tok * wpt;
+                        xs[tok * xpitch + (wd & ~15) + ((wd & 3) << 2) + ((wd >> 2) & 3)] = v[j];
+                    }
+                }
+            } else {
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int i = base + j * stride;
@@ -589,8 +720,9 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                     p.y = pair_lo(v[j].y, v[j].w);   // (x2,x6)
                     p.z = pair_hi(v[j].x, v[j].z);   // (x1,x5)
                     p.w = pair_hi(v[j].y, v[j].w);   // (x3,x7)
-                    // swizzle: XOR the two low bits of the word with (bit 3, token parity)
-                    xs[tok * wpt + (wd ^ (((wd >> 3) & 1) | ((tok & 1) << 1)))] = p;
+                    // word 4t + w of a group sits at 4w + t (rows padded by 4 words:
+                    // the fragment loads of a warp hit distinct banks)
+                    xs[tok * xpitch + (wd & ~15) + ((wd & 3) << 2) + ((wd >> 2) & 3)] = p;
                     const float2 f0 = __half22float2(u32_as_h2(p.x)), f2 = __half22float2(u32_as_h2(p.y));
                     const float2 f1 = __half22float2(u32_as_h2(p.z)), f3 = __half22float2(u32_as_h2(p.w));
                     se = (f0.x + f0.y) + (f2.x + f2.y);
@@ -607,10 +739,11 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                     xsum[(2 * gc + 1) * 8 * NT + tok] = so;
                 }
             }
+            }   // INT4
         }
-        for (int i = threadIdx.x; i < wpt; i += stride) xs[T * wpt + i] = make_uint4(0, 0, 0, 0);
+        for (int i = threadIdx.x; i < wpt; i += stride) xs[T * xpitch + i] = make_uint4(0, 0, 0, 0);
         // padding tokens: zero sums
-        for (int i = threadIdx.x; i < ncta * (8 * NT - T); i += stride) {
+        for (int i = threadIdx.x; FMT == GLOWQ_FMT_INT4 && i < ncta * (8 * NT - T); i += stride) {
             const int gc = i / (8 * NT - T), tok = T + (i - gc * (8 * NT - T));
             xsum[(2 * gc) * 8 * NT + tok] = 0.f;
             xsum[(2 * gc + 1) * 8 * NT + tok] = 0.f;
@@ -618,11 +751,46 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     }
     __syncthreads();
 
-    // 7) the control warp: once R is stored, copy it into rs (padding tokens
-    //     zero) and complete rbar; the last CTA here zeroes the flags, which the
-    //     next call's R kernel writes only after this grid has completed
-    if (control && r > 0) {
-        if (args.flags && lane == 0) flag_wait_geq(args.flags + 1, (unsigned)args.nflag, args.status);
+    // 7) the control warp, beside the main loop: this CTA's items of the anchor
+    //    projection (the last producer of a 16-row block of B reduces it into
+    //    the caller's R), then, once every block is stored, R into rs (padding
+    //    tokens zero) for the epilogue; the last CTA here zeroes the flags
+    if (control && r > 0 && args.rpre) {
+        // R was stored by the preceding launch, complete before this grid's wait
+        const int cpr = r / 8;
+        for (int c = lane; c < 8 * NT * cpr; c += 32) {
+            const int tok = c / cpr, cc = c - tok * cpr;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (tok < T) v = ldcg_128(args.R + (int64_t)tok * r + cc * 8);
+            *reinterpret_cast<uint4*>(rs + tok * (r + 8) + cc * 8) = v;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(rbar);
+    } else if (control && r > 0) {
+        const int nslc = kc * args.rsub;   // partials per element of R
+        for (int pi = block; pi < nrb * args.rsub; pi += nclusters) {
+            const RItem it = ritem(pi, nrb, args.rsub, crank, C0, C1);
+            if (pi == block && staged_b) {
+                mbar_wait(bbar, 0u, args.status);
+                rproj_item<NT, FMT == GLOWQ_FMT_INT4>(args, it, bsl, kBSlicePitch, xs, xpitch, C0, lane);
+            } else {
+                rproj_item<NT, FMT == GLOWQ_FMT_INT4>(args, it,
+                               reinterpret_cast<const unsigned char*>(args.B + (int64_t)(it.rb * 16) * d + it.g0 * 128),
+                               (int64_t)d * 2, xs, xpitch, C0, lane);
+            }
+            __syncwarp();   // every lane's partial sums precede lane 0's release
+            unsigned int prev = 0;
+            if (lane == 0)
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(args.flags + it.rb) : "memory");
+            prev = __shfl_sync(0xffffffffu, prev, 0);
+            if (prev == (unsigned)nslc - 1) {   // the block's last producer
+                __syncwarp();   // lane 0's acquire precedes every lane's loads of the partials
+                rproj_reduce(args, it.rb, nslc, lane);
+                __syncwarp();
+                if (lane == 0) flag_release_add(args.flags + kFlagReady, 1u);
+            }
+        }
+        if (lane == 0) flag_wait_geq(args.flags + kFlagReady, (unsigned)nrb, args.status);
         __syncwarp();
         const int cpr = r / 8;   // 16-byte chunks per row
         for (int c = lane; c < 8 * NT * cpr; c += 32) {
@@ -633,142 +801,174 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         }
         __syncwarp();
         if (lane == 0) {
-            if (args.flags) {
-                unsigned int prev;
-                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(args.flags + 2) : "memory");
-                if (prev == gridDim.x - 1) {
-                    args.flags[0] = 0u;
-                    args.flags[1] = 0u;
-                    args.flags[2] = 0u;
-                }
+            unsigned int prev;
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(args.flags + kFlagDone) : "memory");
+            if (prev == gridDim.x - 1) {
+                for (int i = 0; i < nrb; ++i) args.flags[i] = 0u;
+                args.flags[kFlagReady] = 0u;
+                args.flags[kFlagDone] = 0u;
             }
             mbar_arrive(rbar);
         }
     }
 
     // 8) main loop: two independent MMA chains per 128-group on (64 + q) x,
-    //    then s * (D - (64 + z) S) in fp32
+    //    then s * (D - (64 + z) S) in fp32.  One ring stage (two groups) per
+    //    iteration, not unrolled across stages: a launch lasts microseconds,
+    //    so the loop body has to stay small in the instruction cache; every
+    //    shared-memory read inside it is a running pointer plus a constant.
     float acc[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n)
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[n][i] = 0.f;
     if (active) {
-        const float2* sz_lo = my_sz + g * sz_stride;
-        const float2* sz_hi = sz_lo + 8 * sz_stride;
+        const float2* szl = my_sz + g * sz_stride;     // (s, 64 + z) of row g, group by group
+        const float2* szh = szl + 8 * sz_stride;       // row g + 8
         // lanes of padding tokens read the zero row, so every read is unconditional
-        const uint4* xrow[NT];
-        const int xsw = ((t >> 1) & 1) | ((g & 1) << 1);   // swizzle term of this lane
+        const uint4* xb[NT];
 #pragma unroll
         for (int n = 0; n < NT; ++n) {
             const int tok = (n * 8 + g < T) ? n * 8 + g : T;
-            xrow[n] = xs + tok * wpt + (G0 - C0) * 16;
+            xb[n] = xs + tok * xpitch + (G0 - C0) * 16 + t;
         }
-        const float* xsum_w = xsum + (G0 - C0) * 2 * 8 * NT + 2 * t;
-        // Running pointers, advanced once per round of kStages stages, so that
-        // every shared-memory read inside the unrolled round is base + constant:
-        // activation fragment w of token block n, scale/zero pair, group sums.
-        const uint4* xw[NT][4];
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-            for (int w = 0; w < 4; ++w) xw[n][w] = xrow[n] + ((4 * t + w) ^ xsw);
-        const float2* szl = sz_lo;
-        const float2* szh = sz_hi;
-        const float* xsp = xsum_w;
+        const float* xsp = xsum + (G0 - C0) * 2 * 8 * NT + 2 * t;
         // lane (g, t) reads 16 B of rows g and g+8 per group
-        const unsigned char* rd_lo = my_ring + g * 128 + t * 16;
-        const unsigned char* rd_hi = rd_lo + 8 * 128;
+        const unsigned char* rd = my_ring + g * 128 + t * 16;
         bool ok = true;
-        for (int p0 = 0; p0 < npairs; p0 += kStages,
-                 szl += 2 * kStages, szh += 2 * kStages, xsp += 2 * kStages * 2 * 8 * NT) {
+        int slot = 0;
+        uint32_t phase = 0;
+#pragma unroll 1
+        for (int p = 0; p < npairs; ++p) {
+            if (ok) ok = mbar_wait(my_bars + slot, phase, args.status);
+            const unsigned char* sl = rd + slot * 2048;
+            uint4 w4[2][2];
+            w4[0][0] = *reinterpret_cast<const uint4*>(sl);
+            w4[0][1] = *reinterpret_cast<const uint4*>(sl + 1024);
+            w4[1][0] = *reinterpret_cast<const uint4*>(sl + 64);
+            w4[1][1] = *reinterpret_cast<const uint4*>(sl + 1024 + 64);
+            if (p + kStages < npairs) {
+                fence_proxy_async_smem();   // this lane's reads of the slot precede the refill
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(my_bars + slot, 2048u);
+                    tma_load_2d_hint(ring_smem + slot * 2048, tmq, my_bars + slot, (G0 + 2 * (p + kStages)) * 16,
+                                     tile_row, wpol);
+                }
+            }
+            const bool two = 2 * p + 1 < nsub;    // warp-uniform
+            if constexpr (FMT != GLOWQ_FMT_INT4) {
 #pragma unroll
-            for (int i = 0; i < kStages; ++i) {
-                const int p = p0 + i;
-                if (p < npairs) {
-                    if (ok) ok = mbar_wait(my_bars + i, (uint32_t)((p / kStages) & 1), args.status);
-                    const unsigned char* sl = rd_lo + i * 2048;
-                    const unsigned char* sh = rd_hi + i * 2048;
-                    uint4 w4[2][2];
-                    w4[0][0] = *reinterpret_cast<const uint4*>(sl);
-                    w4[0][1] = *reinterpret_cast<const uint4*>(sh);
-                    w4[1][0] = *reinterpret_cast<const uint4*>(sl + 64);
-                    w4[1][1] = *reinterpret_cast<const uint4*>(sh + 64);
-                    if (p + kStages < npairs) {
-                        fence_proxy_async_smem();   // this lane's reads of the slot precede the refill
-                        __syncwarp();
-                        if (lane == 0) {
-                            mbar_arrive_expect_tx(my_bars + i, 2048u);
-                            tma_load_2d_hint(ring_smem + i * 2048, tmq, my_bars + i, (G0 + 2 * (p + kStages)) * 16,
-                                             tile_row, wpol);
-                        }
+                for (int h = 0; h < 2; ++h) {
+                    if (h == 1 && !two) break;
+                    const uint32_t wl[4] = {w4[h][0].x, w4[h][0].y, w4[h][0].z, w4[h][0].w};
+                    const uint32_t wh[4] = {w4[h][1].x, w4[h][1].y, w4[h][1].z, w4[h][1].w};
+                    // block scales of rows g and g+8: words 0-1 and 2-3 of the lane
+                    // (k 32t .. 32t+15 and 32t+16 .. 32t+31) for NVFP4, all four for MXFP4
+                    __half2 sl0, sl1, sh0, sh1;
+                    if constexpr (FMT == GLOWQ_FMT_MXFP4) {
+                        sl0 = sl1 = __half2half2(reinterpret_cast<const __half*>(szl + h)[t]);
+                        sh0 = sh1 = __half2half2(reinterpret_cast<const __half*>(szh + h)[t]);
+                    } else {
+                        const __half2 ql = e4m3x2_to_h2(reinterpret_cast<const unsigned short*>(szl + h)[t]);
+                        const __half2 qh = e4m3x2_to_h2(reinterpret_cast<const unsigned short*>(szh + h)[t]);
+                        sl0 = __low2half2(ql);
+                        sl1 = __high2half2(ql);
+                        sh0 = __low2half2(qh);
+                        sh1 = __high2half2(qh);
                     }
-                    const bool two = 2 * p + 1 < nsub;    // warp-uniform
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        if (h == 1 && !two) break;
-                        const int gi = 2 * i + h;          // group within this round (a constant)
-                        const uint32_t wl[4] = {w4[h][0].x, w4[h][0].y, w4[h][0].z, w4[h][0].w};
-                        const uint32_t wh[4] = {w4[h][1].x, w4[h][1].y, w4[h][1].z, w4[h][1].w};
-                        // two MMA chains: even k (A = 16 + q/64) and odd k (A = 64 + q)
-                        float te[NT][4], to[NT][4];
+                    for (int w = 0; w < 4; ++w) {
+                        uint32_t pl[4], ph[4];
+                        e2m1_word(wl[w], pl);   // row g: pairs (8w + 2j, 8w + 2j + 1) of the lane's 32 k
+                        e2m1_word(wh[w], ph);   // row g + 8
+                        const __half2 scl = (w < 2) ? sl0 : sl1, sch = (w < 2) ? sh0 : sh1;
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            uint32_t el[2], ol[2], eh[2], oh[2];
-                            unpack_even_odd(wl[w], el, ol);   // row g
-                            unpack_even_odd(wh[w], eh, oh);   // row g + 8
-                            const uint32_t ae[4] = {el[0], eh[0], el[1], eh[1]};
-                            const uint32_t ao[4] = {ol[0], oh[0], ol[1], oh[1]};
-#pragma unroll
-                            for (int n = 0; n < NT; ++n) {
-                                const uint4 x = xw[n][w][gi * 16];
-                                const uint32_t be[2] = {x.x, x.y};   // (x0,x4) (x2,x6)
-                                const uint32_t bo[2] = {x.z, x.w};   // (x1,x5) (x3,x7)
-                                if (w == 0) {
-                                    mma_16816_zc(te[n], ae, be);
-                                    mma_16816_zc(to[n], ao, bo);
-                                } else {
-                                    mma_16816(te[n], ae, be);
-                                    mma_16816(to[n], ao, bo);
-                                }
-                            }
+                        for (int j = 0; j < 4; ++j) {
+                            pl[j] = h2_as_u32(__hmul2(u32_as_h2(pl[j]), scl));
+                            ph[j] = h2_as_u32(__hmul2(u32_as_h2(ph[j]), sch));
                         }
-                        // sum_k (q - z) x = 64 D_E + D_O - (1024 + z) S_E - (64 + z) S_O, times s
-                        const float2 zl = szl[gi], zh = szh[gi];   // (s, 64 + z)
-                        const float cel = zl.y + 960.0f, ceh = zh.y + 960.0f;
+                        const uint32_t a0[4] = {pl[0], ph[0], pl[1], ph[1]};
+                        const uint32_t a1[4] = {pl[2], ph[2], pl[3], ph[3]};
 #pragma unroll
                         for (int n = 0; n < NT; ++n) {
-                            const float2 se = *reinterpret_cast<const float2*>(xsp + (2 * gi) * 8 * NT + n * 8);
-                            const float2 so = *reinterpret_cast<const float2*>(xsp + (2 * gi + 1) * 8 * NT + n * 8);
-                            if (ONE) {
-                                float v0 = fmaf(64.0f, te[n][0], to[n][0]);
-                                float v2 = fmaf(64.0f, te[n][2], to[n][2]);
-                                v0 = fmaf(-zl.y, so.x, fmaf(-cel, se.x, v0));
-                                v2 = fmaf(-zh.y, so.x, fmaf(-ceh, se.x, v2));
-                                acc[n][0] = fmaf(zl.x, v0, acc[n][0]);
-                                acc[n][2] = fmaf(zh.x, v2, acc[n][2]);
-                                continue;
-                            }
-                            float v0 = fmaf(64.0f, te[n][0], to[n][0]);
-                            float v1 = fmaf(64.0f, te[n][1], to[n][1]);
-                            float v2 = fmaf(64.0f, te[n][2], to[n][2]);
-                            float v3 = fmaf(64.0f, te[n][3], to[n][3]);
-                            v0 = fmaf(-zl.y, so.x, fmaf(-cel, se.x, v0));
-                            v1 = fmaf(-zl.y, so.y, fmaf(-cel, se.y, v1));
-                            v2 = fmaf(-zh.y, so.x, fmaf(-ceh, se.x, v2));
-                            v3 = fmaf(-zh.y, so.y, fmaf(-ceh, se.y, v3));
-                            acc[n][0] = fmaf(zl.x, v0, acc[n][0]);
-                            acc[n][1] = fmaf(zl.x, v1, acc[n][1]);
-                            acc[n][2] = fmaf(zh.x, v2, acc[n][2]);
-                            acc[n][3] = fmaf(zh.x, v3, acc[n][3]);
+                            const uint4 x = xb[n][h * 16 + w * 4];   // x of k 8w .. 8w+7 in order
+                            const uint32_t b0[2] = {x.x, x.y};
+                            const uint32_t b1[2] = {x.z, x.w};
+                            mma_16816(acc[n], a0, b0);
+                            mma_16816(acc[n], a1, b1);
                         }
                     }
                 }
+            } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h == 1 && !two) break;
+                const uint32_t wl[4] = {w4[h][0].x, w4[h][0].y, w4[h][0].z, w4[h][0].w};
+                const uint32_t wh[4] = {w4[h][1].x, w4[h][1].y, w4[h][1].z, w4[h][1].w};
+                // two MMA chains: even k (A = 16 + q/64) and odd k (A = 64 + q)
+                float te[NT][4], to[NT][4];
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t el[2], ol[2], eh[2], oh[2];
+                    unpack_even_odd(wl[w], el, ol);   // row g
+                    unpack_even_odd(wh[w], eh, oh);   // row g + 8
+                    const uint32_t ae[4] = {el[0], eh[0], el[1], eh[1]};
+                    const uint32_t ao[4] = {ol[0], oh[0], ol[1], oh[1]};
+#pragma unroll
+                    for (int n = 0; n < NT; ++n) {
+                        const uint4 x = xb[n][h * 16 + w * 4];
+                        const uint32_t be[2] = {x.x, x.y};   // (x0,x4) (x2,x6)
+                        const uint32_t bo[2] = {x.z, x.w};   // (x1,x5) (x3,x7)
+                        if (w == 0) {
+                            mma_16816_zc(te[n], ae, be);
+                            mma_16816_zc(to[n], ao, bo);
+                        } else {
+                            mma_16816(te[n], ae, be);
+                            mma_16816(to[n], ao, bo);
+                        }
+                    }
+                }
+                // sum_k (q - z) x = 64 D_E + D_O - (1024 + z) S_E - (64 + z) S_O, times s
+                const float2 zl = szl[h], zh = szh[h];   // (s, 64 + z)
+                const float cel = zl.y + 960.0f, ceh = zh.y + 960.0f;
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
+                    const float2 se = *reinterpret_cast<const float2*>(xsp + (2 * h) * 8 * NT + n * 8);
+                    const float2 so = *reinterpret_cast<const float2*>(xsp + (2 * h + 1) * 8 * NT + n * 8);
+                    if (ONE) {
+                        float v0 = fmaf(64.0f, te[n][0], to[n][0]);
+                        float v2 = fmaf(64.0f, te[n][2], to[n][2]);
+                        v0 = fmaf(-zl.y, so.x, fmaf(-cel, se.x, v0));
+                        v2 = fmaf(-zh.y, so.x, fmaf(-ceh, se.x, v2));
+                        acc[n][0] = fmaf(zl.x, v0, acc[n][0]);
+                        acc[n][2] = fmaf(zh.x, v2, acc[n][2]);
+                        continue;
+                    }
+                    float v0 = fmaf(64.0f, te[n][0], to[n][0]);
+                    float v1 = fmaf(64.0f, te[n][1], to[n][1]);
+                    float v2 = fmaf(64.0f, te[n][2], to[n][2]);
+                    float v3 = fmaf(64.0f, te[n][3], to[n][3]);
+                    v0 = fmaf(-zl.y, so.x, fmaf(-cel, se.x, v0));
+                    v1 = fmaf(-zl.y, so.y, fmaf(-cel, se.y, v1));
+                    v2 = fmaf(-zh.y, so.x, fmaf(-ceh, se.x, v2));
+                    v3 = fmaf(-zh.y, so.y, fmaf(-ceh, se.y, v3));
+                    acc[n][0] = fmaf(zl.x, v0, acc[n][0]);
+                    acc[n][1] = fmaf(zl.x, v1, acc[n][1]);
+                    acc[n][2] = fmaf(zh.x, v2, acc[n][2]);
+                    acc[n][3] = fmaf(zh.x, v3, acc[n][3]);
+                }
             }
+            }   // INT4
+            szl += 2;
+            szh += 2;
+            xsp += 2 * 2 * 8 * NT;
 #pragma unroll
-            for (int n = 0; n < NT; ++n)
-#pragma unroll
-                for (int w = 0; w < 4; ++w) xw[n][w] += 2 * kStages * 16;
+            for (int n = 0; n < NT; ++n) xb[n] += 32;
+            if (++slot == kStages) {
+                slot = 0;
+                phase ^= 1u;
+            }
         }
     }
     cp_async_wait<0>();
@@ -829,6 +1029,15 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     }
     if (!active) return;
 
+    // NVFP4: the fp32 tensor scale of the base product
+    if constexpr (FMT == GLOWQ_FMT_NVFP4) {
+        const float st = __ldg(M.ts);
+#pragma unroll
+        for (int n = 0; n < NT; ++n)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[n][i] *= st;
+    }
+
     // 10) rank-r correction A_i R^T, accumulated into the same fp32 registers
     //     (R from shared memory, staged by the control warp)
     if (has_corr) {
@@ -873,43 +1082,9 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
 // ---------------------------------------------------------------------------
 // Host-side launchers (called from api.cu after validation).
 // ---------------------------------------------------------------------------
-static cudaError_t launch_ex(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
-                             void** args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = block;
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelExC(&cfg, fn, args);
+size_t decode_partial_bytes(int64_t T, int r) {
+    return (size_t)kRMaxSlices * (size_t)T * (size_t)r * sizeof(float);
 }
-
-// R = X B^T into R (fp16) with one cluster of kRcCtas CTAs.
-cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, uint16_t* R,
-                                unsigned int* flags, cudaStream_t st) {
-    const int nt = (T <= 8) ? 1 : 2;
-    const __half* Xh = reinterpret_cast<const __half*>(X);
-    const __half* Bh = reinterpret_cast<const __half*>(B);
-    __half* Rh = reinterpret_cast<__half*>(R);
-    unsigned int* status = device_status_ptr();
-    void* a1[] = {(void*)&Xh, (void*)&Bh, (void*)&T, (void*)&d, (void*)&r, (void*)&Rh, (void*)&flags, (void*)&status};
-    const void* fn = (nt == 1) ? (const void*)rproj_cluster_kernel<1> : (const void*)rproj_cluster_kernel<2>;
-    const size_t smem = (size_t)rc_smem_bytes(r, d, nt);
-    // opt in to the largest dynamic shared memory requested so far (at most
-    // the staged B slice, the partials of r <= 256 and a 16-token X slice)
-    static size_t opted[2] = {48 * 1024, 48 * 1024};
-    if (smem > opted[nt - 1]) {
-        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        opted[nt - 1] = smem;
-    }
-    return launch_ex(fn, dim3(kRcCtas), dim3(kRcWarps * 32), smem, st, true, a1);
-}
-
 
 // Resident CTAs of one variant and shape (cached: the occupancy query is not free).
 static int resident_ctas(const void* fn, int warps, int kc, size_t smem, int num_sms) {
@@ -944,32 +1119,50 @@ static int resident_ctas(const void* fn, int warps, int kc, size_t smem, int num
     return n;
 }
 
-struct GemvShape { int rt, kw, kc, stages; size_t smem; };
+struct GemvShape { int rt, kw, kc, stages; size_t smem; int res; int bstage; };  // res: resident CTAs of the launch
 
 // one: T == 1 (a single token: only one output column is finished)
-static const void* gemv_fn(int nt, int stages, bool one = false) {
-    if (nt == 1) {
-        if (one)
-            return stages == 8 ? (const void*)corrected_gemv_kernel<1, 8, true>
-                               : (const void*)corrected_gemv_kernel<1, 4, true>;
-        return stages == 8 ? (const void*)corrected_gemv_kernel<1, 8, false> : (const void*)corrected_gemv_kernel<1, 4, false>;
-    }
-    return stages == 8 ? (const void*)corrected_gemv_kernel<2, 8, false> : (const void*)corrected_gemv_kernel<2, 4, false>;
+template <int FMT>
+static const void* gemv_fn_fmt(int nt, bool one) {
+    if (nt == 1)
+        return one ? (const void*)corrected_gemv_kernel<1, true, FMT> : (const void*)corrected_gemv_kernel<1, false, FMT>;
+    return (const void*)corrected_gemv_kernel<2, false, FMT>;
+}
+
+static const void* gemv_fn(int nt, int stages, bool one = false, int fmt = GLOWQ_FMT_INT4) {
+    (void)stages;   // the ring depth is a launch argument
+    if (fmt == GLOWQ_FMT_MXFP4) return gemv_fn_fmt<GLOWQ_FMT_MXFP4>(nt, one);
+    if (fmt == GLOWQ_FMT_NVFP4) return gemv_fn_fmt<GLOWQ_FMT_NVFP4>(nt, one);
+    return gemv_fn_fmt<GLOWQ_FMT_INT4>(nt, one);
 }
 
 // Pick (rt, kw, kc, stages): all CTAs resident in one wave; then as many SMs
 // busy as possible; then as many resident warps per SM as possible (up to 16);
 // then as many weight bytes in flight per SM as possible (up to 128 KB); then
 // the fewest splits of d.  If nothing fits in one wave, the fewest waves.
-static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sms) {
-    struct Key { int tiles, d, T, r, nt; GemvShape s; };
+static GemvShape choose_shape_b(int tiles, int d, int T, int r, int nt, int num_sms, int fmt, bool bstage);
+
+// The B rows of a projection item are staged in shared memory unless that
+// costs the launch its single wave.
+static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sms, int fmt) {
+    GemvShape s = choose_shape_b(tiles, d, T, r, nt, num_sms, fmt, true);
+    if (r > 0 && s.rt > 0 && (long)ceil_div(tiles, s.rt) * s.kc > s.res) {
+        GemvShape u = choose_shape_b(tiles, d, T, r, nt, num_sms, fmt, false);
+        if (u.rt > 0 && (long)ceil_div(tiles, u.rt) * u.kc <= u.res) return u;
+    }
+    return s;
+}
+
+static GemvShape choose_shape_b(int tiles, int d, int T, int r, int nt, int num_sms, int fmt, bool bstage) {
+    struct Key { int tiles, d, T, r, nt, fmt, b; GemvShape s; };
     static Key memo[128];
     static int used = 0;
     for (int i = 0; i < used; ++i)
-        if (memo[i].tiles == tiles && memo[i].d == d && memo[i].T == T && memo[i].r == r && memo[i].nt == nt)
+        if (memo[i].tiles == tiles && memo[i].d == d && memo[i].T == T && memo[i].r == r && memo[i].nt == nt &&
+            memo[i].fmt == fmt && memo[i].b == (int)bstage)
             return memo[i].s;
     const int ngroups = d / 128;
-    GemvShape best = {0, 0, 0, 0, 0};
+    GemvShape best = {0, 0, 0, 0, 0, 0, 0};
     double best_key[5] = {1e30, 1e30, 1e30, 1e30, 1e30};
     // Cost model: the busiest SM sets the time.  CTAs of a cluster launch are
     // packed onto SMs up to their residency (observed: two 8-warp CTAs per SM
@@ -987,11 +1180,11 @@ static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sm
                     if (kc > 1 && kw > 1) break;
                     if (kc > ngroups || ngroups / kc < kw) continue;
                     const int warps = rt * kw;   // compute warps (+1 control warp per CTA)
-                    const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, nt, stages);
+                    const GemvLayout L = gemv_layout(T, d, r, rt, kw, kc, nt, stages, bstage);
                     if (L.total > 220 * 1024) continue;
                     if (pad && (size_t)L.total >= kSpreadSmem) continue;
                     const size_t smem = pad ? kSpreadSmem : (size_t)L.total;
-                    const void* fn = gemv_fn(nt, stages);
+                    const void* fn = gemv_fn(nt, stages, false, fmt);
                     const int res = resident_ctas(fn, warps + 1, kc, smem, num_sms);
                     if (res <= 0) continue;
                     const long ctas = (long)ceil_div(tiles, rt) * kc;
@@ -1016,26 +1209,28 @@ static GemvShape choose_shape(int tiles, int d, int T, int r, int nt, int num_sm
                     }
                     if (better) {
                         for (int j = 0; j < 5; ++j) best_key[j] = key[j];
-                        best = {rt, kw, kc, stages, smem};
+                        best = {rt, kw, kc, stages, smem, res, (int)bstage};
                     }
                 }
-    if (used < 128 && best.rt > 0) memo[used++] = {tiles, d, T, r, nt, best};
+    if (used < 128 && best.rt > 0) memo[used++] = {tiles, d, T, r, nt, fmt, (int)bstage, best};
     if (std::getenv("GLOWQ_VERBOSE"))
         std::fprintf(stderr,
-                     "glowq decode shape: tiles=%d d=%d T=%d r=%d -> rt=%d kw=%d kc=%d stages=%d smem=%zu ctas=%d\n",
-                     tiles, d, T, r, best.rt, best.kw, best.kc, best.stages, best.smem,
+                     "glowq decode shape: tiles=%d d=%d T=%d r=%d b=%d -> rt=%d kw=%d kc=%d stages=%d smem=%zu ctas=%d\n",
+                     tiles, d, T, r, (int)bstage, best.rt, best.kw, best.kc, best.stages, best.smem,
                      best.rt ? ceil_div(tiles, best.rt) * best.kc : 0);
     return best;
 }
 
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
-                               const uint16_t* R, unsigned int* flags, int num_sms, cudaStream_t st) {
+                               const uint16_t* B, uint16_t* R, unsigned int* flags, float* partial, int num_sms,
+                               cudaStream_t st, int fmt) {
     GemvArgs a = {};
     int tiles = 0;
     for (int i = 0; i < m; ++i) {
         a.mod[i].q = mods[i].q;
-        a.mod[i].s = reinterpret_cast<const __half*>(mods[i].s);
+        a.mod[i].s = mods[i].s;
         a.mod[i].z = mods[i].z;
+        a.mod[i].ts = mods[i].ts;
         a.mod[i].A = (r > 0) ? reinterpret_cast<const __half*>(mods[i].A) : nullptr;
         a.mod[i].Y = reinterpret_cast<__half*>(mods[i].Y);
         a.mod[i].ldY = mods[i].ldY;
@@ -1050,16 +1245,16 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     const int nt = (T <= 8) ? 1 : 2;
     static bool opted = false;
     if (!opted) {
-        for (int n = 1; n <= 2; ++n)
-            for (int sg = 4; sg <= 8; sg *= 2)
+        for (int f = 0; f <= 2; ++f)
+            for (int n = 1; n <= 2; ++n)
                 for (int one = 0; one <= (n == 1 ? 1 : 0); ++one) {
-                    cudaError_t e = cudaFuncSetAttribute(gemv_fn(n, sg, one != 0),
+                    cudaError_t e = cudaFuncSetAttribute(gemv_fn(n, 4, one != 0, f),
                                                          cudaFuncAttributeMaxDynamicSharedMemorySize, 220 * 1024);
                     if (e != cudaSuccess) return e;
                 }
         opted = true;
     }
-    GemvShape sh = choose_shape(tiles, d, T, r, nt, num_sms);
+    GemvShape sh = choose_shape(tiles, d, T, r, nt, num_sms, fmt);
     // Tuning override: GLOWQ_DECODE_SHAPE="rt,kw,kc,stages" (validated here).
     if (const char* env = std::getenv("GLOWQ_DECODE_SHAPE")) {
         int v[4] = {0, 0, 0, 0};
@@ -1067,12 +1262,13 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
             v[2] >= 1 && v[2] <= 8 && v[0] * v[1] <= kMaxWarps && (v[2] == 1 || v[1] == 1) &&
             (v[3] == 4 || v[3] == 8) && v[2] <= d / 128 && (d / 128) / v[2] >= v[1]) {
             const GemvLayout L = gemv_layout(T, d, r, v[0], v[1], v[2], nt, v[3]);
-            if (L.total <= 220 * 1024) sh = {v[0], v[1], v[2], v[3], (size_t)L.total};
+            const int res = resident_ctas(gemv_fn(nt, v[3], false, fmt), v[0] * v[1] + 1, v[2], (size_t)L.total, num_sms);
+            if (L.total <= 220 * 1024 && res > 0) sh = {v[0], v[1], v[2], v[3], (size_t)L.total, res, 1};
         }
     }
     if (sh.rt == 0) return cudaErrorInvalidValue;
     GemvPlan plan = {};
-    plan.L = gemv_layout(T, d, r, sh.rt, sh.kw, sh.kc, nt, sh.stages);
+    plan.L = gemv_layout(T, d, r, sh.rt, sh.kw, sh.kc, nt, sh.stages, sh.bstage != 0);
     const int ngroups = d / 128;
     for (int c = 0; c < sh.kc; ++c) {
         const int c0 = c * ngroups / sh.kc, c1 = (c + 1) * ngroups / sh.kc;
@@ -1086,13 +1282,52 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     a.rt = sh.rt;
     a.kw = sh.kw;
     a.kc = sh.kc;
+    const int grid = ceil_div(tiles, sh.rt) * sh.kc;
     a.flags = (r > 0) ? flags : nullptr;
-    a.nflag = kRcCtas;
     a.X = reinterpret_cast<const __half*>(X);
-    a.R = reinterpret_cast<const __half*>(R);
+    a.B = reinterpret_cast<const __half*>(B);
+    a.R = reinterpret_cast<__half*>(R);
+    a.part = partial;
+    // Sub-slices of the anchor projection: items of at most kBSliceGroups
+    // groups (staged in shared memory), at most one per cluster while the grid
+    // and its first wave have room (clusters are dispatched in order, so no CTA
+    // waits on a producer that is not resident), kc * rsub <= kRMaxSlices
+    {
+        const int nrb = (r + 15) / 16;
+        const int room = (grid < sh.res ? grid : sh.res) / sh.kc;
+        const int slice_groups = ceil_div(ngroups, sh.kc);
+        int rs = ceil_div(slice_groups, kBSliceGroups);
+        if (r > 0 && rs * nrb > room) rs = room / nrb;
+        if (rs * sh.kc > kRMaxSlices) rs = kRMaxSlices / sh.kc;
+        if (rs > ngroups / sh.kc) rs = ngroups / sh.kc;
+        a.rsub = rs > 0 ? rs : 1;
+    }
     a.status = device_status_ptr();
+    // A grid larger than one wave gets R from a separate launch first: its
+    // CTAs must not wait on producers that may not be resident.
+    a.rpre = (r > 0 && grid > sh.res) ? 1 : 0;
+    a.stages = sh.stages;
+    if (a.rpre) {
+        int S = ngroups / 4;
+        if (S > kRMaxSlices) S = kRMaxSlices;
+        if (S < 1) S = 1;
+        const int nrb = (r + 15) / 16;
+        cudaLaunchConfig_t rc = {};
+        rc.gridDim = dim3(nrb * S);
+        rc.blockDim = dim3(kRpWarps * 32);
+        rc.stream = st;
+        cudaLaunchAttribute ra[1];
+        ra[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        ra[0].val.programmaticStreamSerializationAllowed = 1;
+        rc.attrs = ra;
+        rc.numAttrs = 1;
+        void* rargs[] = {(void*)&a, (void*)&S};
+        const void* rfn = (nt == 1) ? (const void*)rproj_decode_kernel<1> : (const void*)rproj_decode_kernel<2>;
+        cudaError_t e = cudaLaunchKernelExC(&rc, rfn, rargs);
+        if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(ceil_div(tiles, sh.rt) * sh.kc);
+    cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3((sh.rt * sh.kw + 1) * 32);   // compute warps + the control warp
     cfg.dynamicSmemBytes = sh.smem;
     cfg.stream = st;
@@ -1110,7 +1345,7 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     cfg.attrs = attr;
     cfg.numAttrs = na;
     void* args[] = {(void*)&a, (void*)&plan};
-    return cudaLaunchKernelExC(&cfg, gemv_fn(nt, sh.stages, T == 1), args);
+    return cudaLaunchKernelExC(&cfg, gemv_fn(nt, sh.stages, T == 1, fmt), args);
 }
 
 }  // namespace glowq

@@ -12,9 +12,10 @@ namespace glowq {
 
 // Host-side view of one module of a group (validated by api.cu).
 struct ModuleView {
-    const uint32_t* q;
-    const uint16_t* s;
-    const uint8_t* z;
+    const uint32_t* q;   // packed 4-bit codes [O][d/8]
+    const void* s;       // INT4: fp16 scales [O][d/128]; MXFP4 / NVFP4: scale bytes
+    const uint8_t* z;    // INT4 zeros (nullptr for FP4)
+    const float* ts;     // NVFP4 tensor scale (device), else nullptr
     const uint16_t* A;   // nullptr: correction off for this module
     uint16_t* Y;
     int64_t ldY;
@@ -31,16 +32,14 @@ glowq_status validate_solo_call(const glowq_module* mod, int64_t d, const uint16
 unsigned int* device_status_ptr();
 
 // decode.cu
-// R = X B^T (T <= 16) by one thread-block cluster, written to R in fp16.
-// flags: three zeroed words through which the GEMV that follows learns that X
-// is final and that R is stored (the GEMV zeroes them again).
-constexpr int kDecodeFlagWords = 3;
-cudaError_t launch_rproj_decode(const uint16_t* X, const uint16_t* B, int T, int d, int r, uint16_t* R,
-                                unsigned int* flags, cudaStream_t st);
-// Corrected GEMV over the stacked rows; with flags (after launch_rproj_decode
-// with the same flags) it waits on them instead of on the R kernel's completion.
+// Corrected GEMV over the stacked rows (T <= 16), one launch.  With r > 0 it
+// also computes R = X B^T (written to R) from fp32 partial sums in `partial`
+// (decode_partial_bytes(T, r)); `flags` are 256 zeroed workspace bytes that
+// every completed call leaves zero.
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
-                               const uint16_t* R, unsigned int* flags, int num_sms, cudaStream_t st);
+                               const uint16_t* B, uint16_t* R, unsigned int* flags, float* partial, int num_sms,
+                               cudaStream_t st, int fmt = GLOWQ_FMT_INT4);
+size_t decode_partial_bytes(int64_t T, int r);
 // pack.cu
 cudaError_t launch_pack_int4(const float* W, int64_t O, int64_t d, uint32_t* q, uint16_t* s, uint8_t* z,
                              cudaStream_t st);
@@ -48,6 +47,11 @@ cudaError_t launch_dequant_int4(const uint32_t* q, const uint16_t* s, const uint
                                 uint16_t* out, cudaStream_t st);
 cudaError_t launch_error_norms(const float* W, const uint32_t* q, const uint16_t* s, const uint8_t* z,
                                int64_t O, int64_t d, double* out_rows, cudaStream_t st);
+// fp4.cu
+cudaError_t launch_pack_fp4(int fmt, const float* W, int64_t O, int64_t d, uint32_t* codes, uint8_t* scales,
+                            float* tensor_scale, cudaStream_t st);
+cudaError_t launch_dequant_fp4(int fmt, const uint32_t* codes, const uint8_t* scales, const float* tensor_scale,
+                               int64_t O, int64_t d, uint16_t* out, cudaStream_t st);
 // prefill.cu: TMA tensor maps (driver entry point resolved at run time)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -60,7 +64,7 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
 // (nullptr: one slice of d per CTA, R written directly).
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r,
                                    const uint16_t* X, int64_t T, uint16_t* R, float* partial, int num_sms,
-                                   cudaStream_t st);
+                                   cudaStream_t st, int fmt = GLOWQ_FMT_INT4);
 size_t prefill_partial_bytes(int64_t T, int r);
 
 }  // namespace glowq

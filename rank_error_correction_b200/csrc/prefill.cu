@@ -168,8 +168,9 @@ static_assert(kGemmStages % 2 == 0, "transform groups own alternate stages");
 static_assert(kGemmStages * kStageBytesG + kEpiBufs * kEpiBytes + 1024 + 256 <= 232448, "shared memory per CTA");
 
 struct PrefillModule {
-    const __half* s;
-    const uint8_t* z;
+    const void* s;     // INT4 fp16 scales [O][d/128]; MXFP4 / NVFP4 scale bytes [O][d/32] / [O][d/16]
+    const uint8_t* z;  // INT4 zeros
+    const float* ts;   // NVFP4 tensor scale (device)
     __half* Y;
     int64_t ldY;
     int O;
@@ -326,6 +327,27 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
+// E8M0 scale code -> fp16 bits of 2^(e - 127), clamped to [2^-24, 2^15] (0 below).
+__device__ __forceinline__ uint32_t pf_e8m0_f16(uint32_t e) {
+    if (e >= 113u && e <= 142u) return (e - 112u) << 10;
+    if (e > 142u) return 0x7800u;
+    if (e >= 103u) return 1u << (e - 103u);
+    return 0u;
+}
+// fp16 bits of fp16_RN(e4m3 * s_t) (the E4M3 value is exact in fp32; one
+// rounding to fp32, one to fp16).
+__device__ __forceinline__ uint32_t pf_e4m3_st_f16(uint32_t c, float st) {
+    uint32_t h;
+    asm("{\n\t.reg .b16 b;\n\t.reg .b32 p;\n\tcvt.u16.u32 b, %1;\n\tcvt.rn.f16x2.e4m3x2 p, b;\n\t"
+        "mov.b32 %0, p;\n\t}" : "=r"(h) : "r"(c & 0xffu));
+    const float v = __half2float(__ushort_as_half((unsigned short)(h & 0xffffu))) * st;
+    return (uint32_t)__half_as_ushort(__float2half_rn(v));
+}
+
+// FMT: GLOWQ_FMT_INT4 (w_hat = fp16((q - z) s)), GLOWQ_FMT_MXFP4 or
+// GLOWQ_FMT_NVFP4 (w_hat = fp16 of the E2M1 value times the block scale,
+// see the transform warps).
+template <int FMT>
 __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const __grid_constant__ PrefillArgs args) {
     extern __shared__ __align__(1024) unsigned char gsm_raw[];
     // 1024-byte alignment of the stage buffers (swizzle atoms); the same offset in both CTAs
@@ -462,14 +484,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
         int cur_tile = first_tile;
         int f_tile = cur_tile, f_grp = 0;              // next group to fetch
         TileCoord fc = tile_coord(args, cur_tile < args.ntiles ? cur_tile : 0);
-        auto fetch = [&]() -> uint32_t {
-            uint32_t v = 0;
+        // per group: INT4 (s | z << 16) in .x; MXFP4 the four block scales as
+        // fp16 in .x .y; NVFP4 the eight fp16_RN(e4m3 * s_t) in .x .. .w
+        auto fetch = [&]() -> uint4 {
+            uint4 v = make_uint4(0, 0, 0, 0);
             if (f_tile < args.ntiles) {
                 const int orow = fc.m0 + row_off + row;
                 const PrefillModule& FM = args.mod[fc.mi];
                 if (orow < FM.O) {
                     const int64_t o = (int64_t)orow * ngroups + f_grp;
-                    v = (uint32_t)__half_as_ushort(FM.s[o]) | ((uint32_t)FM.z[o] << 16);
+                    if constexpr (FMT == GLOWQ_FMT_INT4) {
+                        v.x = (uint32_t)__half_as_ushort(static_cast<const __half*>(FM.s)[o]) |
+                              ((uint32_t)FM.z[o] << 16);
+                    } else if constexpr (FMT == GLOWQ_FMT_MXFP4) {
+                        const uint32_t e4 = static_cast<const uint32_t*>(FM.s)[o];
+                        v.x = pf_e8m0_f16(e4 & 0xffu) | (pf_e8m0_f16((e4 >> 8) & 0xffu) << 16);
+                        v.y = pf_e8m0_f16((e4 >> 16) & 0xffu) | (pf_e8m0_f16(e4 >> 24) << 16);
+                    } else {
+                        const uint2 e8 = static_cast<const uint2*>(FM.s)[o];
+                        const float st = __ldg(FM.ts);
+                        v.x = pf_e4m3_st_f16(e8.x, st) | (pf_e4m3_st_f16(e8.x >> 8, st) << 16);
+                        v.y = pf_e4m3_st_f16(e8.x >> 16, st) | (pf_e4m3_st_f16(e8.x >> 24, st) << 16);
+                        v.z = pf_e4m3_st_f16(e8.y, st) | (pf_e4m3_st_f16(e8.y >> 8, st) << 16);
+                        v.w = pf_e4m3_st_f16(e8.y >> 16, st) | (pf_e4m3_st_f16(e8.y >> 24, st) << 16);
+                    }
                 }
                 if (++f_grp == ngroups) {
                     f_grp = 0;
@@ -479,7 +517,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
             }
             return v;
         };
-        uint32_t sz0 = fetch(), sz1 = fetch(), sz2 = fetch(), sz3 = fetch();
+        uint4 sz0 = fetch(), sz1 = fetch(), sz2 = fetch(), sz3 = fetch();
         for (; cur_tile < args.ntiles; cur_tile += tile_step) {
             const TileCoord cc = tile_coord(args, cur_tile);
             const int nblocks = nkb + cc.nslab;
@@ -494,16 +532,45 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                     const unsigned char* qrow = st + kXBytes + kWBytes + row * 32;
                     const uint4 qa = *reinterpret_cast<const uint4*>(qrow + (hsw << 4));
                     const uint4 qb = *reinterpret_cast<const uint4*>(qrow + ((hsw ^ 1u) << 4));
-                    const uint32_t sz = sz0;                         // group i/2 (one block of it is ours)
+                    const uint4 sz = sz0;                            // group i/2 (one block of it is ours)
                     sz0 = sz1;
                     sz1 = sz2;
                     sz2 = sz3;
                     sz3 = fetch();
-                    const __half2 sc = __half2half2(__ushort_as_half((unsigned short)(sz & 0xffffu)));
-                    const __half2 bz = __half2half2(__ushort_as_half((unsigned short)(0x6400u | ((sz >> 16) & 0xffu))));
                     const uint32_t words[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
                     // row `row` of the W tile: 8 chunks of 16 B (8 fp16 in k order), chunk c at c ^ (row % 8)
                     unsigned char* wrow = st + kXBytes + (row >> 3) * 1024 + (row & 7) * 128;
+                    if constexpr (FMT != GLOWQ_FMT_INT4) {
+                        // this k-block is half (i & 1) of its group: 2 MXFP4 / 4 NVFP4 blocks;
+                        // word c holds k 8c .. 8c+7 (bytes = pairs in k order)
+                        const bool second = (i & 1) != 0;
+                        const uint32_t s01 = second ? (FMT == GLOWQ_FMT_MXFP4 ? sz.y : sz.z) : sz.x;
+                        const uint32_t s23 = second ? sz.w : sz.y;   // NVFP4 blocks 2, 3 of the half
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            uint32_t sb;
+                            if constexpr (FMT == GLOWQ_FMT_MXFP4) sb = (c < 4) ? (s01 & 0xffffu) : (s01 >> 16);
+                            else sb = (c < 2) ? (s01 & 0xffffu) : (c < 4) ? (s01 >> 16) : (c < 6) ? (s23 & 0xffffu) : (s23 >> 16);
+                            const __half2 sc = __half2half2(__ushort_as_half((unsigned short)sb));
+                            uint32_t pr[4];
+                            asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+                                "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+                                "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+                                "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+                                "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+                                "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+                                : "=r"(pr[0]), "=r"(pr[1]), "=r"(pr[2]), "=r"(pr[3])
+                                : "r"(words[c]));
+                            uint4 o;
+                            o.x = h2_as_u32(__hmul2(u32_as_h2(pr[0]), sc));
+                            o.y = h2_as_u32(__hmul2(u32_as_h2(pr[1]), sc));
+                            o.z = h2_as_u32(__hmul2(u32_as_h2(pr[2]), sc));
+                            o.w = h2_as_u32(__hmul2(u32_as_h2(pr[3]), sc));
+                            *reinterpret_cast<uint4*>(wrow + (((uint32_t)c ^ swz) << 4)) = o;
+                        }
+                    } else {
+                    const __half2 sc = __half2half2(__ushort_as_half((unsigned short)(sz.x & 0xffffu)));
+                    const __half2 bz = __half2half2(__ushort_as_half((unsigned short)(0x6400u | ((sz.x >> 16) & 0xffu))));
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         __half2 p[4];
@@ -516,6 +583,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                         o.w = pair_hi(u2, u3);   // (6,7)
                         *reinterpret_cast<uint4*>(wrow + (((uint32_t)c ^ swz) << 4)) = o;
                     }
+                    }   // INT4
                     fence_proxy_async_smem();   // generic-proxy writes visible to the tensor cores
                 }
                 // slab blocks are filled by TMA alone; they are still reported (after
@@ -801,7 +869,7 @@ static int gemm_max_pairs(int num_sms) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, (const void*)corrected_gemm_kernel, &cfg) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveClusters(&clusters, (const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4>, &cfg) != cudaSuccess ||
         clusters <= 0) {
         cudaGetLastError();
         clusters = num_sms / 2;
@@ -867,7 +935,7 @@ cudaError_t launch_rproj_prefill(const uint16_t* X, const uint16_t* B, int64_t T
 }
 
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r, const uint16_t* X,
-                                   int64_t T, uint16_t* R, float* partial, int num_sms, cudaStream_t st) {
+                                   int64_t T, uint16_t* R, float* partial, int num_sms, cudaStream_t st, int fmt) {
     if (T > ((int64_t)1 << 30)) return GLOWQ_ERR_SHAPE;
     if (!encode_fn()) return GLOWQ_ERR_CUDA;
     const bool use_r = r > 0 && B != nullptr;
@@ -876,8 +944,12 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     }
     static bool opted = false;
     if (!opted) {
-        if (cudaFuncSetAttribute((const void*)corrected_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)gemm_smem_bytes()) != cudaSuccess)
+        if (cudaFuncSetAttribute((const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes()) != cudaSuccess ||
+            cudaFuncSetAttribute((const void*)corrected_gemm_kernel<GLOWQ_FMT_MXFP4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes()) != cudaSuccess ||
+            cudaFuncSetAttribute((const void*)corrected_gemm_kernel<GLOWQ_FMT_NVFP4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes()) != cudaSuccess)
             return GLOWQ_ERR_CUDA;
         opted = true;
     }
@@ -899,8 +971,9 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
                                 (uint64_t)r * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B);
         ok = ok && make_map(&a->tmY[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, mv.Y, (uint64_t)mv.O, (uint64_t)T,
                             (uint64_t)mv.ldY * 2, kBM, kEpiChunk, CU_TENSOR_MAP_SWIZZLE_NONE);
-        a->mod[i].s = reinterpret_cast<const __half*>(mv.s);
+        a->mod[i].s = mv.s;
         a->mod[i].z = mv.z;
+        a->mod[i].ts = mv.ts;
         a->mod[i].Y = reinterpret_cast<__half*>(mv.Y);
         a->mod[i].ldY = mv.ldY;
         a->mod[i].O = (int)mv.O;
@@ -940,7 +1013,10 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = use_r ? 2 : 1;
-        e = cudaLaunchKernelExC(&cfg, (const void*)corrected_gemm_kernel, args);
+        const void* kfn = fmt == GLOWQ_FMT_MXFP4   ? (const void*)corrected_gemm_kernel<GLOWQ_FMT_MXFP4>
+                          : fmt == GLOWQ_FMT_NVFP4 ? (const void*)corrected_gemm_kernel<GLOWQ_FMT_NVFP4>
+                                                   : (const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4>;
+        e = cudaLaunchKernelExC(&cfg, kfn, args);
     }
     delete a;
     return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;

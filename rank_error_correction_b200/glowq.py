@@ -22,6 +22,9 @@ GROUP_SIZE = 128
 MAX_RANK = 256
 MAX_MODULES = 8
 
+FMT_INT4, FMT_MXFP4, FMT_NVFP4 = 0, 1, 2
+FP4_BLOCK = {FMT_MXFP4: 32, FMT_NVFP4: 16}
+
 STATUS = {0: "GLOWQ_OK", 1: "GLOWQ_ERR_ARG", 2: "GLOWQ_ERR_SHAPE", 3: "GLOWQ_ERR_ALIGN",
           4: "GLOWQ_ERR_CUDA", 5: "GLOWQ_ERR_TIMEOUT", 6: "GLOWQ_ERR_UNSUPPORTED"}
 
@@ -30,6 +33,11 @@ class GlowQError(RuntimeError):
     def __init__(self, code: int, what: str):
         self.code = code
         super().__init__(f"{what}: {STATUS.get(code, code)} ({_status_string(code)})")
+
+
+class _FP4Module(C.Structure):
+    _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("tensor_scale", C.c_void_p),
+                ("A", C.c_void_p), ("out_features", C.c_int64), ("Y", C.c_void_p), ("ldY", C.c_int64)]
 
 
 class _Module(C.Structure):
@@ -51,11 +59,15 @@ def lib() -> C.CDLL:
         p, i64, i32, st = C.c_void_p, C.c_int64, C.c_int32, C.c_int
         L.glowq_pack_int4.argtypes = [p, i64, i64, i32, p, p, p, p]
         L.glowq_dequant_int4.argtypes = [p, p, p, i64, i64, i32, p, p]
+        L.glowq_pack_fp4.argtypes = [st, p, i64, i64, p, p, p, p]
+        L.glowq_dequant_fp4.argtypes = [st, p, p, p, i64, i64, p, p]
         L.glowq_workspace_bytes.argtypes = [i64, i32]
         L.glowq_workspace_bytes.restype = C.c_size_t
         L.glowq_group_forward.argtypes = [C.POINTER(_Module), i32, i64, p, i32, p, i64, p, p, C.c_size_t, p]
         L.glowq_solo_forward.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p, C.c_size_t, p]
         L.glowq_solo_forward_noalloc.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p]
+        L.glowq_group_forward_fp4.argtypes = [st, C.POINTER(_FP4Module), i32, i64, p, i32, p, i64, p, p, C.c_size_t, p]
+        L.glowq_solo_forward_fp4.argtypes = [st, C.POINTER(_FP4Module), i64, p, i32, p, i64, p, C.c_size_t, p]
         L.glowq_noalloc_scratch_bytes.restype = C.c_size_t
         L.glowq_select_restore.argtypes = [p, p, p, p, i32, i32, p, p, p]
         L.glowq_select_restore_scores.argtypes = [p, p, p, i32, i32, p, p, p]
@@ -65,8 +77,8 @@ def lib() -> C.CDLL:
         L.glowq_status_string.argtypes = [st]
         L.glowq_status_string.restype = C.c_char_p
         L.glowq_version.restype = C.c_char_p
-        for f in ("glowq_pack_int4", "glowq_dequant_int4", "glowq_group_forward", "glowq_solo_forward",
-                  "glowq_solo_forward_noalloc",
+        for f in ("glowq_pack_int4", "glowq_dequant_int4", "glowq_pack_fp4", "glowq_dequant_fp4", "glowq_group_forward", "glowq_solo_forward",
+                  "glowq_solo_forward_noalloc", "glowq_group_forward_fp4", "glowq_solo_forward_fp4",
                   "glowq_select_restore", "glowq_select_restore_scores", "glowq_error_norms",
                   "glowq_get_device_status",
                   "glowq_selftest_wait_timeout"):
@@ -139,6 +151,33 @@ def dequant_int4(q, s, z, d: int, stream=None):
     out = torch.empty((O, d), dtype=torch.float16, device=q.device)
     _check(lib().glowq_dequant_int4(_ptr(q), _ptr(s), _ptr(z), O, d, GROUP_SIZE, _ptr(out), _stream(stream)),
            "glowq_dequant_int4")
+    return out
+
+
+def pack_fp4(W, fmt: int, stream=None):
+    """W (O x d fp32, CUDA) -> (codes int32 [O, d/8], scales uint8 [O, d/block], tensor_scale
+    float32 [1] for NVFP4 else None) in MXFP4 (fmt 1) or NVFP4 (fmt 2)."""
+    import torch
+    _require_cuda(W)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 tensor")
+    if fmt not in FP4_BLOCK:
+        raise ValueError("fmt must be FMT_MXFP4 or FMT_NVFP4")
+    O, d = W.shape
+    q = torch.empty((O, d // 8), dtype=torch.int32, device=W.device)
+    sc = torch.empty((O, d // FP4_BLOCK[fmt]), dtype=torch.uint8, device=W.device)
+    ts = torch.empty(1, dtype=torch.float32, device=W.device) if fmt == FMT_NVFP4 else None
+    _check(lib().glowq_pack_fp4(fmt, _ptr(W), O, d, _ptr(q), _ptr(sc), _ptr(ts), _stream(stream)), "glowq_pack_fp4")
+    return q, sc, ts
+
+
+def dequant_fp4(codes, scales, tensor_scale, d: int, fmt: int, stream=None):
+    import torch
+    _require_cuda(codes, scales, tensor_scale)
+    O = codes.shape[0]
+    out = torch.empty((O, d), dtype=torch.float16, device=codes.device)
+    _check(lib().glowq_dequant_fp4(fmt, _ptr(codes), _ptr(scales), _ptr(tensor_scale), O, d, _ptr(out),
+                                   _stream(stream)), "glowq_dequant_fp4")
     return out
 
 
@@ -248,6 +287,68 @@ def solo_forward(mod: QModule, B, X, Y=None, workspace=None, stream=None):
     ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().glowq_solo_forward(arr, d, _ptr(B), r, _ptr(X), T, _ptr(workspace), ws_n, _stream(stream)),
            "glowq_solo_forward")
+    return Y
+
+
+@dataclasses.dataclass
+class FP4Module:
+    """One MXFP4 / NVFP4 module: codes (int32 [O, d/8]), block scales (uint8),
+    tensor scale (float32 [1], NVFP4) and optional left factor A (O x r fp16)."""
+    fmt: int
+    codes: "object"
+    scales: "object"
+    tensor_scale: Optional["object"] = None
+    A: Optional["object"] = None
+
+    @property
+    def out_features(self) -> int:
+        return int(self.codes.shape[0])
+
+
+def _fp4_structs(mods: Sequence[FP4Module], Ys, use_A: bool):
+    items = []
+    for m, Y in zip(mods, Ys):
+        _require_cuda(m.codes, m.scales, m.tensor_scale, m.A)
+        items.append(_FP4Module(m.codes.data_ptr(), m.scales.data_ptr(), _ptr(m.tensor_scale),
+                                _ptr(m.A) if use_A else None, m.out_features, Y.data_ptr(), Y.stride(0)))
+    return (_FP4Module * len(items))(*items)
+
+
+def group_forward_fp4(mods: Sequence[FP4Module], B, X, Ys=None, R_out=None, workspace=None, stream=None):
+    """group_forward with MXFP4 / NVFP4 base weights (all modules of one format)."""
+    import torch
+    _require_cuda(B, X)
+    T, d = X.shape
+    r = 0 if B is None else int(B.shape[0])
+    fmt = mods[0].fmt
+    if any(m.fmt != fmt for m in mods):
+        raise ValueError("all modules of a group share one format")
+    if Ys is None:
+        Ys = [torch.empty((T, m.out_features), dtype=torch.float16, device=X.device) for m in mods]
+    if r > 0 and R_out is None:
+        R_out = torch.empty((T, r), dtype=torch.float16, device=X.device)
+    if workspace is None and r > 0:
+        workspace = alloc_workspace(T, r, X.device)
+    arr = _fp4_structs(mods, Ys, r > 0)
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().glowq_group_forward_fp4(fmt, arr, len(mods), d, _ptr(B), r, _ptr(X), T, _ptr(R_out),
+                                         _ptr(workspace), ws_n, _stream(stream)), "glowq_group_forward_fp4")
+    return Ys, R_out
+
+
+def solo_forward_fp4(mod: FP4Module, B, X, Y=None, workspace=None, stream=None):
+    import torch
+    _require_cuda(B, X)
+    T, d = X.shape
+    r = 0 if B is None else int(B.shape[0])
+    if Y is None:
+        Y = torch.empty((T, mod.out_features), dtype=torch.float16, device=X.device)
+    if workspace is None and r > 0:
+        workspace = alloc_workspace(T, r, X.device)
+    arr = _fp4_structs([mod], [Y], r > 0)
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().glowq_solo_forward_fp4(mod.fmt, arr, d, _ptr(B), r, _ptr(X), T, _ptr(workspace), ws_n,
+                                        _stream(stream)), "glowq_solo_forward_fp4")
     return Y
 
 

@@ -42,8 +42,9 @@ def test_workspace_bytes(L):
     assert glowq.workspace_bytes(0, 64) == 0
     assert glowq.workspace_bytes(16, 0) == 0
     small = glowq.workspace_bytes(16, 64)
-    assert small == 256 + 16 * 64 * 2                    # hand-off flags + solo R (decode reduces R on chip)
-    assert glowq.workspace_bytes(1, 64) == 256 + 256     # solo R rounded up to 256 B
+    # hand-off flags + up to 16 d-slices of fp32 partial sums of R + solo R
+    assert small == 256 + 16 * 16 * 64 * 4 + 16 * 64 * 2
+    assert glowq.workspace_bytes(1, 64) == 256 + 16 * 64 * 4 + 256     # solo R rounded up to 256 B
     big = glowq.workspace_bytes(2048, 64)
     assert big >= 256 + 8 * 2048 * 64 * 4 + 2048 * 64 * 2   # flags + split-d fp32 partials of R + solo R
     assert small % 256 == 0 and big % 256 == 0

@@ -296,7 +296,7 @@ def test_workspace_flags_shared_by_decode_prefill_and_solo_calls():
         Ys, R = glowq.group_forward(dev, Bd, Xd, workspace=ws)
         Yo = glowq.solo_forward(dev[1], Bd, Xd, workspace=ws)
         torch.cuda.synchronize()
-        assert int(ws[:12].view(torch.int32).abs().sum()) == 0, (T, ws[:12].tolist())
+        assert int(ws[:256].view(torch.int32).abs().sum()) == 0, (T, ws[:72].tolist())
         refs, R_ref = _oracle_group(mods, B, X)
         assert normwise(_np(R).astype(np.float64), R_ref) < 1e-3
         for y, ref in zip(Ys, refs):

@@ -139,3 +139,51 @@ def test_nvfp4_scales_error_bound_and_zero_tensor():
     assert scales[3, 1] == 0x7e
     cz, sz, stz = oracle.quantize_nvfp4(np.zeros((2, 32), np.float32))
     assert stz == 1.0 and np.all(cz == 0) and np.all(sz == 0)
+
+
+def _grid_weights(O, d, seed):
+    """Weights on the MXFP4 grid: every 32-block is E2M1 magnitudes times 2^k with
+    a 4 or 6 in it, so the block scale is 2^k and dequantisation is lossless."""
+    g = np.random.default_rng(seed)
+    mags = _e2m1_magnitudes()
+    W = np.zeros((O, d), np.float32)
+    for o in range(O):
+        for b in range(d // 32):
+            k = int(g.integers(-9, -3))
+            blk = g.choice(mags, 32) * g.choice([-1.0, 1.0], 32)
+            blk[int(g.integers(0, 32))] = g.choice([4.0, 6.0])
+            W[o, 32 * b:32 * b + 32] = blk * 2.0 ** k
+    return W
+
+
+def test_fp4_group_forward_is_the_definition():
+    """On the MXFP4 grid w_hat == W exactly, so the forward must equal X W^T + R A^T
+    computed directly from W (numpy float64, other association order), and the
+    shared R must equal each module's own projection."""
+    g = np.random.default_rng(5)
+    d, T, r = 256, 3, 8
+    Ws = [_grid_weights(O, d, 10 + i) for i, O in enumerate((64, 32))]
+    X = (g.standard_normal((T, d)) * 0.5).astype(np.float16)
+    B = (g.standard_normal((r, d)) * 0.05).astype(np.float16)
+    As = [(g.standard_normal((W.shape[0], r)) * 0.05).astype(np.float16) for W in Ws]
+    mods = []
+    for W, A in zip(Ws, As):
+        codes, scales = oracle.quantize_mxfp4(W)
+        mods.append((codes, scales, None, A.view(np.uint16)))
+    outs, R = oracle.fp4_group_forward("mx", mods, B.view(np.uint16), X.view(np.uint16))
+    Xd, Bd = X.astype(np.float64), B.astype(np.float64)
+    Rn = (Bd @ Xd.T).T
+    assert np.allclose(R, Rn, rtol=1e-13, atol=1e-15)
+    for W, A, Y in zip(Ws, As, outs):
+        want = (W.astype(np.float64) @ Xd.T).T + (A.astype(np.float64) @ Rn.T).T
+        assert np.allclose(Y, want, rtol=1e-12, atol=1e-14)
+    # NVFP4: the forward uses the NVFP4 dequantised weight (a different w_hat)
+    mods_nv = []
+    for W, A in zip(Ws, As):
+        codes, scales, st = oracle.quantize_nvfp4(W)
+        mods_nv.append((codes, scales, st, A.view(np.uint16)))
+    outs_nv, _ = oracle.fp4_group_forward("nv", mods_nv, B.view(np.uint16), X.view(np.uint16))
+    for (codes, scales, st, A), Y in zip(mods_nv, outs_nv):
+        Wh = _f16(oracle.dequant_nvfp4(codes, scales, st, d))
+        want = (Wh @ Xd.T).T + (A.view(np.float16).astype(np.float64) @ Rn.T).T
+        assert np.allclose(Y, want, rtol=1e-12, atol=1e-14)
