@@ -56,7 +56,8 @@ typedef enum glowq_status {
     GLOWQ_ERR_ALIGN = 3,        /* pointer or leading dimension misaligned  */
     GLOWQ_ERR_CUDA = 4,         /* CUDA runtime error while enqueueing      */
     GLOWQ_ERR_TIMEOUT = 5,      /* a device-side bounded wait ran out       */
-    GLOWQ_ERR_UNSUPPORTED = 6   /* valid request outside this build's scope */
+    GLOWQ_ERR_UNSUPPORTED = 6,  /* valid request outside this build's scope */
+    GLOWQ_ERR_NUMERIC = 7       /* a factorisation met a non-positive pivot  */
 } glowq_status;
 
 #define GLOWQ_GROUP_SIZE 128    /* INT4 quantisation group along d          */
@@ -253,6 +254,38 @@ GLOWQ_API glowq_status glowq_solo_forward_fp4(glowq_format fmt, const glowq_fp4_
                                               void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * W4A8: FP8 E4M3 activations (thelatestinai.com GlowQ page, Tables 14-15:
+ * GlowQ with 8-bit activations; the format is not defined there, a reading):
+ * each token t gets one fp32 scale s_t = amax_t / 448 (1 for an all-zero
+ * row) and codes E4M3(x / s_t), nearest with ties to even, saturating at 448,
+ * NaN -> 0x7f; the layer consumes x_hat = dec(code) s_t.
+ * glowq_quantize_act_e4m3: X (device, T x d fp16) -> codes (device, T x d
+ * bytes; may be NULL), scales (device, T floats), X_q (device, T x d fp16 of
+ * the exact code values dec(code), so x_hat = s_t X_q).
+ */
+GLOWQ_API glowq_status glowq_quantize_act_e4m3(const uint16_t* X, int64_t T, int64_t d, uint8_t* codes,
+                                               float* scales, uint16_t* X_q, void* stream);
+
+/* Device scratch of the W4A8 forward calls (it includes the forward workspace). */
+GLOWQ_API size_t glowq_w4a8_workspace_bytes(int64_t T, int64_t d, int32_t r);
+
+/*
+ * W4A8 group and solo forward with INT4 base weights: R = x_hat B^T and
+ * Y_i = x_hat w_hat_i^T + R A_i^T with x_hat the FP8 activations above.
+ * Computed exactly as s_t (X_q w_hat_i^T + X_q B^T A_i^T) on the fp16 tensor
+ * cores (X_q holds exact fp16 values), the per-token scale applied to the
+ * fp32 sums before the one rounding to fp16.  Arguments as for
+ * glowq_group_forward / glowq_solo_forward; X is the fp16 input (quantised
+ * inside the call); workspace of glowq_w4a8_workspace_bytes(T, d, r).
+ */
+GLOWQ_API glowq_status glowq_group_forward_w4a8(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B,
+                                                int32_t r, const uint16_t* X, int64_t T, uint16_t* R_out,
+                                                void* workspace, size_t workspace_bytes, void* stream);
+GLOWQ_API glowq_status glowq_solo_forward_w4a8(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r,
+                                               const uint16_t* X, int64_t T, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+
+/*
  * Solo module forward that allocates nothing (the GlowQ pages have no
  * counterpart: this is a deployment convenience of this library).
  *
@@ -286,6 +319,55 @@ GLOWQ_API glowq_status glowq_solo_forward_noalloc(const glowq_module* mod, int64
 
 /* Size of the fixed scratch array used by glowq_solo_forward_noalloc. */
 GLOWQ_API size_t glowq_noalloc_scratch_bytes(void);
+
+/*
+ * One module of a group for the offline solve: its fp32 weight and INT4 pack
+ * (device pointers, as produced by glowq_pack_int4).
+ */
+typedef struct glowq_solve_module {
+    const float* W;             /* O x d fp32 */
+    const uint32_t* qweight;    /* [O][d/8] */
+    const uint16_t* scales;     /* [O][d/128] fp16 bits */
+    const uint8_t* zeros;       /* [O][d/128] */
+    int64_t out_features;       /* O */
+} glowq_solve_module;
+
+/* Device scratch bytes glowq_group_solve needs for `rows` stacked rows (sum of
+   out_features), input dimension d, rank r and oversampling p. */
+GLOWQ_API size_t glowq_solve_workspace_bytes(int64_t rows, int64_t d, int32_t r, int32_t p);
+
+/*
+ * Offline whitened group solve on the GPU (papernotes.org summary, key
+ * designs 1-3; thelatestinai.com GlowQ page, Tables 11-12: randomised SVD of
+ * the covariance-aligned core with oversampling p and q power iterations).
+ * For the stacked error E_cat = [W_1 - w_hat_1; ...] (M = sum O_i rows):
+ *   E_w = E_cat Sx^{1/2};  Halko randomised SVD of E_w with the test matrix
+ *   Omega (d x (r+p)), orthonormalising after every product (Y = E_w Omega,
+ *   then q times E_w^T Q and E_w Z);  A = Q U_r S_r^{1/2} (M x r, the row
+ *   blocks are the A_i), B = S_r^{1/2} V_r^T Sx^{+1/2} (r x d);  the top r
+ *   singular values sigma_j of E_w; g_ec = sum_j sigma_j^2 / ||E_w||_F^2.
+ * E_w has the singular values and right vectors of the pages' thin-QR core
+ * M = R_e Sx^{1/2} (E_w = Q_e M), so the factors are the core's.  All
+ * arithmetic is float64 on the device.
+ *   mods, m        host array of 1..GLOWQ_MAX_MODULES modules
+ *   Sx_half        device, d x d float64 Sx^{1/2} (symmetric)
+ *   Sx_half_pinv   device, d x d float64 pseudo-inverse of Sx^{1/2}
+ *   r, p, q        rank (>= 1, r % 8 == 0), oversampling (even, r + p <= 112
+ *                  and <= min(M, d)), power iterations (0..16)
+ *   Omega          device, d x (r+p) float64 Gaussian test matrix (caller's draw)
+ *   A, B           device outputs, float64, M x r and r x d
+ *   sing, g_ec     device outputs, r doubles and one double (either may be NULL)
+ *   A16, B16       optional device outputs, the same factors rounded to fp16
+ *   workspace      device scratch of glowq_solve_workspace_bytes(M, d, r, p)
+ * Errors: GLOWQ_ERR_ARG / GLOWQ_ERR_SHAPE / GLOWQ_ERR_ALIGN before anything is
+ * enqueued; a non-positive Cholesky pivot while orthonormalising (a
+ * rank-deficient iterate) records GLOWQ_ERR_NUMERIC in the device status word.
+ */
+GLOWQ_API glowq_status glowq_group_solve(const glowq_solve_module* mods, int32_t m, int64_t d,
+                                         const double* Sx_half, const double* Sx_half_pinv, int32_t r, int32_t p,
+                                         int32_t q, const double* Omega, double* A, double* B, double* sing,
+                                         double* g_ec, uint16_t* A16, uint16_t* B16, void* workspace,
+                                         size_t workspace_bytes, void* stream);
 
 /*
  * GlowQ-S selective restore (key design 4; about half of the units restored
@@ -333,8 +415,8 @@ GLOWQ_API glowq_status glowq_error_norms(const float* W, const uint32_t* qweight
                                const uint16_t* scales, const uint8_t* zeros,
                                int64_t O, int64_t d, double* row_norms, void* stream);
 
-/* Reads and clears this device's status word (GLOWQ_OK or GLOWQ_ERR_TIMEOUT);
-   synchronises `stream` first. */
+/* Reads and clears this device's status word (GLOWQ_OK, GLOWQ_ERR_TIMEOUT or
+   GLOWQ_ERR_NUMERIC); synchronises `stream` first. */
 GLOWQ_API glowq_status glowq_get_device_status(void* stream);
 
 /*

@@ -25,7 +25,7 @@ LIB = os.path.join(PKG, "libglowq.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
               "-Xcompiler", "-fvisibility=hidden", f"-I{INCLUDE}", f"-I{CSRC}"]
-SOURCES = ["api.cu", "pack.cu", "fp4.cu", "decode.cu", "prefill.cu", "noalloc.cu", "select.cpp"]
+SOURCES = ["api.cu", "pack.cu", "fp4.cu", "decode.cu", "prefill.cu", "solve.cu", "noalloc.cu", "select.cpp"]
 HEADERS = ["common.cuh", "internal.cuh"]
 
 

@@ -91,9 +91,13 @@ glowq_status validate_solo_call(const glowq_module* mod, int64_t d, const uint16
     return validate_forward(mod, 1, d, B, r, X, T);
 }
 
+// R: the projection the kernels write and read; W4A8 (tok_scale != nullptr):
+// the decode kernels write R = fp16(s_t X' B^T) there, the prefill kernels
+// write the unscaled fp16(X' B^T) there for the GEMM and fp16(s_t X' B^T) to
+// R_scaled (when not null).
 static glowq_status forward_views(const ModuleView* hm, int32_t m, int64_t d, const uint16_t* B, int32_t r,
                                   const uint16_t* X, int64_t T, uint16_t* R, void* workspace, cudaStream_t st,
-                                  int fmt) {
+                                  int fmt, const float* tok_scale = nullptr, uint16_t* R_scaled = nullptr) {
     if (T == 0) return GLOWQ_OK;
     const bool use_r = r > 0;
     float* partial = (use_r && workspace_partial_bytes(T, r) > 0)
@@ -102,11 +106,11 @@ static glowq_status forward_views(const ModuleView* hm, int32_t m, int64_t d, co
     if (T <= kDecodeMaxTokens) {
         unsigned int* flags = use_r ? reinterpret_cast<unsigned int*>(workspace) : nullptr;
         cudaError_t e = launch_gemv_decode(hm, m, (int)d, (int)T, use_r ? r : 0, X, use_r ? B : nullptr, R, flags,
-                                           partial, device_sm_count(), st, fmt);
+                                           partial, device_sm_count(), st, fmt, tok_scale);
         return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
     }
     return prefill_group_forward(hm, m, (int)d, use_r ? B : nullptr, use_r ? r : 0, X, T, R, partial,
-                                 device_sm_count(), st, fmt);
+                                 device_sm_count(), st, fmt, tok_scale, use_r ? R_scaled : nullptr);
 }
 
 static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
@@ -159,6 +163,7 @@ const char* glowq_status_string(glowq_status s) {
         case GLOWQ_ERR_CUDA: return "CUDA error while enqueueing work";
         case GLOWQ_ERR_TIMEOUT: return "a device-side bounded wait ran out";
         case GLOWQ_ERR_UNSUPPORTED: return "request outside this build's scope";
+        case GLOWQ_ERR_NUMERIC: return "a factorisation met a non-positive pivot";
     }
     return "unknown status";
 }
@@ -305,6 +310,115 @@ glowq_status glowq_solo_forward_fp4(glowq_format fmt, const glowq_fp4_module* mo
                                         workspace_partial_bytes(T, r));
     }
     return forward_views(hm, 1, d, B, r, X, T, R, workspace, (cudaStream_t)stream, (int)fmt);
+}
+
+size_t glowq_solve_workspace_bytes(int64_t rows, int64_t d, int32_t r, int32_t p) {
+    if (rows <= 0 || d <= 0 || r <= 0 || p < 0) return 0;
+    return solve_workspace_bytes(rows, d, r + p);
+}
+
+glowq_status glowq_group_solve(const glowq_solve_module* mods, int32_t m, int64_t d, const double* Sx_half,
+                               const double* Sx_half_pinv, int32_t r, int32_t p, int32_t q, const double* Omega,
+                               double* A, double* B, double* sing, double* g_ec, uint16_t* A16, uint16_t* B16,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+    if (!mods || m < 1 || m > GLOWQ_MAX_MODULES || d <= 0 || r < 1 || p < 0 || q < 0 || q > 16) return GLOWQ_ERR_ARG;
+    if (!Sx_half || !Sx_half_pinv || !Omega || !A || !B || !workspace) return GLOWQ_ERR_ARG;
+    if (d % GLOWQ_GROUP_SIZE != 0 || r % 8 != 0 || p % 2 != 0 || r + p > 112) return GLOWQ_ERR_SHAPE;
+    SolveModule sm[GLOWQ_MAX_MODULES];
+    int64_t M = 0;
+    for (int i = 0; i < m; ++i) {
+        const glowq_solve_module& md = mods[i];
+        if (!md.W || !md.qweight || !md.scales || !md.zeros || md.out_features <= 0) return GLOWQ_ERR_ARG;
+        if ((reinterpret_cast<uintptr_t>(md.qweight) & 3u) || (reinterpret_cast<uintptr_t>(md.scales) & 1u) ||
+            (reinterpret_cast<uintptr_t>(md.W) & 3u))
+            return GLOWQ_ERR_ALIGN;
+        sm[i] = {md.W, md.qweight, md.scales, md.zeros, md.out_features};
+        M += md.out_features;
+    }
+    if (r + p > M || r + p > d) return GLOWQ_ERR_SHAPE;
+    const uintptr_t al8 = 7u;
+    if ((reinterpret_cast<uintptr_t>(Sx_half) & al8) || (reinterpret_cast<uintptr_t>(Sx_half_pinv) & al8) ||
+        (reinterpret_cast<uintptr_t>(Omega) & al8) || (reinterpret_cast<uintptr_t>(A) & al8) ||
+        (reinterpret_cast<uintptr_t>(B) & al8) || (sing && (reinterpret_cast<uintptr_t>(sing) & al8)) ||
+        (g_ec && (reinterpret_cast<uintptr_t>(g_ec) & al8)) || (A16 && (reinterpret_cast<uintptr_t>(A16) & 1u)) ||
+        (B16 && (reinterpret_cast<uintptr_t>(B16) & 1u)) || !aligned16(workspace))
+        return GLOWQ_ERR_ALIGN;
+    if (workspace_bytes < solve_workspace_bytes(M, d, r + p)) return GLOWQ_ERR_ARG;
+    return group_solve_impl(sm, m, d, Sx_half, Sx_half_pinv, r, p, q, Omega, A, B, sing, g_ec, A16, B16,
+                            workspace, device_status_ptr(), (cudaStream_t)stream);
+}
+
+glowq_status glowq_quantize_act_e4m3(const uint16_t* X, int64_t T, int64_t d, uint8_t* codes, float* scales,
+                                     uint16_t* X_q, void* stream) {
+    if (T < 0 || d < 0) return GLOWQ_ERR_ARG;
+    if (T == 0 || d == 0) return GLOWQ_OK;
+    if (!X || !scales || !X_q) return GLOWQ_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(X) & 1u) || (reinterpret_cast<uintptr_t>(X_q) & 1u) ||
+        (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return GLOWQ_ERR_ALIGN;
+    return launch_quantize_act_e4m3(X, T, d, codes, scales, X_q, (cudaStream_t)stream) == cudaSuccess
+               ? GLOWQ_OK
+               : GLOWQ_ERR_CUDA;
+}
+
+// W4A8 workspace: [forward workspace][X' T x d fp16][s_t T floats][R' T x r fp16]
+static size_t w4a8_xq_offset(int64_t T, int32_t r) { return align_up(glowq_workspace_bytes(T, r) + 16, 256); }
+static size_t w4a8_scale_offset(int64_t T, int64_t d, int32_t r) {
+    return w4a8_xq_offset(T, r) + align_up((size_t)T * d * 2, 256);
+}
+static size_t w4a8_rprime_offset(int64_t T, int64_t d, int32_t r) {
+    return w4a8_scale_offset(T, d, r) + align_up((size_t)T * 4, 256);
+}
+
+size_t glowq_w4a8_workspace_bytes(int64_t T, int64_t d, int32_t r) {
+    if (T <= 0 || d <= 0 || r < 0) return 0;
+    return w4a8_rprime_offset(T, d, r) + align_up((size_t)T * (size_t)r * 2, 256);
+}
+
+static glowq_status w4a8_impl(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
+                              const uint16_t* X, int64_t T, uint16_t* R_out, void* workspace, size_t workspace_bytes,
+                              cudaStream_t st, bool solo) {
+    glowq_status v = validate_forward(mods, m, d, B, r, X, T);
+    if (v != GLOWQ_OK) return v;
+    if (T == 0) return GLOWQ_OK;
+    if (!solo && r > 0) {
+        if (!R_out) return GLOWQ_ERR_ARG;
+        if (!aligned16(R_out)) return GLOWQ_ERR_ALIGN;
+    }
+    if (!workspace || workspace_bytes < glowq_w4a8_workspace_bytes(T, d, r)) return GLOWQ_ERR_ARG;
+    if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
+    char* ws = static_cast<char*>(workspace);
+    uint16_t* Xq = reinterpret_cast<uint16_t*>(ws + w4a8_xq_offset(T, r));
+    float* ts = reinterpret_cast<float*>(ws + w4a8_scale_offset(T, d, r));
+    uint16_t* Rp = reinterpret_cast<uint16_t*>(ws + w4a8_rprime_offset(T, d, r));
+    if (launch_quantize_act_e4m3(X, T, d, nullptr, ts, Xq, st) != cudaSuccess) return GLOWQ_ERR_CUDA;
+    ModuleView hm[GLOWQ_MAX_MODULES];
+    for (int i = 0; i < m; ++i)
+        hm[i] = {mods[i].qweight, mods[i].scales, mods[i].zeros, nullptr, (r > 0) ? mods[i].A : nullptr,
+                 mods[i].Y, mods[i].ldY, mods[i].out_features};
+    uint16_t* Rsolo = r > 0 ? reinterpret_cast<uint16_t*>(ws + workspace_flag_bytes(r) + workspace_partial_bytes(T, r))
+                            : nullptr;
+    uint16_t* R;
+    uint16_t* Rs = nullptr;
+    if (T <= kDecodeMaxTokens) {
+        R = solo ? Rsolo : R_out;          // the decode kernels write the scaled R
+    } else {
+        R = solo ? Rsolo : Rp;             // the GEMM reads the unscaled R'
+        Rs = solo ? nullptr : R_out;
+    }
+    return forward_views(hm, m, d, B, r, Xq, T, R, workspace, st, GLOWQ_FMT_INT4, ts, Rs);
+}
+
+glowq_status glowq_group_forward_w4a8(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
+                                      const uint16_t* X, int64_t T, uint16_t* R_out, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+    return w4a8_impl(mods, m, d, B, r, X, T, R_out, workspace, workspace_bytes, (cudaStream_t)stream, false);
+}
+
+glowq_status glowq_solo_forward_w4a8(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r,
+                                     const uint16_t* X, int64_t T, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+    return w4a8_impl(mod, 1, d, B, r, X, T, nullptr, workspace, workspace_bytes, (cudaStream_t)stream, true);
 }
 
 glowq_status glowq_selftest_wait_timeout(uint32_t polls, void* stream) {

@@ -131,6 +131,7 @@ struct GemvArgs {
     int rsub;          // sub-slices of each cluster rank's slice of d (kc * rsub <= kRMaxSlices)
     int rpre;          // 1: R was computed by the preceding launch (rproj_decode_kernel)
     int stages;        // weight-ring stages per warp (4 or 8)
+    const float* tok_scale;   // W4A8: per-token scale s_t of X = s_t X' (nullptr: none)
     unsigned int* flags;    // hand-off words (r > 0), see above
     unsigned int* status;   // device status word (bounded-wait timeouts)
 };
@@ -322,6 +323,10 @@ __device__ __forceinline__ void rproj_reduce(const GemvArgs& a, int rb, int S, i
                         v.x += p8[u].x; v.y += p8[u].y; v.z += p8[u].z; v.w += p8[u].w;
                     }
                 }
+        }
+        if (a.tok_scale) {   // W4A8: R = s_t X' B^T
+            const float ts = a.tok_scale[tok];
+            v.x *= ts; v.y *= ts; v.z *= ts; v.w *= ts;
         }
         __half2 h01 = __floats2half2_rn(v.x, v.y), h23 = __floats2half2_rn(v.z, v.w);
         uint2 pk;
@@ -1029,6 +1034,19 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     }
     if (!active) return;
 
+    // W4A8: the per-token scale s_t of the base product (R is already s_t X' B^T)
+    if (args.tok_scale) {
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int tk = n * 8 + 2 * t;
+            const float s0 = (tk < T) ? __ldg(args.tok_scale + tk) : 0.f;
+            const float s1 = (tk + 1 < T) ? __ldg(args.tok_scale + tk + 1) : 0.f;
+            acc[n][0] *= s0;
+            acc[n][1] *= s1;
+            acc[n][2] *= s0;
+            acc[n][3] *= s1;
+        }
+    }
     // NVFP4: the fp32 tensor scale of the base product
     if constexpr (FMT == GLOWQ_FMT_NVFP4) {
         const float st = __ldg(M.ts);
@@ -1223,7 +1241,7 @@ static GemvShape choose_shape_b(int tiles, int d, int T, int r, int nt, int num_
 
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
                                const uint16_t* B, uint16_t* R, unsigned int* flags, float* partial, int num_sms,
-                               cudaStream_t st, int fmt) {
+                               cudaStream_t st, int fmt, const float* tok_scale) {
     GemvArgs a = {};
     int tiles = 0;
     for (int i = 0; i < m; ++i) {
@@ -1306,6 +1324,7 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     // A grid larger than one wave gets R from a separate launch first: its
     // CTAs must not wait on producers that may not be resident.
     a.rpre = (r > 0 && grid > sh.res) ? 1 : 0;
+    a.tok_scale = tok_scale;
     a.stages = sh.stages;
     if (a.rpre) {
         int S = ngroups / 4;

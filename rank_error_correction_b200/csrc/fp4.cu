@@ -188,6 +188,61 @@ __global__ void __launch_bounds__(256) dequant_fp4_kernel(int fmt, const uint32_
     *reinterpret_cast<uint4*>(out + o * d + k0) = *reinterpret_cast<const uint4*>(h);
 }
 
+// ---------------------------------------------------------------------------
+// W4A8 activations (thelatestinai.com GlowQ page, Tables 14-15: GlowQ with
+// FP8 activations): per token t, s_t = amax_t / 448 (1 for an all-zero row)
+// and codes E4M3(x / s_t), nearest, ties to even, saturating at 448, NaN ->
+// 0x7f; a value that rounds to zero keeps code 0 whatever its sign.  One CTA
+// per token.  Writes the codes (optional), s_t, and the exact code values as
+// fp16 (X' = x_hat / s_t, so that x_hat = s_t X').
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3_encode(float v) {
+    if (!(v == v)) return 0x7fu;
+    const uint32_t c = e4m3_encode_nonneg(fabsf(v));
+    return (c != 0u && v < 0.0f) ? (c | 0x80u) : c;
+}
+
+__global__ void __launch_bounds__(256) quantize_act_e4m3_kernel(const __half* __restrict__ X, int64_t d,
+                                                                 uint8_t* __restrict__ codes, float* __restrict__ scales,
+                                                                 __half* __restrict__ Xq) {
+    __shared__ float wmax[8];
+    const int64_t t = blockIdx.x;
+    const __half* x = X + t * d;
+    float amax = 0.0f;
+    for (int64_t k = threadIdx.x; k < d; k += blockDim.x) {
+        const float a = fabsf(__half2float(x[k]));
+        if (a > amax) amax = a;                       // NaN never compares greater
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float b = __shfl_xor_sync(0xffffffffu, amax, o);
+        if (b > amax) amax = b;
+    }
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+    __syncthreads();
+    amax = 0.0f;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w)
+        if (wmax[w] > amax) amax = wmax[w];
+    float s = __fdiv_rn(amax, 448.0f);
+    if (!(s > 0.0f)) s = 1.0f;
+    if (threadIdx.x == 0) scales[t] = s;
+    for (int64_t k = threadIdx.x; k < d; k += blockDim.x) {
+        const uint32_t c = e4m3_encode(__fdiv_rn(__half2float(x[k]), s));
+        if (codes) codes[t * d + k] = (uint8_t)c;
+        // exact: E4M3 values are fp16 values (the NaN codes stay NaN)
+        Xq[t * d + k] = ((c & 0x7fu) == 0x7fu) ? __ushort_as_half((unsigned short)0x7e00u)
+                                               : __float2half_rn(e4m3_value(c));
+    }
+}
+
+cudaError_t launch_quantize_act_e4m3(const uint16_t* X, int64_t T, int64_t d, uint8_t* codes, float* scales,
+                                     uint16_t* Xq, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    quantize_act_e4m3_kernel<<<(unsigned)T, 256, 0, st>>>(reinterpret_cast<const __half*>(X), d, codes, scales,
+                                                           reinterpret_cast<__half*>(Xq));
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pack_fp4(int fmt, const float* W, int64_t O, int64_t d, uint32_t* codes, uint8_t* scales,
                             float* tensor_scale, cudaStream_t st) {
     const int64_t units = O * (d / 128);

@@ -38,7 +38,7 @@ unsigned int* device_status_ptr();
 // every completed call leaves zero.
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
                                const uint16_t* B, uint16_t* R, unsigned int* flags, float* partial, int num_sms,
-                               cudaStream_t st, int fmt = GLOWQ_FMT_INT4);
+                               cudaStream_t st, int fmt = GLOWQ_FMT_INT4, const float* tok_scale = nullptr);
 size_t decode_partial_bytes(int64_t T, int r);
 // pack.cu
 cudaError_t launch_pack_int4(const float* W, int64_t O, int64_t d, uint32_t* q, uint16_t* s, uint8_t* z,
@@ -48,10 +48,25 @@ cudaError_t launch_dequant_int4(const uint32_t* q, const uint16_t* s, const uint
 cudaError_t launch_error_norms(const float* W, const uint32_t* q, const uint16_t* s, const uint8_t* z,
                                int64_t O, int64_t d, double* out_rows, cudaStream_t st);
 // fp4.cu
+cudaError_t launch_quantize_act_e4m3(const uint16_t* X, int64_t T, int64_t d, uint8_t* codes, float* scales,
+                                     uint16_t* Xq, cudaStream_t st);
 cudaError_t launch_pack_fp4(int fmt, const float* W, int64_t O, int64_t d, uint32_t* codes, uint8_t* scales,
                             float* tensor_scale, cudaStream_t st);
 cudaError_t launch_dequant_fp4(int fmt, const uint32_t* codes, const uint8_t* scales, const float* tensor_scale,
                                int64_t O, int64_t d, uint16_t* out, cudaStream_t st);
+// solve.cu: the offline group solve (float64)
+struct SolveModule {
+    const float* W;      // O x d fp32 weights
+    const uint32_t* q;   // INT4 packed codes
+    const uint16_t* s;   // fp16 scales
+    const uint8_t* z;    // zeros
+    int64_t O;
+};
+size_t solve_workspace_bytes(int64_t M, int64_t d, int l);
+glowq_status group_solve_impl(const SolveModule* mods, int m, int64_t d, const double* Sh, const double* Shp,
+                              int r, int p, int qit, const double* Omega, double* A, double* B, double* sing,
+                              double* gec, uint16_t* A16, uint16_t* B16, void* workspace, unsigned int* err,
+                              cudaStream_t st);
 // prefill.cu: TMA tensor maps (driver entry point resolved at run time)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -64,7 +79,8 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
 // (nullptr: one slice of d per CTA, R written directly).
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r,
                                    const uint16_t* X, int64_t T, uint16_t* R, float* partial, int num_sms,
-                                   cudaStream_t st, int fmt = GLOWQ_FMT_INT4);
+                                   cudaStream_t st, int fmt = GLOWQ_FMT_INT4, const float* tok_scale = nullptr,
+                                   uint16_t* R_scaled = nullptr);
 size_t prefill_partial_bytes(int64_t T, int r);
 
 }  // namespace glowq

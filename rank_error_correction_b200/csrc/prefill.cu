@@ -192,6 +192,7 @@ struct PrefillArgs {
     int ntiles_n;                          // token tiles
     int ntiles;                            // all pair tiles
     int wait_dep;                          // R comes from the preceding (PDL) kernel
+    const float* tok_scale;                // W4A8: per-token scale s_t of the outputs (nullptr: none)
     unsigned int* status;
 };
 
@@ -619,8 +620,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                 if (leader) bulk_wait_read<kEpiBufs - 1>();   // the store from this buffer is done reading
                 named_barrier_sync(1, kEpiThreads);
                 __half* col = reinterpret_cast<__half*>(sb) + row;
+                if (args.tok_scale) {   // W4A8: y = s_t (X' w_hat^T + R' A^T), one rounding
+                    const int t0 = c.n0 + ch * kEpiChunk;
 #pragma unroll
-                for (int j = 0; j < 32; ++j) col[j * kBM] = __float2half_rn(__uint_as_float(v[j]));
+                    for (int j = 0; j < 32; ++j) {
+                        const float ts = (t0 + j < args.T) ? __ldg(args.tok_scale + t0 + j) : 0.f;
+                        col[j * kBM] = __float2half_rn(__uint_as_float(v[j]) * ts);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) col[j * kBM] = __float2half_rn(__uint_as_float(v[j]));
+                }
                 fence_proxy_async_smem();
                 named_barrier_sync(1, kEpiThreads);
                 const int tok0 = c.n0 + ch * kEpiChunk;
@@ -658,6 +668,8 @@ struct RprojArgs {
     CUtensorMap tmX;   // X [T][d], box {64, 128}, SW128
     CUtensorMap tmB;   // B [r][d], box {64, rn}, SW128
     __half* R;         // T x r (chunks == 1)
+    const float* tok_scale;   // W4A8: also write R_scaled = fp16(s_t R) (nullptr: none)
+    __half* R_scaled;
     float* partial;    // chunks x T x r (chunks > 1)
     int d, T, r, rn, chunks;
     unsigned int* status;
@@ -772,6 +784,14 @@ __global__ void __launch_bounds__(kRThreads, 1) rproj_tc_kernel(const __grid_con
                         o.z = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j + 4]), __uint_as_float(v[j + 5])));
                         o.w = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j + 6]), __uint_as_float(v[j + 7])));
                         *reinterpret_cast<uint4*>(dst + j) = o;
+                        if (args.R_scaled) {
+                            const float ts = args.tok_scale[tok];
+                            o.x = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j]) * ts, __uint_as_float(v[j + 1]) * ts));
+                            o.y = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j + 2]) * ts, __uint_as_float(v[j + 3]) * ts));
+                            o.z = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j + 4]) * ts, __uint_as_float(v[j + 5]) * ts));
+                            o.w = h2_as_u32(__floats2half2_rn(__uint_as_float(v[j + 6]) * ts, __uint_as_float(v[j + 7]) * ts));
+                            *reinterpret_cast<uint4*>(args.R_scaled + (int64_t)tok * r + c + j) = o;
+                        }
                     }
                 }
             }
@@ -784,7 +804,8 @@ __global__ void __launch_bounds__(kRThreads, 1) rproj_tc_kernel(const __grid_con
 
 // R[i] = fp16_RN(sum_y partial[y][i]) in ascending y, four elements per thread.
 __global__ void __launch_bounds__(256) rproj_sum_kernel(const float4* __restrict__ partial, int chunks, int n4,
-                                                         uint2* __restrict__ R) {
+                                                         uint2* __restrict__ R, const float* __restrict__ tok_scale,
+                                                         uint2* __restrict__ R_scaled, int r) {
     pdl_launch_dependents();
     pdl_wait();                 // partial sums complete
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
@@ -804,6 +825,12 @@ __global__ void __launch_bounds__(256) rproj_sum_kernel(const float4* __restrict
     o.x = h2_as_u32(__floats2half2_rn(acc.x, acc.y));
     o.y = h2_as_u32(__floats2half2_rn(acc.z, acc.w));
     R[i] = o;
+    if (R_scaled) {   // W4A8: fp16(s_t R) for the caller
+        const float ts = tok_scale[(4 * i) / r];
+        o.x = h2_as_u32(__floats2half2_rn(acc.x * ts, acc.y * ts));
+        o.y = h2_as_u32(__floats2half2_rn(acc.z * ts, acc.w * ts));
+        R_scaled[i] = o;
+    }
 }
 
 // Number of d slices of the prefill R projection: enough CTAs to cover the
@@ -897,7 +924,8 @@ static cudaError_t launch_with(const void* fn, dim3 grid, dim3 block, size_t sme
 }
 
 cudaError_t launch_rproj_prefill(const uint16_t* X, const uint16_t* B, int64_t T, int d, int r, uint16_t* R,
-                                 float* partial, int num_sms, cudaStream_t st) {
+                                 float* partial, int num_sms, cudaStream_t st, const float* tok_scale,
+                                 uint16_t* R_scaled) {
     static bool opted = false;
     if (!opted) {
         cudaError_t e = cudaFuncSetAttribute((const void*)rproj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -916,6 +944,8 @@ cudaError_t launch_rproj_prefill(const uint16_t* X, const uint16_t* B, int64_t T
         return cudaErrorInvalidValue;
     const int chunks = partial ? prefill_r_chunks(T, d, num_sms) : 1;
     a.R = reinterpret_cast<__half*>(R);
+    a.tok_scale = tok_scale;
+    a.R_scaled = reinterpret_cast<__half*>(R_scaled);
     a.partial = partial;
     a.d = d;
     a.T = (int)T;
@@ -930,17 +960,20 @@ cudaError_t launch_rproj_prefill(const uint16_t* X, const uint16_t* B, int64_t T
     const float4* p4 = reinterpret_cast<const float4*>(partial);
     const int n4 = (int)(T * r / 4);
     uint2* R4 = reinterpret_cast<uint2*>(R);
-    void* a2[] = {(void*)&p4, (void*)&chunks, (void*)&n4, (void*)&R4};
+    uint2* RS4 = reinterpret_cast<uint2*>(R_scaled);
+    void* a2[] = {(void*)&p4, (void*)&chunks, (void*)&n4, (void*)&R4, (void*)&tok_scale, (void*)&RS4, (void*)&r};
     return launch_with((const void*)rproj_sum_kernel, dim3((unsigned)((n4 + 255) / 256)), dim3(256), 0, st, true, a2);
 }
 
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r, const uint16_t* X,
-                                   int64_t T, uint16_t* R, float* partial, int num_sms, cudaStream_t st, int fmt) {
+                                   int64_t T, uint16_t* R, float* partial, int num_sms, cudaStream_t st, int fmt,
+                                   const float* tok_scale, uint16_t* R_scaled) {
     if (T > ((int64_t)1 << 30)) return GLOWQ_ERR_SHAPE;
     if (!encode_fn()) return GLOWQ_ERR_CUDA;
     const bool use_r = r > 0 && B != nullptr;
     if (use_r) {
-        if (launch_rproj_prefill(X, B, T, d, r, R, partial, num_sms, st) != cudaSuccess) return GLOWQ_ERR_CUDA;
+        if (launch_rproj_prefill(X, B, T, d, r, R, partial, num_sms, st, tok_scale, R_scaled) != cudaSuccess)
+            return GLOWQ_ERR_CUDA;
     }
     static bool opted = false;
     if (!opted) {
@@ -991,6 +1024,7 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     a->r = use_r ? r : 0;
     a->ntiles_n = (int)((T + kBN - 1) / kBN);
     a->wait_dep = use_r ? 1 : 0;
+    a->tok_scale = tok_scale;
     a->status = device_status_ptr();
     const int64_t ntiles = (int64_t)mtiles * a->ntiles_n;
     a->ntiles = (int)ntiles;

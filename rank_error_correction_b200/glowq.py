@@ -26,7 +26,7 @@ FMT_INT4, FMT_MXFP4, FMT_NVFP4 = 0, 1, 2
 FP4_BLOCK = {FMT_MXFP4: 32, FMT_NVFP4: 16}
 
 STATUS = {0: "GLOWQ_OK", 1: "GLOWQ_ERR_ARG", 2: "GLOWQ_ERR_SHAPE", 3: "GLOWQ_ERR_ALIGN",
-          4: "GLOWQ_ERR_CUDA", 5: "GLOWQ_ERR_TIMEOUT", 6: "GLOWQ_ERR_UNSUPPORTED"}
+          4: "GLOWQ_ERR_CUDA", 5: "GLOWQ_ERR_TIMEOUT", 6: "GLOWQ_ERR_UNSUPPORTED", 7: "GLOWQ_ERR_NUMERIC"}
 
 
 class GlowQError(RuntimeError):
@@ -38,6 +38,11 @@ class GlowQError(RuntimeError):
 class _FP4Module(C.Structure):
     _fields_ = [("codes", C.c_void_p), ("scales", C.c_void_p), ("tensor_scale", C.c_void_p),
                 ("A", C.c_void_p), ("out_features", C.c_int64), ("Y", C.c_void_p), ("ldY", C.c_int64)]
+
+
+class _SolveModule(C.Structure):
+    _fields_ = [("W", C.c_void_p), ("qweight", C.c_void_p), ("scales", C.c_void_p), ("zeros", C.c_void_p),
+                ("out_features", C.c_int64)]
 
 
 class _Module(C.Structure):
@@ -70,6 +75,15 @@ def lib() -> C.CDLL:
         L.glowq_solo_forward_fp4.argtypes = [st, C.POINTER(_FP4Module), i64, p, i32, p, i64, p, C.c_size_t, p]
         L.glowq_noalloc_scratch_bytes.restype = C.c_size_t
         L.glowq_select_restore.argtypes = [p, p, p, p, i32, i32, p, p, p]
+        L.glowq_quantize_act_e4m3.argtypes = [p, i64, i64, p, p, p, p]
+        L.glowq_w4a8_workspace_bytes.argtypes = [i64, i64, i32]
+        L.glowq_w4a8_workspace_bytes.restype = C.c_size_t
+        L.glowq_group_forward_w4a8.argtypes = [C.POINTER(_Module), i32, i64, p, i32, p, i64, p, p, C.c_size_t, p]
+        L.glowq_solo_forward_w4a8.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p, C.c_size_t, p]
+        L.glowq_solve_workspace_bytes.argtypes = [i64, i64, i32, i32]
+        L.glowq_solve_workspace_bytes.restype = C.c_size_t
+        L.glowq_group_solve.argtypes = [C.POINTER(_SolveModule), i32, i64, p, p, i32, i32, i32, p, p, p, p, p, p, p,
+                                        p, C.c_size_t, p]
         L.glowq_select_restore_scores.argtypes = [p, p, p, i32, i32, p, p, p]
         L.glowq_error_norms.argtypes = [p, p, p, p, i64, i64, p, p]
         L.glowq_get_device_status.argtypes = [p]
@@ -79,7 +93,8 @@ def lib() -> C.CDLL:
         L.glowq_version.restype = C.c_char_p
         for f in ("glowq_pack_int4", "glowq_dequant_int4", "glowq_pack_fp4", "glowq_dequant_fp4", "glowq_group_forward", "glowq_solo_forward",
                   "glowq_solo_forward_noalloc", "glowq_group_forward_fp4", "glowq_solo_forward_fp4",
-                  "glowq_select_restore", "glowq_select_restore_scores", "glowq_error_norms",
+                  "glowq_select_restore", "glowq_select_restore_scores", "glowq_error_norms", "glowq_group_solve",
+                  "glowq_quantize_act_e4m3", "glowq_group_forward_w4a8", "glowq_solo_forward_w4a8",
                   "glowq_get_device_status",
                   "glowq_selftest_wait_timeout"):
             getattr(L, f).restype = st
@@ -381,6 +396,99 @@ def device_status(stream=None) -> int:
 def selftest_wait_timeout(polls: int = 4096, stream=None) -> None:
     """Enqueues the failure-path self-test (a bounded wait that must run out)."""
     _check(lib().glowq_selftest_wait_timeout(int(polls), _stream(stream)), "glowq_selftest_wait_timeout")
+
+
+# ------------------------------------------------------------------- W4A8 ----
+
+def quantize_act_e4m3(X, stream=None):
+    """Per-token FP8 E4M3 activations: X (T x d fp16, CUDA) -> (codes uint8 [T, d],
+    scales float32 [T], X_q fp16 [T, d] exact code values; x_hat = scales[:, None] * X_q)."""
+    import torch
+    _require_cuda(X)
+    T, d = X.shape
+    codes = torch.empty((T, d), dtype=torch.uint8, device=X.device)
+    scales = torch.empty(T, dtype=torch.float32, device=X.device)
+    Xq = torch.empty((T, d), dtype=torch.float16, device=X.device)
+    _check(lib().glowq_quantize_act_e4m3(_ptr(X), T, d, _ptr(codes), _ptr(scales), _ptr(Xq), _stream(stream)),
+           "glowq_quantize_act_e4m3")
+    return codes, scales, Xq
+
+
+def w4a8_workspace(T: int, d: int, r: int, device="cuda"):
+    import torch
+    n = max(int(lib().glowq_w4a8_workspace_bytes(T, d, r)), 16)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def group_forward_w4a8(mods: Sequence[QModule], B, X, Ys=None, R_out=None, workspace=None, stream=None):
+    """group_forward with FP8 (E4M3, per-token scale) activations; X is fp16 and
+    is quantised inside the call."""
+    import torch
+    _require_cuda(B, X)
+    T, d = X.shape
+    r = 0 if B is None else int(B.shape[0])
+    if Ys is None:
+        Ys = [torch.empty((T, m.out_features), dtype=torch.float16, device=X.device) for m in mods]
+    if r > 0 and R_out is None:
+        R_out = torch.empty((T, r), dtype=torch.float16, device=X.device)
+    if workspace is None:
+        workspace = w4a8_workspace(T, d, r, X.device)
+    arr = _module_structs(mods, Ys, r > 0)
+    ws_n = workspace.numel() * workspace.element_size()
+    _check(lib().glowq_group_forward_w4a8(arr, len(mods), d, _ptr(B), r, _ptr(X), T, _ptr(R_out), _ptr(workspace),
+                                          ws_n, _stream(stream)), "glowq_group_forward_w4a8")
+    return Ys, R_out
+
+
+def solo_forward_w4a8(mod: QModule, B, X, Y=None, workspace=None, stream=None):
+    import torch
+    _require_cuda(B, X)
+    T, d = X.shape
+    r = 0 if B is None else int(B.shape[0])
+    if Y is None:
+        Y = torch.empty((T, mod.out_features), dtype=torch.float16, device=X.device)
+    if workspace is None:
+        workspace = w4a8_workspace(T, d, r, X.device)
+    arr = _module_structs([mod], [Y], r > 0)
+    ws_n = workspace.numel() * workspace.element_size()
+    _check(lib().glowq_solo_forward_w4a8(arr, d, _ptr(B), r, _ptr(X), T, _ptr(workspace), ws_n, _stream(stream)),
+           "glowq_solo_forward_w4a8")
+    return Y
+
+
+# ---------------------------------------------------------- offline solve ----
+
+def solve_workspace_bytes(rows: int, d: int, r: int, p: int) -> int:
+    return int(lib().glowq_solve_workspace_bytes(rows, d, r, p))
+
+
+def group_solve(Ws, packs, Sx_half, Sx_half_pinv, r: int, p: int, q: int, Omega, fp16=True, stream=None):
+    """Whitened shared-B solve on the GPU for one group.  Ws: fp32 weights
+    (O_i x d); packs: (qweight, scales, zeros) of each; Sx_half, Sx_half_pinv:
+    d x d float64; Omega: d x (r+p) float64.  All CUDA tensors.  Returns
+    (A float64 [M, r], B float64 [r, d], sing float64 [r], g_ec float64 [1],
+    A16, B16 fp16 or None)."""
+    import torch
+    d = int(Ws[0].shape[1])
+    M = sum(int(W.shape[0]) for W in Ws)
+    dev = Ws[0].device
+    for t in (*Ws, Sx_half, Sx_half_pinv, Omega):
+        _require_cuda(t)
+    items = [_SolveModule(W.data_ptr(), q_.data_ptr(), s_.data_ptr(), z_.data_ptr(), int(W.shape[0]))
+             for W, (q_, s_, z_) in zip(Ws, packs)]
+    arr = (_SolveModule * len(items))(*items)
+    A = torch.empty((M, r), dtype=torch.float64, device=dev)
+    B = torch.empty((r, d), dtype=torch.float64, device=dev)
+    sing = torch.empty(r, dtype=torch.float64, device=dev)
+    gec = torch.empty(1, dtype=torch.float64, device=dev)
+    A16 = torch.empty((M, r), dtype=torch.float16, device=dev) if fp16 else None
+    B16 = torch.empty((r, d), dtype=torch.float16, device=dev) if fp16 else None
+    nws = max(solve_workspace_bytes(M, d, r, p), 16)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    _check(lib().glowq_group_solve(arr, len(items), d, _ptr(Sx_half), _ptr(Sx_half_pinv), r, p, q, _ptr(Omega),
+                                   _ptr(A), _ptr(B), _ptr(sing), _ptr(gec), _ptr(A16), _ptr(B16), _ptr(ws), nws,
+                                   _stream(stream)), "glowq_group_solve")
+    return A, B, sing, gec, A16, B16
 
 
 # ---------------------------------------------------------------- GlowQ-S ----
