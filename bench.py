@@ -761,6 +761,49 @@ def unit_lines(shapes, tokens, device, hbm_peak, tf_peak, seed=0, sub0=0, ranks=
     return out
 
 
+# ----------------------------------------------------- offline solve (GPU)
+
+def solve_line(device, r=64, p=16, q=2, seed=0):
+    """The offline whitened group solve on the GPU for one LLaMA-2-7B Q/K/V
+    group (3 x 4096 x 4096, r = 64, p = 16, q = 2), float64.  Context: the
+    pages' Table 11 times the randomised SVD of the covariance-aligned core
+    per layer on an A100.  Synthetic inputs: random-init weights and a
+    diagonal power-law Sx^{1/2} (alpha = 1.19) stored dense."""
+    import torch
+    from rank_error_correction_b200 import glowq, synth
+    d, outs = D, QKV_OUTS
+    Ws, packs = [], []
+    for j, O in enumerate(outs):
+        W = synth.device_weights(O, d, seed, sub=7000 + j, device=device)
+        Ws.append(W)
+        packs.append(glowq.pack_int4(W))
+    lam = torch.from_numpy(synth.power_law_spectrum(d, synth.ALPHA_QKV)).to(device)
+    Sh = torch.diag(lam.sqrt()).contiguous()
+    Shp = torch.diag(1.0 / lam.sqrt()).contiguous()
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    Om = torch.randn((d, r + p), generator=g, device=device, dtype=torch.float64)
+    glowq.group_solve(Ws, packs, Sh, Shp, r, p, q, Om)          # warm (module load, attributes)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    _, _, sing, gec, _, _ = glowq.group_solve(Ws, packs, Sh, Shp, r, p, q, Om)
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1)
+    st = glowq.device_status()
+    M = sum(outs)
+    l = r + p
+    flops = 2 * M * d * d + 2 * (2 * q + 2) * M * d * l
+    return {"workload": "whitened shared-B solve of one LLaMA-2-7B Q/K/V group (12288 x 4096 stacked error), "
+                        "r=64, p=16, q=2, float64 on the GPU",
+            "ms": ms, "fp64_GFLOP": flops / 1e9, "fp64_TFLOPs": flops / (ms * 1e-3) / 1e12,
+            "g_ec": float(gec.cpu()[0]), "sigma_1": float(sing.cpu()[0]), "status": st,
+            "context_pages_table11": "randomised SVD per layer 0.09 s, LLaMA-3.2-3B, A100 (thelatestinai.com "
+                                     "GlowQ page, Table 11)"}
+
+
 # ------------------------------------------------------------ profile cases
 
 def profile_case(case, device, steps=4):
@@ -796,6 +839,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-prefill", action="store_true", help="skip the T=2048 prefill line")
     ap.add_argument("--no-stack", action="store_true", help="skip the 40-layer LLaMA-2-13B stack line")
+    ap.add_argument("--no-solve", action="store_true", help="skip the GPU offline solve line")
     ap.add_argument("--no-units", action="store_true",
                     help="skip the per-unit lines (LLaMA-3.1-8B layer, LLaMA-2-13B decode batches)")
     ap.add_argument("--profile-case", choices=["decode", "prefill"],
@@ -878,6 +922,9 @@ def main():
     if not args.no_stack:
         stack = stack13b_line(device, args.warmup, ranks=ranks)
 
+    solve = None
+    if not args.no_solve:
+        solve = solve_line(device)
     l31 = s13b = None
     if not args.no_units:
         l31 = unit_lines(L31_UNITS, (1, 4096), device, hbm_peak, tf_peak, sub0=20000, ranks=ranks)
@@ -930,6 +977,7 @@ def main():
             "prefill": prefill,
             "stack13b": stack,
             "llama31_8b_layer": l31,
+            "offline_solve": solve,
             "llama2_13b_units_decode_batches": s13b,
         }
         print(json.dumps(line), flush=True)
