@@ -367,6 +367,42 @@ def solo_forward_fp4(mod: FP4Module, B, X, Y=None, workspace=None, stream=None):
     return Y
 
 
+class ForwardPlan:
+    """A group or solo forward with its arguments marshalled once: calling the
+    plan enqueues the kernels with a single C call (no per-call Python
+    marshalling), for callers that repeat one call on fixed buffers, e.g. a
+    decode loop that refills X in place.  The tensors must stay alive and at
+    the same addresses while the plan is used."""
+
+    def __init__(self, mods, B, X, Ys, R_out=None, workspace=None, solo: bool = False, stream=None):
+        import torch
+        _require_cuda(B, X)
+        T, d = X.shape
+        r = 0 if B is None else int(B.shape[0])
+        if r > 0 and workspace is None:
+            workspace = alloc_workspace(T, r, X.device)
+        if not solo and r > 0 and R_out is None:
+            R_out = torch.empty((T, r), dtype=torch.float16, device=X.device)
+        self._keep = (mods, B, X, Ys, R_out, workspace)
+        arr = _module_structs(mods, Ys, r > 0)
+        ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+        L = lib()
+        if solo:
+            self._fn = L.glowq_solo_forward
+            self._args = (arr, d, _ptr(B), r, _ptr(X), T, _ptr(workspace), ws_n)
+        else:
+            self._fn = L.glowq_group_forward
+            self._args = (arr, len(mods), d, _ptr(B), r, _ptr(X), T, _ptr(R_out), _ptr(workspace), ws_n)
+        self._stream = _stream(stream)
+        self.Ys, self.R = Ys, R_out
+
+    def __call__(self, stream=None):
+        rc = self._fn(*self._args, self._stream if stream is None else _stream(stream))
+        if rc != 0:
+            raise GlowQError(rc, "ForwardPlan")
+        return self.Ys
+
+
 def solo_forward_noalloc(mod: QModule, B, X, Y=None, stream=None):
     """Solo module forward with no workspace argument: the library's fixed
     scratch array is used, so the call allocates no device memory.  For callers

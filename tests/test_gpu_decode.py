@@ -330,3 +330,30 @@ def test_decode_activation_outliers(T):
     Yo = _np(glowq.solo_forward(to_dev(o)[0], torch.from_numpy(Bo).cuda(), torch.from_numpy(X).cuda()))
     ref = oracle.solo_forward(o[0].q, o[0].s, o[0].z, synth.bits(o[0].A), synth.bits(Bo), synth.bits(X))
     check(Yo.astype(np.float64), ref)
+
+
+@pytest.mark.parametrize("T", [1, 16, 100])
+def test_forward_plan_repeats_with_refilled_input(T):
+    """glowq.ForwardPlan marshals a call once; refilling X in place and calling
+    the plan again gives the new input's outputs (group and solo plans)."""
+    import torch
+    d, r = 1024, 32
+    mods = make_modules(d, [256, 128], seed=110 + T)
+    B = attach_random_factors(mods, d, r, seed=110 + T)
+    dev = to_dev(mods)
+    Bt = torch.from_numpy(B).cuda()
+    Xd = torch.empty((T, d), dtype=torch.float16, device="cuda")
+    Ys = [torch.empty((T, m.out_features), dtype=torch.float16, device="cuda") for m in dev]
+    Yo = torch.empty((T, 128), dtype=torch.float16, device="cuda")
+    pg = glowq.ForwardPlan(dev, Bt, Xd, Ys)
+    ps = glowq.ForwardPlan([dev[1]], Bt, Xd, [Yo], solo=True)
+    for k in range(2):
+        X = synth.activations(T, d, synth.ALPHA_QKV, seed=120 + 10 * T + k)
+        Xd.copy_(torch.from_numpy(X))
+        pg()
+        ps()
+        torch.cuda.synchronize()
+        refs, _ = _oracle_group(mods, B, X)
+        for Y, ref in zip(Ys, refs):
+            check(_np(Y).astype(np.float64), ref)
+        check(_np(Yo).astype(np.float64), refs[1])
