@@ -66,8 +66,16 @@ typedef enum glowq_status {
 
 /*
  * One quantised module of a group.  Device pointers:
- *   qweight  [O][d/8]  uint32: code k of row o is nibble (k % 8) of word k/8,
- *                      lowest nibble first (codes 0..15)
+ *   qweight  O * d/8 uint32 words: code k of row o is nibble (k % 8) of word
+ *                      kw = k/8 of that row, lowest nibble first (codes
+ *                      0..15).  The words are stored in blocks of 16 rows x
+ *                      64 k (16 x 8 words, 512 B): word kw of row o is at
+ *                      index ((o/16) * (d/64) + kw/8) * 128 + (o%16) * 8
+ *                      + kw%8, i.e. blocks along k within a 16-row tile,
+ *                      tiles in row order.  Every call that takes a qweight
+ *                      uses this layout (glowq_pack_int4 writes it); a decode
+ *                      ring stage (16 rows x 256 k) is then 2 KB of
+ *                      contiguous memory.
  *   scales   [O][d/128] fp16 bits (s)
  *   zeros    [O][d/128] uint8   (z, 0..15)
  *            dequantised weight w_hat[o][k] = fp16_RN((q - z) * s)
@@ -93,8 +101,9 @@ typedef struct glowq_module {
  *   s  = fp16_RN((mx - mn) / 15)   (s == 0 -> 1.0, s == inf -> 65504)
  *   z  = clamp(rint(-mn / s), 0, 15)
  *   q  = clamp(rint(w / s) + z, 0, 15)      (NaN weights -> code 0)
- * W: device, O x d fp32.  Outputs: qweight [O][d/8], scales [O][d/128],
- * zeros [O][d/128] (device, caller-allocated).  group_size must be 128.
+ * W: device, O x d fp32.  Outputs: qweight (O * d/8 words in the block
+ * layout described at glowq_module), scales [O][d/128], zeros [O][d/128]
+ * (device, caller-allocated).  group_size must be 128; O % 16 == 0.
  */
 GLOWQ_API glowq_status glowq_pack_int4(const float* W, int64_t O, int64_t d, int32_t group_size,
                              uint32_t* qweight, uint16_t* scales, uint8_t* zeros,
@@ -102,9 +111,10 @@ GLOWQ_API glowq_status glowq_pack_int4(const float* W, int64_t O, int64_t d, int
 
 /*
  * Dequantise to fp16: W_deq[o][k] = fp16_RN((q - z) * s), one rounding of the
- * exact product.  W_deq: device, O x d fp16 bits.  Used to check the packed
- * format; the forward kernels dequantise in registers / shared memory and
- * never materialise W_deq.
+ * exact product.  qweight in the block layout (glowq_module); W_deq: device,
+ * O x d fp16 bits, row-major.  O % 16 == 0.  Used to check the packed format;
+ * the forward kernels dequantise in registers / shared memory and never
+ * materialise W_deq.
  */
 GLOWQ_API glowq_status glowq_dequant_int4(const uint32_t* qweight, const uint16_t* scales,
                                 const uint8_t* zeros, int64_t O, int64_t d,
@@ -326,7 +336,7 @@ GLOWQ_API size_t glowq_noalloc_scratch_bytes(void);
  */
 typedef struct glowq_solve_module {
     const float* W;             /* O x d fp32 */
-    const uint32_t* qweight;    /* [O][d/8] */
+    const uint32_t* qweight;    /* O * d/8 words, block layout (glowq_module) */
     const uint16_t* scales;     /* [O][d/128] fp16 bits */
     const uint8_t* zeros;       /* [O][d/128] */
     int64_t out_features;       /* O */
@@ -349,7 +359,8 @@ GLOWQ_API size_t glowq_solve_workspace_bytes(int64_t rows, int64_t d, int32_t r,
  * E_w has the singular values and right vectors of the pages' thin-QR core
  * M = R_e Sx^{1/2} (E_w = Q_e M), so the factors are the core's.  All
  * arithmetic is float64 on the device.
- *   mods, m        host array of 1..GLOWQ_MAX_MODULES modules
+ *   mods, m        host array of 1..GLOWQ_MAX_MODULES modules (out_features
+ *                  % 16 == 0, qweight in the block layout of glowq_module)
  *   Sx_half        device, d x d float64 Sx^{1/2} (symmetric)
  *   Sx_half_pinv   device, d x d float64 pseudo-inverse of Sx^{1/2}
  *   r, p, q        rank (>= 1, r % 8 == 0), oversampling (even, r + p <= 112
@@ -408,8 +419,8 @@ GLOWQ_API glowq_status glowq_select_restore_scores(const double* score, const in
  * row_norms[2*o+1] = ||W[o]||^2 (fp64, deterministic), from a module's fp32
  * weight and its packed form.  Summing the rows of every module of a unit
  * gives err_fro2 and w_fro2 for glowq_select_restore.
- *   W          device, O x d fp32
- *   row_norms  device, 2*O doubles (caller-allocated)
+ *   W          device, O x d fp32; qweight in the block layout (glowq_module)
+ *   row_norms  device, 2*O doubles (caller-allocated); O % 16 == 0
  */
 GLOWQ_API glowq_status glowq_error_norms(const float* W, const uint32_t* qweight,
                                const uint16_t* scales, const uint8_t* zeros,

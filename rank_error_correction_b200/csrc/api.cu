@@ -172,7 +172,7 @@ glowq_status glowq_pack_int4(const float* W, int64_t O, int64_t d, int32_t group
                              uint16_t* scales, uint8_t* zeros, void* stream) {
     if (O < 0 || d < 0) return GLOWQ_ERR_ARG;
     if (group_size != GLOWQ_GROUP_SIZE) return GLOWQ_ERR_UNSUPPORTED;
-    if (d % GLOWQ_GROUP_SIZE != 0) return GLOWQ_ERR_SHAPE;
+    if (d % GLOWQ_GROUP_SIZE != 0 || O % 16 != 0) return GLOWQ_ERR_SHAPE;   // 16-row blocks
     if (O == 0 || d == 0) return GLOWQ_OK;
     if (!W || !qweight || !scales || !zeros) return GLOWQ_ERR_ARG;
     if (!aligned16(W) || (reinterpret_cast<uintptr_t>(qweight) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 1u))
@@ -185,7 +185,7 @@ glowq_status glowq_dequant_int4(const uint32_t* qweight, const uint16_t* scales,
                                 int64_t d, int32_t group_size, uint16_t* W_deq, void* stream) {
     if (O < 0 || d < 0) return GLOWQ_ERR_ARG;
     if (group_size != GLOWQ_GROUP_SIZE) return GLOWQ_ERR_UNSUPPORTED;
-    if (d % GLOWQ_GROUP_SIZE != 0) return GLOWQ_ERR_SHAPE;
+    if (d % GLOWQ_GROUP_SIZE != 0 || O % 16 != 0) return GLOWQ_ERR_SHAPE;
     if (O == 0 || d == 0) return GLOWQ_OK;
     if (!qweight || !scales || !zeros || !W_deq) return GLOWQ_ERR_ARG;
     if (!aligned16(W_deq) || (reinterpret_cast<uintptr_t>(qweight) & 3u) || (reinterpret_cast<uintptr_t>(scales) & 1u))
@@ -198,7 +198,7 @@ glowq_status glowq_dequant_int4(const uint32_t* qweight, const uint16_t* scales,
 glowq_status glowq_error_norms(const float* W, const uint32_t* qweight, const uint16_t* scales,
                                const uint8_t* zeros, int64_t O, int64_t d, double* row_norms, void* stream) {
     if (O < 0 || d < 0) return GLOWQ_ERR_ARG;
-    if (d % GLOWQ_GROUP_SIZE != 0) return GLOWQ_ERR_SHAPE;
+    if (d % GLOWQ_GROUP_SIZE != 0 || O % 16 != 0) return GLOWQ_ERR_SHAPE;
     if (O == 0 || d == 0) return GLOWQ_OK;
     if (!W || !qweight || !scales || !zeros || !row_norms) return GLOWQ_ERR_ARG;
     if ((reinterpret_cast<uintptr_t>(row_norms) & 7u) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
@@ -329,6 +329,7 @@ glowq_status glowq_group_solve(const glowq_solve_module* mods, int32_t m, int64_
     for (int i = 0; i < m; ++i) {
         const glowq_solve_module& md = mods[i];
         if (!md.W || !md.qweight || !md.scales || !md.zeros || md.out_features <= 0) return GLOWQ_ERR_ARG;
+        if (md.out_features % 16 != 0) return GLOWQ_ERR_SHAPE;   // 16-row code blocks
         if ((reinterpret_cast<uintptr_t>(md.qweight) & 3u) || (reinterpret_cast<uintptr_t>(md.scales) & 1u) ||
             (reinterpret_cast<uintptr_t>(md.W) & 3u))
             return GLOWQ_ERR_ALIGN;

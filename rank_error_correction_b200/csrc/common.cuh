@@ -11,6 +11,16 @@ namespace glowq {
 
 constexpr int kGroup = GLOWQ_GROUP_SIZE;   // INT4 quantisation group along d
 
+// INT4 packed weights are stored in blocks of 16 rows x 64 k (8 words of 8
+// codes per row, 512 B), blocks ordered along k within a 16-row tile and tiles
+// in row order: word kw of row o (codes of k = 8 kw .. 8 kw + 7) sits at this
+// index.  A decode ring stage (16 rows x two 128-groups) is then 2 KB of
+// contiguous memory, and a prefill k-block (128 rows x 64 k) eight
+// contiguous 512-byte blocks.
+__host__ __device__ __forceinline__ int64_t qword_index(int64_t o, int64_t kw, int64_t d) {
+    return ((((o >> 4) * (d >> 6) + (kw >> 3)) << 7) | ((o & 15) << 3) | (kw & 7));
+}
+
 // Bounded waits that run out record a code in the per-device status word
 // (defined in api.cu; kernels receive its device address as an argument).
 __device__ __forceinline__ void record_status(unsigned int* status, unsigned int code) {
@@ -136,6 +146,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* map, uint6
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* map, uint64_t* bar, int c0, int c1, int c2,
+                                            int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
         : "memory");
 }
 // L2 policy for data read exactly once per call (decode weight streams): its

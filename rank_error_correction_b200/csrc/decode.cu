@@ -114,7 +114,9 @@ struct GemvModule {
 };
 
 struct GemvArgs {
-    CUtensorMap tmq[GLOWQ_MAX_MODULES];   // qweight [O][d/8] u32, box {32 words, 16 rows}
+    // INT4: qweight as [O/16 x d/64 blocks][64 u64] (512-byte blocks), box {64, 4};
+    // FP4: codes [O][d/8] u32, box {32 words, 16 rows}
+    CUtensorMap tmq[GLOWQ_MAX_MODULES];
     GemvModule mod[GLOWQ_MAX_MODULES];
     int m;
     int d;
@@ -333,6 +335,51 @@ __device__ __forceinline__ void rproj_reduce(const GemvArgs& a, int rb, int S, i
         pk.x = h2_as_u32(h01);
         pk.y = h2_as_u32(h23);
         *reinterpret_cast<uint2*>(a.R + (int64_t)tok * r + rb * 16 + qd * 4) = pk;
+    }
+}
+
+// Every CTA's control warp, once all nrb x S items have stored their partial
+// sums: the whole R[t][c] = fp16(sum over s ascending of part[s][t][c]) (the
+// order and rounding of rproj_reduce, so every CTA holds the same bits) into
+// its shared-memory copy rs (rows of `pitch` halves, tokens T .. ntok-1 zero);
+// `store` also writes it to the caller's R.  One hop after the last partial
+// instead of a reduction by the block's last producer followed by a second
+// hand-off of R.
+__device__ __forceinline__ void rproj_reduce_all(const GemvArgs& a, int S, int lane, __half* rs, int pitch, int ntok,
+                                                 bool store) {
+    const int T = a.T, r = a.r;
+    const int qpr = r / 4;   // 4-column quads per token (r % 8 == 0)
+    const int64_t stride = (int64_t)T * r;
+    for (int o = lane; o < ntok * qpr; o += 32) {
+        const int tok = o / qpr, col = (o - tok * qpr) * 4;
+        uint2 pk = make_uint2(0, 0);
+        if (tok < T) {
+            const float* pp = a.part + (int64_t)tok * r + col;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s0 = 0; s0 < S; s0 += 8) {
+                float4 p8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (s0 + u < S) p8[u] = __ldcg(reinterpret_cast<const float4*>(pp + (s0 + u) * stride));
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    if (s0 + u < S) {
+                        if (s0 + u == 0) {
+                            v = p8[u];
+                        } else {
+                            v.x += p8[u].x; v.y += p8[u].y; v.z += p8[u].z; v.w += p8[u].w;
+                        }
+                    }
+            }
+            if (a.tok_scale) {   // W4A8: R = s_t X' B^T
+                const float ts = a.tok_scale[tok];
+                v.x *= ts; v.y *= ts; v.z *= ts; v.w *= ts;
+            }
+            pk.x = h2_as_u32(__floats2half2_rn(v.x, v.y));
+            pk.y = h2_as_u32(__floats2half2_rn(v.z, v.w));
+            if (store) *reinterpret_cast<uint2*>(a.R + (int64_t)tok * r + col) = pk;
+        }
+        *reinterpret_cast<uint2*>(rs + tok * pitch + col) = pk;
     }
 }
 
@@ -580,6 +627,12 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     unsigned char* my_ring = ring + warp * kStages * 2048;
     const uint32_t ring_smem = smem_u32(my_ring);
     const CUtensorMap* tmq = &args.tmq[mi];
+    // stage i of this warp covers groups G0 + 2i, G0 + 2i + 1 of its 16 rows:
+    // INT4 the four 64-k blocks (tile * 2 ngroups + 2 group ..) of those groups,
+    // FP4 a 16-row box
+    const int qx0 = (FMT == GLOWQ_FMT_INT4) ? 0 : G0 * 16;
+    const int qy0 = (FMT == GLOWQ_FMT_INT4) ? ((tile - tb) * ngroups + G0) * 2 : tile_row;
+    const int qdx = (FMT == GLOWQ_FMT_INT4) ? 0 : 32, qdy = (FMT == GLOWQ_FMT_INT4) ? 4 : 0;
     const int nsub = G1 - G0;
     const int npairs = (nsub + 1) / 2;
     // the barriers are initialised and fenced while this thread has no memory
@@ -598,10 +651,31 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     const int64_t sz_base = (int64_t)(tile_row + rr) * ngroups + G0;
     const int nsub0 = G1 - G0;
     const bool one_batch = active && nsub0 <= 32;
+    // INT4 with 8-group-aligned rows and split: one 16-byte scale load and one
+    // 8-byte zero load per (row, 8 groups), two per lane, instead of one 2-byte
+    // and one 1-byte load per (row, group): 3 warp loads instead of 32 in the
+    // prologue's load queue ahead of the weight stream
+    const bool vec_sz = FMT == GLOWQ_FMT_INT4 && one_batch && (nsub0 & 7) == 0 && (G0 & 7) == 0 &&
+                        (ngroups & 7) == 0 && (reinterpret_cast<uintptr_t>(Ms) & 15) == 0 &&
+                        (reinterpret_cast<uintptr_t>(Mz) & 7) == 0;
+    const int szc = nsub0 >> 3;   // 8-group chunks per row (vec_sz)
+    uint4 vs[2];
+    uint2 vz[2];
     unsigned short sv[16];
     unsigned char zv[16];
     uint2 fv[16];      // MXFP4: 4 E8M0 bytes of the group; NVFP4: 8 E4M3 bytes
-    if (one_batch) {
+    if (vec_sz) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = lane + 32 * h;
+            if (c < 16 * szc) {
+                const int row = c / szc, part = c - row * szc;
+                const int64_t e = (int64_t)(tile_row + row) * ngroups + G0 + part * 8;
+                vs[h] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __half*>(Ms) + e));
+                vz[h] = __ldg(reinterpret_cast<const uint2*>(Mz + e));
+            }
+        }
+    } else if (one_batch) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int gg = (lane >> 4) + 2 * j;
@@ -639,7 +713,7 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         if (lane == 0) {
             for (int i = 0; i < kStages && i < npairs; ++i) {
                 mbar_arrive_expect_tx(my_bars + i, 2048u);
-                tma_load_2d_hint(ring_smem + i * 2048, tmq, my_bars + i, (G0 + 2 * i) * 16, tile_row, wpol);
+                tma_load_2d_hint(ring_smem + i * 2048, tmq, my_bars + i, qx0 + i * qdx, qy0 + i * qdy, wpol);
             }
         }
         __syncwarp();
@@ -657,7 +731,20 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
 
     // 5) stage (s, 64 + z) of the warp's rows x groups [G0, G1); longer splits
     //    load in batches of 16 per lane, all issued before any is used
-    if (one_batch) {
+    if (vec_sz) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int c = lane + 32 * h;
+            if (c < 16 * szc) {
+                const int row = c / szc, part = c - row * szc;
+                const __half* sh = reinterpret_cast<const __half*>(&vs[h]);
+                const uint8_t* zb = reinterpret_cast<const uint8_t*>(&vz[h]);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    my_sz[row * sz_stride + part * 8 + k] = make_float2(__half2float(sh[k]), 64.0f + (float)zb[k]);
+            }
+        }
+    } else if (one_batch) {
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             const int gg = (lane >> 4) + 2 * j;
@@ -757,9 +844,11 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     __syncthreads();
 
     // 7) the control warp, beside the main loop: this CTA's items of the anchor
-    //    projection (the last producer of a 16-row block of B reduces it into
-    //    the caller's R), then, once every block is stored, R into rs (padding
-    //    tokens zero) for the epilogue; the last CTA here zeroes the flags
+    //    projection (fp32 partial sums), then R into rs (padding tokens zero)
+    //    for the epilogue: for T <= 8 every CTA reduces the partials itself once
+    //    all items are counted on one flag; for more tokens each 16-row block's
+    //    last producer reduces it into the caller's R and every CTA copies R.
+    //    The last CTA here zeroes the flags.
     if (control && r > 0 && args.rpre) {
         // R was stored by the preceding launch, complete before this grid's wait
         const int cpr = r / 8;
@@ -784,25 +873,40 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                                (int64_t)d * 2, xs, xpitch, C0, lane);
             }
             __syncwarp();   // every lane's partial sums precede lane 0's release
-            unsigned int prev = 0;
-            if (lane == 0)
-                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(args.flags + it.rb) : "memory");
-            prev = __shfl_sync(0xffffffffu, prev, 0);
-            if (prev == (unsigned)nslc - 1) {   // the block's last producer
-                __syncwarp();   // lane 0's acquire precedes every lane's loads of the partials
-                rproj_reduce(args, it.rb, nslc, lane);
-                __syncwarp();
+            if constexpr (NT == 1) {
                 if (lane == 0) flag_release_add(args.flags + kFlagReady, 1u);
+            } else {
+                unsigned int prev = 0;
+                if (lane == 0)
+                    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(args.flags + it.rb) : "memory");
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev == (unsigned)nslc - 1) {   // the block's last producer
+                    __syncwarp();   // lane 0's acquire precedes every lane's loads of the partials
+                    rproj_reduce(args, it.rb, nslc, lane);
+                    __syncwarp();
+                    if (lane == 0) flag_release_add(args.flags + kFlagReady, 1u);
+                }
             }
         }
-        if (lane == 0) flag_wait_geq(args.flags + kFlagReady, (unsigned)nrb, args.status);
-        __syncwarp();
-        const int cpr = r / 8;   // 16-byte chunks per row
-        for (int c = lane; c < 8 * NT * cpr; c += 32) {
-            const int tok = c / cpr, cc = c - tok * cpr;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (tok < T) v = ldcg_128(args.R + (int64_t)tok * r + cc * 8);
-            *reinterpret_cast<uint4*>(rs + tok * (r + 8) + cc * 8) = v;
+        if constexpr (NT == 1) {
+            // T <= 8: all items of all blocks stored, this CTA reduces R itself
+            // (CTA 0 also stores it for the caller): one hop after the last partial
+            if (lane == 0) flag_wait_geq(args.flags + kFlagReady, (unsigned)(nrb * nslc), args.status);
+            __syncwarp();   // lane 0's acquire precedes every lane's loads of the partials
+            rproj_reduce_all(args, nslc, lane, rs, r + 8, 8 * NT, blockIdx.x == 0);
+        } else {
+            // more tokens: each block's last producer reduces it into the caller's
+            // R; every CTA then copies R (the reduction is T x r x slices of
+            // loads, too many for one warp per CTA)
+            if (lane == 0) flag_wait_geq(args.flags + kFlagReady, (unsigned)nrb, args.status);
+            __syncwarp();
+            const int cpr = r / 8;   // 16-byte chunks per row
+            for (int c = lane; c < 8 * NT * cpr; c += 32) {
+                const int tok = c / cpr, cc = c - tok * cpr;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (tok < T) v = ldcg_128(args.R + (int64_t)tok * r + cc * 8);
+                *reinterpret_cast<uint4*>(rs + tok * (r + 8) + cc * 8) = v;
+            }
         }
         __syncwarp();
         if (lane == 0) {
@@ -838,8 +942,14 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
             xb[n] = xs + tok * xpitch + (G0 - C0) * 16 + t;
         }
         const float* xsp = xsum + (G0 - C0) * 2 * 8 * NT + 2 * t;
-        // lane (g, t) reads 16 B of rows g and g+8 per group
-        const unsigned char* rd = my_ring + g * 128 + t * 16;
+        // lane (g, t) reads 16 B (words 4t .. 4t+3 of a group row) of rows g and
+        // g+8 per group: INT4 stages are four [16 rows][32 B] blocks (words 4t..
+        // are in block 2h + t/2 at byte 16 (t % 2)), FP4 stages one [16 rows][128 B] box
+        constexpr int kRowPitch = (FMT == GLOWQ_FMT_INT4) ? 32 : 128;
+        constexpr int kGrp1 = (FMT == GLOWQ_FMT_INT4) ? 1024 : 64;   // second group
+        constexpr int kRow8 = 8 * kRowPitch;                           // row g + 8
+        const unsigned char* rd = my_ring + g * kRowPitch +
+                                  ((FMT == GLOWQ_FMT_INT4) ? (t >> 1) * 512 + (t & 1) * 16 : t * 16);
         bool ok = true;
         int slot = 0;
         uint32_t phase = 0;
@@ -849,16 +959,16 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
             const unsigned char* sl = rd + slot * 2048;
             uint4 w4[2][2];
             w4[0][0] = *reinterpret_cast<const uint4*>(sl);
-            w4[0][1] = *reinterpret_cast<const uint4*>(sl + 1024);
-            w4[1][0] = *reinterpret_cast<const uint4*>(sl + 64);
-            w4[1][1] = *reinterpret_cast<const uint4*>(sl + 1024 + 64);
+            w4[0][1] = *reinterpret_cast<const uint4*>(sl + kRow8);
+            w4[1][0] = *reinterpret_cast<const uint4*>(sl + kGrp1);
+            w4[1][1] = *reinterpret_cast<const uint4*>(sl + kGrp1 + kRow8);
             if (p + kStages < npairs) {
                 fence_proxy_async_smem();   // this lane's reads of the slot precede the refill
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive_expect_tx(my_bars + slot, 2048u);
-                    tma_load_2d_hint(ring_smem + slot * 2048, tmq, my_bars + slot, (G0 + 2 * (p + kStages)) * 16,
-                                     tile_row, wpol);
+                    tma_load_2d_hint(ring_smem + slot * 2048, tmq, my_bars + slot, qx0 + (p + kStages) * qdx,
+                                     qy0 + (p + kStages) * qdy, wpol);
                 }
             }
             const bool two = 2 * p + 1 < nsub;    // warp-uniform
@@ -1255,9 +1365,13 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
         a.mod[i].O = (int)mods[i].O;
         a.mod[i].tile_begin = tiles;
         tiles += (int)(mods[i].O / 16);
-        if (!make_map(&a.tmq[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, mods[i].q, (uint64_t)(d / 8), (uint64_t)mods[i].O,
-                      (uint64_t)d / 2, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE))
-            return cudaErrorInvalidValue;
+        const bool mapped =
+            (fmt == GLOWQ_FMT_INT4)
+                ? make_map(&a.tmq[i], CU_TENSOR_MAP_DATA_TYPE_UINT64, mods[i].q, 64,
+                           (uint64_t)(mods[i].O / 16) * (uint64_t)(d / 64), 512, 64, 4, CU_TENSOR_MAP_SWIZZLE_NONE)
+                : make_map(&a.tmq[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, mods[i].q, (uint64_t)(d / 8),
+                           (uint64_t)mods[i].O, (uint64_t)d / 2, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (!mapped) return cudaErrorInvalidValue;
     }
     if (tiles == 0) return cudaSuccess;
     const int nt = (T <= 8) ? 1 : 2;

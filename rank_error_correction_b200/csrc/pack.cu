@@ -56,14 +56,15 @@ __global__ void __launch_bounds__(256) pack_int4_kernel(const float* __restrict_
         nib |= ((uint32_t)c & 0xfu) << (4 * i);
     }
     const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
-    if ((lane & 1) == 0) q[o * (d / 8) + g * (kGroup / 8) + lane / 2] = nib | (hi << 16);
+    if ((lane & 1) == 0) q[qword_index(o, g * (kGroup / 8) + lane / 2, d)] = nib | (hi << 16);
     if (lane == 0) {
         s[o * ng + g] = sh;
         z[o * ng + g] = (uint8_t)zf;
     }
 }
 
-// One thread per packed word: 8 fp16 outputs (one 16-byte store).
+// One thread per packed word (row-major order of the output): 8 fp16 outputs
+// (one 16-byte store).
 __global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t* __restrict__ q,
                                                             const __half* __restrict__ s,
                                                             const uint8_t* __restrict__ z, int64_t O,
@@ -74,7 +75,7 @@ __global__ void __launch_bounds__(256) dequant_int4_kernel(const uint32_t* __res
     const int64_t o = i / (d / 8), kw = i % (d / 8);
     const int64_t g = (kw * 8) / kGroup;
     const int64_t ng = d / kGroup;
-    const uint32_t w = q[i];
+    const uint32_t w = q[qword_index(o, kw, d)];
     const float sf = __half2float(s[o * ng + g]);
     const int zz = z[o * ng + g];
     __align__(16) __half v[8];
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(256) error_norms_kernel(const float* __restric
     double se = 0.0, sw = 0.0;
     for (int64_t kw = lane; kw < d / 8; kw += 32) {
         const int64_t g = (kw * 8) / kGroup;
-        const uint32_t w = q[o * (d / 8) + kw];
+        const uint32_t w = q[qword_index(o, kw, d)];
         const float sf = __half2float(s[o * ng + g]);
         const int zz = z[o * ng + g];
 #pragma unroll

@@ -181,7 +181,10 @@ struct PrefillModule {
 struct PrefillArgs {
     CUtensorMap tmX;                       // X [T][d] fp16, box {64, 128}, SW128
     CUtensorMap tmR;                       // R [T][r] fp16, box {64, 128}, SW128
-    CUtensorMap tmQ[GLOWQ_MAX_MODULES];    // qweight [O][d/8] u32, box {8, 128}, SW32
+    // INT4 qweight in 16-row x 64-k blocks as 4-D {8 words, 16 rows, d/64
+    // blocks, O/16 tiles}, box {8, 16, 1, 8} (eight contiguous 512-byte blocks);
+    // FP4 codes [O][d/8] u32, box {8, 128}; both land as 128 rows x 32 B, SW32
+    CUtensorMap tmQ[GLOWQ_MAX_MODULES];
     CUtensorMap tmA[GLOWQ_MAX_MODULES];    // A [O][r] fp16, box {64, 128}, SW128
     CUtensorMap tmY[GLOWQ_MAX_MODULES];    // Y [T][ldY] fp16 (O columns), box {128, 32} (TMA store)
     PrefillModule mod[GLOWQ_MAX_MODULES];
@@ -399,7 +402,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                     if (i < nkb) {
                         mbar_arrive_expect_tx(&bars->full[s], kXBytes + kQBytes);
                         tma_load_2d(xs, &args.tmX, &bars->full[s], i * kBK, c.n0 + tok_off);
-                        tma_load_2d(qs, &args.tmQ[c.mi], &bars->full[s], i * (kBK / 8), c.m0 + row_off);
+                        if constexpr (FMT == GLOWQ_FMT_INT4)
+                            tma_load_4d(qs, &args.tmQ[c.mi], &bars->full[s], 0, 0, i, (c.m0 + row_off) / 16);
+                        else
+                            tma_load_2d(qs, &args.tmQ[c.mi], &bars->full[s], i * (kBK / 8), c.m0 + row_off);
                     } else {
                         if (!waited && args.wait_dep) {   // R is complete
                             pdl_wait();
@@ -875,6 +881,21 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// INT4 codes in 16-row x 64-k blocks (512 B, blocks along k within a 16-row
+// tile): a 128-row x 64-k box is 8 tiles' blocks of one k-block, written to
+// shared memory in row order like the row-major layout's 2-D box.
+static bool make_map_q4(CUtensorMap* map, const void* q, int d, int64_t O) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {8, 16, (cuuint64_t)(d / 64), (cuuint64_t)(O / 16)};
+    const cuuint64_t strides[3] = {32, 512, (cuuint64_t)(d / 64) * 512};
+    const cuuint32_t box[4] = {8, 16, 1, kBM / 16};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, const_cast<void*>(q), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static size_t gemm_smem_bytes() {
     return (size_t)kGemmStages * kStageBytesG + kEpiBufs * kEpiBytes + sizeof(GemmBarriers) + 1024;
 }
@@ -996,8 +1017,10 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     int mtiles = 0;
     for (int i = 0; i < m && ok; ++i) {
         const ModuleView& mv = mods[i];
-        ok = ok && make_map(&a->tmQ[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, mv.q, (uint64_t)(d / 8), (uint64_t)mv.O,
-                            (uint64_t)d / 2, kBK / 8, kBM, CU_TENSOR_MAP_SWIZZLE_32B);
+        ok = ok && ((fmt == GLOWQ_FMT_INT4)
+                        ? make_map_q4(&a->tmQ[i], mv.q, d, mv.O)
+                        : make_map(&a->tmQ[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, mv.q, (uint64_t)(d / 8), (uint64_t)mv.O,
+                                   (uint64_t)d / 2, kBK / 8, kBM, CU_TENSOR_MAP_SWIZZLE_32B));
         const bool has_A = use_r && mv.A != nullptr;
         if (has_A)
             ok = ok && make_map(&a->tmA[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, mv.A, (uint64_t)r, (uint64_t)mv.O,

@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(256) error_rows_f64_kernel(const float* __rest
     if (i >= O * (d / 8)) return;
     const int64_t o = i / (d / 8), k0 = (i % (d / 8)) * 8;
     const int64_t g = o * (d / 128) + k0 / 128;
-    const uint32_t w = q[i];
+    const uint32_t w = q[qword_index(o, i % (d / 8), d)];
     const float sc = __half2float(s[g]);
     const int zz = z[g];
 #pragma unroll

@@ -145,7 +145,9 @@ def _require_cuda(*ts):
 # ---------------------------------------------------------------- packing ----
 
 def pack_int4(W, stream=None):
-    """W (O x d fp32, CUDA) -> (qweight int32 [O, d/8], scales fp16 [O, d/128], zeros uint8 [O, d/128])."""
+    """W (O x d fp32, CUDA) -> (qweight int32 [O, d/8], scales fp16 [O, d/128], zeros uint8 [O, d/128]).
+    qweight holds O * d/8 words in the library's block layout (16-row x 64-k
+    blocks of 512 B; see tile_int4), not row by row."""
     import torch
     _require_cuda(W)
     if W.dtype != torch.float32 or W.dim() != 2:
@@ -157,6 +159,21 @@ def pack_int4(W, stream=None):
     _check(lib().glowq_pack_int4(_ptr(W), O, d, GROUP_SIZE, _ptr(q), _ptr(s), _ptr(z), _stream(stream)),
            "glowq_pack_int4")
     return q, s, z
+
+
+def tile_int4(q):
+    """Row-major INT4 words (int32 [O, d/8], code k of row o in word k/8) ->
+    the library's block layout: blocks of 16 rows x 64 k (16 x 8 words),
+    blocks along k within a 16-row tile, tiles in row order.  Same shape and
+    dtype; O % 16 == 0.  For codes packed elsewhere."""
+    O, w = q.shape
+    return q.reshape(O // 16, 16, w // 8, 8).permute(0, 2, 1, 3).contiguous().reshape(O, w)
+
+
+def untile_int4(q):
+    """Inverse of tile_int4: the library's block layout -> row-major words."""
+    O, w = q.shape
+    return q.reshape(O // 16, w // 8, 16, 8).permute(0, 2, 1, 3).contiguous().reshape(O, w)
 
 
 def dequant_int4(q, s, z, d: int, stream=None):

@@ -96,13 +96,27 @@ def check(y_gpu: np.ndarray, y_ref: np.ndarray, ymax: Optional[float] = None, to
     assert ex <= 1.0, f"per-element bound exceeded by {ex:.2f}x"
 
 
+def tile_int4(q: np.ndarray) -> np.ndarray:
+    """Row-major INT4 words [O][d/8] (the oracle's layout) -> the library's
+    block layout: 16-row x 64-k blocks of 16 x 8 words, blocks along k within
+    a 16-row tile, tiles in row order (returned with shape [O, d/8])."""
+    O, w = q.shape
+    return np.ascontiguousarray(q.reshape(O // 16, 16, w // 8, 8).transpose(0, 2, 1, 3)).reshape(O, w)
+
+
+def untile_int4(q: np.ndarray) -> np.ndarray:
+    """Inverse of tile_int4."""
+    O, w = q.shape
+    return np.ascontiguousarray(q.reshape(O // 16, w // 8, 16, 8).transpose(0, 2, 1, 3)).reshape(O, w)
+
+
 def to_dev(mods: List[HostModule], device="cuda", with_A: bool = True):
     import torch
     from rank_error_correction_b200 import glowq
     out = []
     for m in mods:
         out.append(glowq.QModule(
-            torch.from_numpy(m.q.view(np.int32)).to(device),
+            torch.from_numpy(tile_int4(m.q).view(np.int32)).to(device),
             torch.from_numpy(m.s.view(np.float16)).to(device),
             torch.from_numpy(m.z).to(device),
             None if (m.A is None or not with_A) else torch.from_numpy(m.A).to(device)))

@@ -85,6 +85,9 @@ def test_host_validation_errors(L):
     assert L.glowq_pack_int4(0x1000, 16, 256, 64, 0x2000, 0x3000, 0x4000, None) == 6
     assert L.glowq_pack_int4(0x1000, 16, 200, 128, 0x2000, 0x3000, 0x4000, None) == 2
     assert L.glowq_pack_int4(0x1000, 0, 256, 128, 0x2000, 0x3000, 0x4000, None) == 0
+    # the codes are stored in 16-row blocks: row counts must be multiples of 16
+    assert L.glowq_pack_int4(0x1000, 8, 256, 128, 0x2000, 0x3000, 0x4000, None) == 2
+    assert L.glowq_dequant_int4(0x1000, 0x2000, 0x3000, 24, 256, 128, 0x4000, None) == 2
     assert L.glowq_dequant_int4(0x1000, 0x2000, 0x3000, 16, 256, 128, 0x4008, None) == 3
 
 

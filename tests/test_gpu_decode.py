@@ -11,7 +11,8 @@ import pytest
 import oracle
 from rank_error_correction_b200 import build, glowq, synth
 
-from helpers import (check, TOL, attach_random_factors, attach_solved_factors, make_modules, normwise, to_dev)
+from helpers import (check, TOL, attach_random_factors, attach_solved_factors, make_modules, normwise, tile_int4,
+                     to_dev, untile_int4)
 
 pytestmark = pytest.mark.gpu
 
@@ -38,7 +39,7 @@ def test_pack_bit_exact(O, d, outliers):
     W = synth.weights(O, d, seed=21, outlier_cols=outliers)
     q_o, s_o, z_o = oracle.quantize_int4(W)
     q, s, z = glowq.pack_int4(torch.from_numpy(W).cuda())
-    assert np.array_equal(_np(q).view(np.uint32), q_o)
+    assert np.array_equal(untile_int4(_np(q).view(np.uint32)), q_o)
     assert np.array_equal(_np(s).view(np.uint16), s_o)
     assert np.array_equal(_np(z), z_o)
 
@@ -46,7 +47,7 @@ def test_pack_bit_exact(O, d, outliers):
 def test_pack_edge_values_bit_exact():
     import torch
     d = 512
-    W = synth.weights(8, d, seed=22)
+    W = synth.weights(16, d, seed=22)                  # one 16-row block
     W[0, :128] = 0.0                                  # all-zero group
     W[1, :128] = 1e-30                                # scale underflow -> 1.0
     W[2, 5] = np.nan                                  # NaN weight -> code 0
@@ -56,7 +57,7 @@ def test_pack_edge_values_bit_exact():
     W[6, 256:384] = np.linspace(-1, 3, 128, dtype=np.float32)
     q_o, s_o, z_o = oracle.quantize_int4(W)
     q, s, z = glowq.pack_int4(torch.from_numpy(W).cuda())
-    assert np.array_equal(_np(q).view(np.uint32), q_o)
+    assert np.array_equal(untile_int4(_np(q).view(np.uint32)), q_o)
     assert np.array_equal(_np(s).view(np.uint16), s_o)
     assert np.array_equal(_np(z), z_o)
 
@@ -67,7 +68,7 @@ def test_dequant_bit_exact(O, d):
     W = synth.weights(O, d, seed=23, outlier_cols=3)
     q_o, s_o, z_o = oracle.quantize_int4(W)
     ref = oracle.dequant_int4(q_o, s_o, z_o, d)
-    out = glowq.dequant_int4(torch.from_numpy(q_o.view(np.int32)).cuda(),
+    out = glowq.dequant_int4(torch.from_numpy(tile_int4(q_o).view(np.int32)).cuda(),
                              torch.from_numpy(s_o.view(np.float16)).cuda(), torch.from_numpy(z_o).cuda(), d)
     assert np.array_equal(_np(out).view(np.uint16), ref)
 
@@ -77,7 +78,7 @@ def test_error_norms_match_oracle():
     O, d = 512, 1024
     W = synth.weights(O, d, seed=24, outlier_cols=4)
     q, s, z = oracle.quantize_int4(W)
-    rows = _np(glowq.error_norms(torch.from_numpy(W).cuda(), torch.from_numpy(q.view(np.int32)).cuda(),
+    rows = _np(glowq.error_norms(torch.from_numpy(W).cuda(), torch.from_numpy(tile_int4(q).view(np.int32)).cuda(),
                                  torch.from_numpy(s.view(np.float16)).cuda(), torch.from_numpy(z).cuda()))
     _, e2, w2 = oracle.quant_error(W, q, s, z, want_matrix=False)
     assert rows.sum(axis=0)[0] == pytest.approx(e2, rel=1e-12)

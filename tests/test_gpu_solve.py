@@ -9,7 +9,7 @@ import pytest
 import oracle
 from rank_error_correction_b200 import build, glowq, synth
 
-from helpers import make_modules
+from helpers import make_modules, tile_int4
 
 pytestmark = pytest.mark.gpu
 
@@ -32,7 +32,7 @@ def _case(d, outs, r, p, alpha, seed, outlier_cols=0):
     Om = synth.gaussian_test_matrix(d, r + p, seed=seed)
     E = np.vstack([oracle.quant_error(m.W, m.q, m.s, m.z)[0] for m in mods])
     dev = dict(Ws=[torch.from_numpy(m.W).cuda() for m in mods],
-               packs=[(torch.from_numpy(m.q.view(np.int32)).cuda(), torch.from_numpy(m.s.view(np.float16)).cuda(),
+               packs=[(torch.from_numpy(tile_int4(m.q).view(np.int32)).cuda(), torch.from_numpy(m.s.view(np.float16)).cuda(),
                        torch.from_numpy(m.z).cuda()) for m in mods],
                Sh=torch.from_numpy(np.ascontiguousarray(Sh)).cuda(),
                Shp=torch.from_numpy(np.ascontiguousarray(Shp)).cuda(),
