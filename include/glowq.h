@@ -426,8 +426,10 @@ GLOWQ_API glowq_status glowq_error_norms(const float* W, const uint32_t* qweight
                                const uint16_t* scales, const uint8_t* zeros,
                                int64_t O, int64_t d, double* row_norms, void* stream);
 
-/* Reads and clears this device's status word (GLOWQ_OK, GLOWQ_ERR_TIMEOUT or
-   GLOWQ_ERR_NUMERIC); synchronises `stream` first. */
+/* Reads and clears this device's status word (GLOWQ_OK, GLOWQ_ERR_TIMEOUT,
+   GLOWQ_ERR_NUMERIC, or GLOWQ_ERR_ALIGN if a decode kernel found its shared
+   memory base not 1 KB-aligned and skipped its work); synchronises `stream`
+   first. */
 GLOWQ_API glowq_status glowq_get_device_status(void* stream);
 
 /*

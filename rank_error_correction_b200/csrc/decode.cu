@@ -114,8 +114,9 @@ struct GemvModule {
 };
 
 struct GemvArgs {
-    // INT4: qweight as [O/16 x d/64 blocks][64 u64] (512-byte blocks), box {64, 4};
-    // FP4: codes [O][d/8] u32, box {32 words, 16 rows}
+    // INT4: qweight as lines of 128 B (a 16-row x 64-k block is 4 lines), box
+    // {16 u64, 16 lines} = four blocks (2 KB), 128-byte swizzle; FP4: codes
+    // [O][d/8] u32, box {32 words, 16 rows}
     CUtensorMap tmq[GLOWQ_MAX_MODULES];
     GemvModule mod[GLOWQ_MAX_MODULES];
     int m;
@@ -558,6 +559,14 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
                                                                            const __grid_constant__ GemvPlan plan) {
     pdl_launch_dependents();
     extern __shared__ __align__(1024) unsigned char smem[];
+    // the INT4 weight ring is written with the 128-byte swizzle, which needs
+    // 1 KB-aligned stage buffers: a misaligned base is reported, not used
+    if constexpr (FMT == GLOWQ_FMT_INT4) {
+        if ((smem_u32(smem) & 1023u) != 0u) {
+            if (threadIdx.x == 0) record_status(args.status, GLOWQ_ERR_ALIGN);
+            return;
+        }
+    }
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // the weight streams' TMA descriptors into the descriptor cache
     if (threadIdx.x < GLOWQ_MAX_MODULES && (int)threadIdx.x < args.m)
@@ -628,11 +637,11 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
     const uint32_t ring_smem = smem_u32(my_ring);
     const CUtensorMap* tmq = &args.tmq[mi];
     // stage i of this warp covers groups G0 + 2i, G0 + 2i + 1 of its 16 rows:
-    // INT4 the four 64-k blocks (tile * 2 ngroups + 2 group ..) of those groups,
-    // FP4 a 16-row box
+    // INT4 the four 64-k blocks (tile * 2 ngroups + 2 group ..) of those groups
+    // (4 lines of 128 B each), FP4 a 16-row box
     const int qx0 = (FMT == GLOWQ_FMT_INT4) ? 0 : G0 * 16;
-    const int qy0 = (FMT == GLOWQ_FMT_INT4) ? ((tile - tb) * ngroups + G0) * 2 : tile_row;
-    const int qdx = (FMT == GLOWQ_FMT_INT4) ? 0 : 32, qdy = (FMT == GLOWQ_FMT_INT4) ? 4 : 0;
+    const int qy0 = (FMT == GLOWQ_FMT_INT4) ? ((tile - tb) * ngroups + G0) * 8 : tile_row;
+    const int qdx = (FMT == GLOWQ_FMT_INT4) ? 0 : 32, qdy = (FMT == GLOWQ_FMT_INT4) ? 16 : 0;
     const int nsub = G1 - G0;
     const int npairs = (nsub + 1) / 2;
     // the barriers are initialised and fenced while this thread has no memory
@@ -943,13 +952,18 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         }
         const float* xsp = xsum + (G0 - C0) * 2 * 8 * NT + 2 * t;
         // lane (g, t) reads 16 B (words 4t .. 4t+3 of a group row) of rows g and
-        // g+8 per group: INT4 stages are four [16 rows][32 B] blocks (words 4t..
-        // are in block 2h + t/2 at byte 16 (t % 2)), FP4 stages one [16 rows][128 B] box
-        constexpr int kRowPitch = (FMT == GLOWQ_FMT_INT4) ? 32 : 128;
+        // g+8 per group.  INT4 stages are four [16 rows][32 B] blocks (words 4t..
+        // in block 2h + t/2 at byte 16 (t % 2)), copied as 16 lines of 128 B with
+        // the 128-byte swizzle (16-byte chunk c of line l of a 1 KB atom lands at
+        // chunk c ^ (l % 8)), so that the eight lanes of a 16-byte read phase hit
+        // eight different chunks; FP4 stages are one [16 rows][128 B] box.
         constexpr int kGrp1 = (FMT == GLOWQ_FMT_INT4) ? 1024 : 64;   // second group
-        constexpr int kRow8 = 8 * kRowPitch;                           // row g + 8
-        const unsigned char* rd = my_ring + g * kRowPitch +
-                                  ((FMT == GLOWQ_FMT_INT4) ? (t >> 1) * 512 + (t & 1) * 16 : t * 16);
+        auto swz = [](int o) { return o ^ (((o >> 7) & 7) << 4); };
+        const int o_lo = (FMT == GLOWQ_FMT_INT4) ? swz((t >> 1) * 512 + g * 32 + (t & 1) * 16) : g * 128 + t * 16;
+        const int o_hi = (FMT == GLOWQ_FMT_INT4) ? swz((t >> 1) * 512 + (g + 8) * 32 + (t & 1) * 16)
+                                                 : (g + 8) * 128 + t * 16;
+        const unsigned char* rd = my_ring + o_lo;   // row g
+        const unsigned char* rh = my_ring + o_hi;   // row g + 8
         bool ok = true;
         int slot = 0;
         uint32_t phase = 0;
@@ -957,11 +971,12 @@ __global__ void __launch_bounds__(512, 1) corrected_gemv_kernel(const __grid_con
         for (int p = 0; p < npairs; ++p) {
             if (ok) ok = mbar_wait(my_bars + slot, phase, args.status);
             const unsigned char* sl = rd + slot * 2048;
+            const unsigned char* sh8 = rh + slot * 2048;
             uint4 w4[2][2];
             w4[0][0] = *reinterpret_cast<const uint4*>(sl);
-            w4[0][1] = *reinterpret_cast<const uint4*>(sl + kRow8);
+            w4[0][1] = *reinterpret_cast<const uint4*>(sh8);
             w4[1][0] = *reinterpret_cast<const uint4*>(sl + kGrp1);
-            w4[1][1] = *reinterpret_cast<const uint4*>(sl + kGrp1 + kRow8);
+            w4[1][1] = *reinterpret_cast<const uint4*>(sh8 + kGrp1);
             if (p + kStages < npairs) {
                 fence_proxy_async_smem();   // this lane's reads of the slot precede the refill
                 __syncwarp();
@@ -1367,8 +1382,8 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
         tiles += (int)(mods[i].O / 16);
         const bool mapped =
             (fmt == GLOWQ_FMT_INT4)
-                ? make_map(&a.tmq[i], CU_TENSOR_MAP_DATA_TYPE_UINT64, mods[i].q, 64,
-                           (uint64_t)(mods[i].O / 16) * (uint64_t)(d / 64), 512, 64, 4, CU_TENSOR_MAP_SWIZZLE_NONE)
+                ? make_map(&a.tmq[i], CU_TENSOR_MAP_DATA_TYPE_UINT64, mods[i].q, 16,
+                           (uint64_t)mods[i].O * (uint64_t)d / 256, 128, 16, 16, CU_TENSOR_MAP_SWIZZLE_128B)
                 : make_map(&a.tmq[i], CU_TENSOR_MAP_DATA_TYPE_UINT32, mods[i].q, (uint64_t)(d / 8),
                            (uint64_t)mods[i].O, (uint64_t)d / 2, 32, 16, CU_TENSOR_MAP_SWIZZLE_NONE);
         if (!mapped) return cudaErrorInvalidValue;
