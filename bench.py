@@ -606,7 +606,9 @@ def time_stack13b(units, T, steps, warmup, device, mode, seed=0, ranks=None):
           for k, (n, _, d, _) in enumerate(S13_UNITS)}
     Ys = {n: [torch.empty((T, O), dtype=torch.float16, device=device) for O in outs]
           for n, outs, _, _ in S13_UNITS}
-    ws = glowq.alloc_workspace(T, R_RANK, device)
+    # one workspace for every unit: the largest any unit's call can use
+    wsn = max(glowq.workspace_bytes_for(T, R_RANK, d, outs) for _, outs, d, _ in S13_UNITS)
+    ws = torch.zeros(max(wsn, 16), dtype=torch.uint8, device=device)
     calls = []
     for u in units:
         a = u["name"]
@@ -709,7 +711,7 @@ def time_unit_chain(reps, X, T, calls, device, ranks=None):
     mods0, _ = reps[0]
     Ys = [torch.empty((T, m.out_features), dtype=torch.float16, device=device) for m in mods0]
     R = torch.empty((T, R_RANK), dtype=torch.float16, device=device)
-    ws = glowq.alloc_workspace(T, R_RANK, device)
+    ws = glowq.alloc_workspace(T, R_RANK, device, mods0[0].in_features, [m.out_features for m in mods0])
 
     def call(i):
         mods, B = reps[i % len(reps)]

@@ -173,21 +173,44 @@ GLOWQ_API glowq_status glowq_dequant_fp4(glowq_format fmt, const uint32_t* codes
 
 /*
  * Bytes of device scratch the forward calls need for T tokens at rank r:
- *   - 256 bytes of hand-off flags at offset 0, through which the decode GEMV
- *     (T <= 16) learns, while it already streams weights, that the kernel
- *     computing R = X B^T has seen X final and has stored R;
+ *   - a 4096-byte zero region at offset 0: the hand-off flags (bytes 0..255),
+ *     through which the decode GEMV (T <= 16) learns, while it already streams
+ *     weights, that the kernel computing R = X B^T has seen X final and has
+ *     stored R, and the k-split tickets (bytes 256..4095, see
+ *     glowq_workspace_bytes_for);
  *   - for T > 16, the fp32 partial sums of R split along d into up to 8 slices
  *     (added in a fixed order, so R does not depend on timing);
  *   - the solo call's R.
- * 0 when r == 0 or T == 0.  The caller allocates it once and may reuse it
- * across calls issued in order on one stream (any T); calls that may overlap
- * need separate workspaces.  Ownership: caller's device memory, 16-byte
- * aligned.  The first 256 bytes must be zero before the first call that uses
- * the workspace; every call that completes leaves them zero.  After a call
- * returned GLOWQ_ERR_CUDA, or glowq_get_device_status reported
- * GLOWQ_ERR_TIMEOUT, zero them again.
+ * 0 when r == 0 or T == 0 (no workspace is required then).  The caller
+ * allocates it once and may reuse it across calls issued in order on one
+ * stream (any T); calls that may overlap need separate workspaces.
+ * Ownership: caller's device memory, 16-byte aligned.  The first 4096 bytes
+ * must be zero before the first call that uses the workspace; every call that
+ * completes leaves them zero.  After a call returned GLOWQ_ERR_CUDA, or
+ * glowq_get_device_status reported GLOWQ_ERR_TIMEOUT, zero them again.
  */
 GLOWQ_API size_t glowq_workspace_bytes(int64_t T, int32_t r);
+
+/*
+ * Workspace size that also lets one forward call of this shape split the
+ * reduction over d across CTA pairs (any r >= 0, also r == 0):
+ *   T, r, d        as for the forward call
+ *   out_features   host array of the m modules' output widths
+ * Small batches (16 < T <= 64) run the tensor-core GEMM on 64-token tiles,
+ * whose 256-row tiles are too few to occupy every SM (an o_proj or down_proj
+ * has 16-20); each tile's d range is then split into S parts of whole
+ * 128-groups, each part stores its fp32 sums to a slot behind the other
+ * workspace regions (2 x 128 x 64 x 4 bytes per part), and the part that
+ * counts last on the tile's ticket (zero region, bytes 256..4095) adds the S
+ * slots in ascending part order and stores Y.  The order of the sum is fixed,
+ * so Y does not depend on timing; no CTA waits for another.  A forward call
+ * splits only when it is given a workspace (workspace_bytes) larger than
+ * glowq_workspace_bytes(T, r) plus the solo R, and uses as many parts as fit;
+ * with less it runs whole tiles.  Returns glowq_workspace_bytes(T, r) when the
+ * call would not split (T <= 16, T > 64, enough tiles, invalid arguments).
+ */
+GLOWQ_API size_t glowq_workspace_bytes_for(int64_t T, int32_t r, int64_t d, const int64_t* out_features,
+                                           int32_t m);
 
 /*
  * Input-sharing group forward (key design 4): R = X B^T is computed once and
@@ -203,8 +226,10 @@ GLOWQ_API size_t glowq_workspace_bytes(int64_t T, int32_t r);
  *   T          tokens (>= 0; T == 0 is a no-op)
  *   R_out      device, T x r fp16 bits (the cached projection; NULL iff r == 0)
  *   workspace  device scratch of at least glowq_workspace_bytes(T, r) bytes
+ *              (glowq_workspace_bytes_for: the size that enables the k-split;
+ *              may be NULL when r == 0; 16-byte aligned when not NULL)
  * Small T (<= 16) runs the weight-streaming decode kernels; larger T runs the
- * tcgen05 tensor-core kernels.  Accumulation is fp32; R and Y are rounded to
+ * tcgen05 tensor-core kernels (64-token tiles up to T = 64, 256 above).  Accumulation is fp32; R and Y are rounded to
  * fp16 (round-to-nearest-even).
  */
 GLOWQ_API glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d,
@@ -310,19 +335,22 @@ GLOWQ_API glowq_status glowq_solo_forward_w4a8(const glowq_module* mod, int64_t 
  * allocation of device memory.
  *   - Sizes whose scratch need, glowq_workspace_bytes(T, r), exceeds
  *     glowq_noalloc_scratch_bytes() are rejected with GLOWQ_ERR_SHAPE before
- *     anything is enqueued.  At r = 64 the largest accepted T is 481 (for
- *     T > 16 the split-d partial sums need 8 x T x r x 4 bytes).
+ *     anything is enqueued.  At r = 64 the largest accepted T is 480 (for
+ *     T > 16 the split-d partial sums need 8 x T x r x 4 bytes).  The rest of
+ *     the array serves the k-split of small batches (glowq_workspace_bytes_for)
+ *     as far as it reaches.
  *   - The first call on a device looks up the array's device address (once per
  *     device, with that device current) and keeps it for the life of the CUDA
  *     context (not across a cudaDeviceReset); make that first call before any
  *     stream capture.
  *   - All calls on a device share the one array, which keeps the last call's
  *     contents: calls that may overlap on the GPU (different streams without
- *     ordering between them) race on it.  Each call (r > 0) first clears the
- *     array's 256 flag bytes on `stream` (cudaMemsetAsync, which allocates
- *     nothing), so flags left non-zero by a failed or timed-out call never
- *     reach the next one; every other value a call reads there is written
- *     earlier by the same call.
+ *     ordering between them) race on it.  Each call first clears the
+ *     array's 4096-byte zero region (hand-off flags, k-split tickets) on
+ *     `stream` (cudaMemsetAsync, which allocates nothing), so flags or tickets
+ *     left non-zero by a failed or timed-out call never reach the next one;
+ *     every other value a call reads there is written earlier by the same
+ *     call.
  */
 GLOWQ_API glowq_status glowq_solo_forward_noalloc(const glowq_module* mod, int64_t d, const uint16_t* B,
                                                   int32_t r, const uint16_t* X, int64_t T, void* stream);

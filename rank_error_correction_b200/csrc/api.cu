@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" boundary of libglowq: argument validation, path
 // dispatch (decode kernels for T <= 16, tcgen05 kernels above) and launches.
 // Argument meaning, layouts and error behaviour are documented in glowq.h.
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 
@@ -44,11 +45,11 @@ static int device_sm_count() {
 
 static size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace layout (r > 0): [hand-off flags, 256 B][R partials][solo R].
-// The flags are the decode GEMV's (producers of R -> consumers) and sit at
-// offset 0 for every T, so a prefill call sharing the workspace never
-// overwrites them.
-static size_t workspace_flag_bytes(int32_t r) { return r > 0 ? 256 : 0; }
+// Workspace layout: [zero region, 4 KB][R partials][solo R][k-split slots].
+// The zero region holds the decode GEMV's hand-off flags (producers of R ->
+// consumers) and the tcgen05 GEMM's k-split tickets; it sits at offset 0 for
+// every T, so no other call sharing the workspace overwrites it.
+static size_t workspace_flag_bytes(int32_t r) { return r > 0 ? kWorkspaceZeroBytes : 0; }
 
 // fp32 partial sums of R = X B^T split along d: up to 16 slices for T <= 16
 // (decode), up to 8 when the prefill token tiles alone would not fill the GPU.
@@ -95,9 +96,17 @@ glowq_status validate_solo_call(const glowq_module* mod, int64_t d, const uint16
 // the decode kernels write R = fp16(s_t X' B^T) there, the prefill kernels
 // write the unscaled fp16(X' B^T) there for the GEMM and fp16(s_t X' B^T) to
 // R_scaled (when not null).
+// Offset of the k-split slots: behind everything else the call may use.
+static size_t split_base_bytes(int64_t T, int32_t r) {
+    return kWorkspaceZeroBytes + workspace_partial_bytes(T, r) + workspace_solo_R_bytes(T, r);
+}
+
+// split_bytes: the workspace's size when the bytes behind split_base_bytes(T, r)
+// may hold k-split slots (0: no split).
 static glowq_status forward_views(const ModuleView* hm, int32_t m, int64_t d, const uint16_t* B, int32_t r,
-                                  const uint16_t* X, int64_t T, uint16_t* R, void* workspace, cudaStream_t st,
-                                  int fmt, const float* tok_scale = nullptr, uint16_t* R_scaled = nullptr) {
+                                  const uint16_t* X, int64_t T, uint16_t* R, void* workspace, size_t split_bytes,
+                                  cudaStream_t st, int fmt, const float* tok_scale = nullptr,
+                                  uint16_t* R_scaled = nullptr) {
     if (T == 0) return GLOWQ_OK;
     const bool use_r = r > 0;
     float* partial = (use_r && workspace_partial_bytes(T, r) > 0)
@@ -109,17 +118,28 @@ static glowq_status forward_views(const ModuleView* hm, int32_t m, int64_t d, co
                                            partial, device_sm_count(), st, fmt, tok_scale);
         return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;
     }
+    unsigned int* tickets = nullptr;
+    float* slots = nullptr;
+    int64_t max_slots = 0;
+    const size_t base = split_base_bytes(T, r);
+    if (workspace && split_bytes > base) {
+        tickets = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + kTicketOffsetBytes);
+        slots = reinterpret_cast<float*>(static_cast<char*>(workspace) + base);
+        max_slots = (int64_t)((split_bytes - base) / prefill_slot_bytes(prefill_tile_n(T)));
+    }
     return prefill_group_forward(hm, m, (int)d, use_r ? B : nullptr, use_r ? r : 0, X, T, R, partial,
-                                 device_sm_count(), st, fmt, tok_scale, use_r ? R_scaled : nullptr);
+                                 device_sm_count(), st, fmt, tok_scale, use_r ? R_scaled : nullptr, tickets, slots,
+                                 max_slots);
 }
 
 static glowq_status forward_impl(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
-                                 const uint16_t* X, int64_t T, uint16_t* R, void* workspace, cudaStream_t st) {
+                                 const uint16_t* X, int64_t T, uint16_t* R, void* workspace, size_t ws_bytes,
+                                 cudaStream_t st) {
     ModuleView hm[GLOWQ_MAX_MODULES];
     for (int i = 0; i < m; ++i)
         hm[i] = {mods[i].qweight, mods[i].scales, mods[i].zeros, nullptr, (r > 0) ? mods[i].A : nullptr,
                  mods[i].Y, mods[i].ldY, mods[i].out_features};
-    return forward_views(hm, m, d, B, r, X, T, R, workspace, st, GLOWQ_FMT_INT4);
+    return forward_views(hm, m, d, B, r, X, T, R, workspace, ws_bytes, st, GLOWQ_FMT_INT4);
 }
 
 // Validation of MXFP4 / NVFP4 modules and their conversion to module views.
@@ -243,12 +263,28 @@ size_t glowq_workspace_bytes(int64_t T, int32_t r) {
     return workspace_flag_bytes(r) + workspace_partial_bytes(T, r) + workspace_solo_R_bytes(T, r);
 }
 
+size_t glowq_workspace_bytes_for(int64_t T, int32_t r, int64_t d, const int64_t* out_features, int32_t m) {
+    const size_t need = (r >= 0) ? glowq_workspace_bytes(T, r) : 0;
+    if (T <= kDecodeMaxTokens || r < 0 || d <= 0 || d % GLOWQ_GROUP_SIZE != 0 || !out_features || m < 1 ||
+        m > GLOWQ_MAX_MODULES)
+        return need;
+    int64_t mtiles = 0;
+    for (int i = 0; i < m; ++i) {
+        if (out_features[i] <= 0) return need;
+        mtiles += (out_features[i] + 255) / 256;
+    }
+    const SplitPlan p = plan_prefill_split(T, (int)d, mtiles, gemm_max_pairs(device_sm_count()), INT64_MAX);
+    if (p.S <= 1) return need;
+    return split_base_bytes(T, r) + (size_t)p.slots * prefill_slot_bytes(p.bn);
+}
+
 glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,
                                  const uint16_t* X, int64_t T, uint16_t* R_out, void* workspace,
                                  size_t workspace_bytes, void* stream) {
     glowq_status v = validate_forward(mods, m, d, B, r, X, T);
     if (v != GLOWQ_OK) return v;
     if (T == 0) return GLOWQ_OK;
+    if (workspace && !aligned16(workspace)) return GLOWQ_ERR_ALIGN;
     if (r > 0) {
         if (!R_out) return GLOWQ_ERR_ARG;
         if (!aligned16(R_out)) return GLOWQ_ERR_ALIGN;
@@ -256,8 +292,7 @@ glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d,
         if (!workspace || workspace_bytes < need) return GLOWQ_ERR_ARG;
         if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
     }
-    (void)workspace_bytes;
-    return forward_impl(mods, m, d, B, r, X, T, R_out, workspace, (cudaStream_t)stream);
+    return forward_impl(mods, m, d, B, r, X, T, R_out, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r, const uint16_t* X,
@@ -265,6 +300,7 @@ glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16
     glowq_status v = validate_forward(mod, 1, d, B, r, X, T);
     if (v != GLOWQ_OK) return v;
     if (T == 0) return GLOWQ_OK;
+    if (workspace && !aligned16(workspace)) return GLOWQ_ERR_ALIGN;
     uint16_t* R = nullptr;
     if (r > 0) {
         const size_t need = glowq_workspace_bytes(T, r);
@@ -273,8 +309,7 @@ glowq_status glowq_solo_forward(const glowq_module* mod, int64_t d, const uint16
         R = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(workspace) + workspace_flag_bytes(r) +
                                         workspace_partial_bytes(T, r));
     }
-    (void)workspace_bytes;
-    return forward_impl(mod, 1, d, B, r, X, T, R, workspace, (cudaStream_t)stream);
+    return forward_impl(mod, 1, d, B, r, X, T, R, workspace, workspace_bytes, (cudaStream_t)stream);
 }
 
 glowq_status glowq_group_forward_fp4(glowq_format fmt, const glowq_fp4_module* mods, int32_t m, int64_t d,
@@ -284,6 +319,7 @@ glowq_status glowq_group_forward_fp4(glowq_format fmt, const glowq_fp4_module* m
     glowq_status v = fp4_views(fmt, mods, m, d, B, r, X, T, hm);
     if (v != GLOWQ_OK) return v;
     if (T == 0) return GLOWQ_OK;
+    if (workspace && !aligned16(workspace)) return GLOWQ_ERR_ALIGN;
     if (r > 0) {
         if (!R_out) return GLOWQ_ERR_ARG;
         if (!aligned16(R_out)) return GLOWQ_ERR_ALIGN;
@@ -291,7 +327,7 @@ glowq_status glowq_group_forward_fp4(glowq_format fmt, const glowq_fp4_module* m
         if (!workspace || workspace_bytes < need) return GLOWQ_ERR_ARG;
         if (!aligned16(workspace)) return GLOWQ_ERR_ALIGN;
     }
-    return forward_views(hm, m, d, B, r, X, T, R_out, workspace, (cudaStream_t)stream, (int)fmt);
+    return forward_views(hm, m, d, B, r, X, T, R_out, workspace, workspace_bytes, (cudaStream_t)stream, (int)fmt);
 }
 
 glowq_status glowq_solo_forward_fp4(glowq_format fmt, const glowq_fp4_module* mod, int64_t d, const uint16_t* B,
@@ -301,6 +337,7 @@ glowq_status glowq_solo_forward_fp4(glowq_format fmt, const glowq_fp4_module* mo
     glowq_status v = fp4_views(fmt, mod, 1, d, B, r, X, T, hm);
     if (v != GLOWQ_OK) return v;
     if (T == 0) return GLOWQ_OK;
+    if (workspace && !aligned16(workspace)) return GLOWQ_ERR_ALIGN;
     uint16_t* R = nullptr;
     if (r > 0) {
         const size_t need = glowq_workspace_bytes(T, r);
@@ -309,7 +346,7 @@ glowq_status glowq_solo_forward_fp4(glowq_format fmt, const glowq_fp4_module* mo
         R = reinterpret_cast<uint16_t*>(reinterpret_cast<char*>(workspace) + workspace_flag_bytes(r) +
                                         workspace_partial_bytes(T, r));
     }
-    return forward_views(hm, 1, d, B, r, X, T, R, workspace, (cudaStream_t)stream, (int)fmt);
+    return forward_views(hm, 1, d, B, r, X, T, R, workspace, workspace_bytes, (cudaStream_t)stream, (int)fmt);
 }
 
 size_t glowq_solve_workspace_bytes(int64_t rows, int64_t d, int32_t r, int32_t p) {
@@ -407,7 +444,7 @@ static glowq_status w4a8_impl(const glowq_module* mods, int32_t m, int64_t d, co
         R = solo ? Rsolo : Rp;             // the GEMM reads the unscaled R'
         Rs = solo ? nullptr : R_out;
     }
-    return forward_views(hm, m, d, B, r, Xq, T, R, workspace, st, GLOWQ_FMT_INT4, ts, Rs);
+    return forward_views(hm, m, d, B, r, Xq, T, R, workspace, 0, st, GLOWQ_FMT_INT4, ts, Rs);
 }
 
 glowq_status glowq_group_forward_w4a8(const glowq_module* mods, int32_t m, int64_t d, const uint16_t* B, int32_t r,

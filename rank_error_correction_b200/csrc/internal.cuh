@@ -23,6 +23,23 @@ struct ModuleView {
 };
 
 constexpr int kDecodeMaxTokens = 16;
+// Tokens up to which the tcgen05 path uses 64-token pair tiles and may split k.
+constexpr int kSmallBatchMaxTokens = 64;
+
+// Workspace layout: [zero region][R partials][solo R][k-split slots].  The
+// zero region holds the decode hand-off flags (bytes 0..255) and the k-split
+// tickets (bytes 256..4095, one u32 per CTA of a split tile); it must be zero
+// before a call and every call that completes leaves it zero.
+constexpr size_t kWorkspaceZeroBytes = 4096;
+constexpr size_t kTicketOffsetBytes = 256;
+constexpr int kMaxTickets = (int)((kWorkspaceZeroBytes - kTicketOffsetBytes) / 4);
+constexpr int kMaxSplit = 8;          // parts per tile
+constexpr int kMinSplitBlocks = 8;    // k-blocks (of 64) per part, at least
+// Cost of a part's 64 KB of fp32 partial sums in k-blocks of streamed weights
+// (8 KB each at a 64-token tile; the sums stay in L2, ~2.5x HBM's bandwidth):
+// written once by every part, read once by the part that reduces.
+constexpr int kSplitWriteCost = 3;
+constexpr int kSplitReduceCost = 3;
 
 // Argument checks of glowq_solo_forward, without the workspace (api.cu).
 glowq_status validate_solo_call(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r, const uint16_t* X,
@@ -34,8 +51,8 @@ unsigned int* device_status_ptr();
 // decode.cu
 // Corrected GEMV over the stacked rows (T <= 16), one launch.  With r > 0 it
 // also computes R = X B^T (written to R) from fp32 partial sums in `partial`
-// (decode_partial_bytes(T, r)); `flags` are 256 zeroed workspace bytes that
-// every completed call leaves zero.
+// (decode_partial_bytes(T, r)); `flags` are the first 256 bytes of the
+// workspace's zero region, which every completed call leaves zero.
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
                                const uint16_t* B, uint16_t* R, unsigned int* flags, float* partial, int num_sms,
                                cudaStream_t st, int fmt = GLOWQ_FMT_INT4, const float* tok_scale = nullptr);
@@ -77,10 +94,26 @@ bool make_map(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64
               uint64_t pitch, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw);
 // `partial`: scratch of prefill_partial_bytes(T, r) for the split R projection
 // (nullptr: one slice of d per CTA, R written directly).
+// `tickets` (zeroed workspace words) and `slots` (max_slots fp32 partial
+// tiles of prefill_slot_bytes) enable the k-split; nullptr / 0: whole tiles.
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r,
                                    const uint16_t* X, int64_t T, uint16_t* R, float* partial, int num_sms,
                                    cudaStream_t st, int fmt = GLOWQ_FMT_INT4, const float* tok_scale = nullptr,
-                                   uint16_t* R_scaled = nullptr);
+                                   uint16_t* R_scaled = nullptr, unsigned int* tickets = nullptr,
+                                   float* slots = nullptr, int64_t max_slots = 0);
 size_t prefill_partial_bytes(int64_t T, int r);
+// Work decomposition of the tcgen05 GEMM: token width bn of the pair tiles,
+// tiles [0, split_from) whole, the rest split into S parts of kbs k-blocks;
+// slots = fp32 partial tiles the split needs.
+struct SplitPlan {
+    int bn;
+    int64_t ntiles_n, ntiles, split_from;
+    int S, kbs;
+    int64_t slots;
+};
+SplitPlan plan_prefill_split(int64_t T, int d, int64_t mtiles, int pairs, int64_t max_slots);
+int gemm_max_pairs(int num_sms);
+int prefill_tile_n(int64_t T);
+size_t prefill_slot_bytes(int bn);
 
 }  // namespace glowq

@@ -18,9 +18,9 @@
 namespace {
 
 constexpr size_t kNoallocScratchBytes = (size_t)1 << 20;   // 1 MiB per device
-// The decode kernels' hand-off flags sit in the first bytes of any workspace
-// and must read zero when a call starts.
-constexpr size_t kFlagBytes = 256;
+// The first 4 KB of any workspace (the decode kernels' hand-off flags and the
+// tensor-core GEMM's k-split tickets) must read zero when a call starts.
+constexpr size_t kZeroBytes = 4096;
 
 // Lives in every device that loads the library, for the life of the process.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
@@ -68,12 +68,10 @@ glowq_status glowq_solo_forward_noalloc(const glowq_module* mod, int64_t d, cons
     glowq_status err = GLOWQ_OK;
     void* scratch = scratch_for_current_device(&err);
     if (!scratch) return err;
-    if (r > 0) {
-        // The array keeps whatever the previous call left, including flags a
-        // failed or timed-out call may have left non-zero: clear them, ordered
-        // on the caller's stream before this call's kernels (no allocation).
-        if (cudaMemsetAsync(scratch, 0, kFlagBytes, (cudaStream_t)stream) != cudaSuccess) return GLOWQ_ERR_CUDA;
-    }
+    // The array keeps whatever the previous call left, including flags or
+    // tickets a failed or timed-out call may have left non-zero: clear them,
+    // ordered on the caller's stream before this call's kernels (no allocation).
+    if (cudaMemsetAsync(scratch, 0, kZeroBytes, (cudaStream_t)stream) != cudaSuccess) return GLOWQ_ERR_CUDA;
     return glowq_solo_forward(mod, d, B, r, X, T, scratch, kNoallocScratchBytes, stream);
 }
 

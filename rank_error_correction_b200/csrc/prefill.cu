@@ -149,23 +149,32 @@ __device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
 // ---------------------------------------------------------------------------
 constexpr int kBM = 128;          // W rows per CTA (TMEM lanes)
 constexpr int kPairM = 2 * kBM;   // W rows per pair tile (MMA M)
-constexpr int kBN = 256;          // tokens per pair tile (MMA N, TMEM columns)
-constexpr int kHalfN = kBN / 2;   // tokens staged by each CTA
 constexpr int kBK = 64;           // k per stage: one 128-byte swizzle atom of fp16
 constexpr int kGemmStages = 6;                // even: each stage belongs to one transform group
 constexpr int kEpiBufs = 1;                   // epilogue staging buffers
-constexpr int kXBytes = kHalfN * kBK * 2;    // 16 KB
 constexpr int kWBytes = kBM * kBK * 2;       // 16 KB
 constexpr int kQBytes = kBM * (kBK / 8) * 4; // 4 KB packed codes (32B-swizzled rows)
-constexpr int kStageBytesG = kXBytes + kWBytes + kQBytes;   // multiple of 1024
 constexpr int kGemmThreads = 448;            // 14 warps
 constexpr int kTransformThreads = 256;
 constexpr int kEpiThreads = 128;
-constexpr int kAccCols = 2 * kBN;            // double-buffered accumulator
 constexpr int kEpiChunk = 32;                // tokens per epilogue chunk (TMEM columns)
 constexpr int kEpiBytes = kEpiChunk * kBM * 2;   // 8 KB: [32 tokens][128 rows] fp16
 static_assert(kGemmStages % 2 == 0, "transform groups own alternate stages");
-static_assert(kGemmStages * kStageBytesG + kEpiBufs * kEpiBytes + 1024 + 256 <= 232448, "shared memory per CTA");
+
+// The pair tile's token width BN (MMA N, TMEM columns per accumulator): 256
+// for prefill, 64 for small batches (17 <= T <= 64), where N = 256 would
+// spend four times the MMA time of the tokens present on every k-block.
+template <int BN>
+struct PairTile {
+    static constexpr int kN = BN;                          // tokens per pair tile
+    static constexpr int kHalf = BN / 2;                   // tokens staged by each CTA
+    static constexpr int kXBytes = kHalf * kBK * 2;        // X half-tile of a stage
+    static constexpr int kStageBytes = kXBytes + kWBytes + kQBytes;   // multiple of 1024
+    static constexpr int kAccCols = 2 * BN;                // double-buffered accumulator
+    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "MMA N (cta_group::2, M = 256)");
+    static_assert(kStageBytes % 1024 == 0, "stage buffers hold whole swizzle atoms");
+    static_assert(kGemmStages * kStageBytes + kEpiBufs * kEpiBytes + 1024 + 256 <= 232448, "shared memory per CTA");
+};
 
 struct PrefillModule {
     const void* s;     // INT4 fp16 scales [O][d/128]; MXFP4 / NVFP4 scale bytes [O][d/32] / [O][d/16]
@@ -194,6 +203,16 @@ struct PrefillArgs {
     int r;
     int ntiles_n;                          // token tiles
     int ntiles;                            // all pair tiles
+    // k-split work units: tiles [0, split_from) are one unit each; every later
+    // tile is S units, part j covering k-blocks [j kbs, min((j+1) kbs, d/64)).
+    // Each part stores fp32 partial sums to its slot; the last part to count
+    // itself on the tile's ticket adds the S slots in ascending j and stores y.
+    int split_from;
+    int S;
+    int kbs;                               // k-blocks per part (even: whole 128-groups)
+    int nunits;
+    float* slots;                          // [(tile - split_from) S + j][2 CTAs][128 rows][BN tokens] fp32
+    unsigned int* tickets;                 // [(tile - split_from)][2 CTAs], zero between calls
     int wait_dep;                          // R comes from the preceding (PDL) kernel
     const float* tok_scale;                // W4A8: per-token scale s_t of the outputs (nullptr: none)
     unsigned int* status;
@@ -206,15 +225,38 @@ struct __align__(8) GemmBarriers {
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint32_t tmem_base;
+    uint32_t last_part;                    // epilogue: this CTA counted last on its tile's ticket
 };
 
 struct TileCoord {
-    int mi, m0, n0, nslab;
+    int mi, m0, n0;
+    int kb0, nkb;     // k-blocks [kb0, kb0 + nkb) of the base product
+    int nslab;        // correction slab blocks (the tile's last part only)
+    int split;        // stored as a partial (0: y stored directly)
+    int slot0;        // slot of part 0 of the tile
+    int part;
+    int ticket;       // ticket index of the tile (times 2 CTAs)
 };
 
-// m0: first W row of the pair tile within module mi; n0: first token.
-__device__ __forceinline__ TileCoord tile_coord(const PrefillArgs& args, int tile) {
+// Work unit u: m0 = first W row of the pair tile within module mi, n0 = first
+// token, and its range of k.
+template <int BN>
+__device__ __forceinline__ TileCoord tile_coord(const PrefillArgs& args, int u) {
     TileCoord c;
+    int tile = u, part = 0, nparts = 1;
+    c.split = 0;
+    c.slot0 = 0;
+    c.ticket = 0;
+    if (u >= args.split_from) {
+        const int v = u - args.split_from;
+        const int rel = v / args.S;
+        part = v - rel * args.S;
+        tile = args.split_from + rel;
+        nparts = args.S;
+        c.split = nparts > 1;
+        c.slot0 = rel * args.S;
+        c.ticket = rel;
+    }
     const int mt = tile / args.ntiles_n;
     const int nt = tile - mt * args.ntiles_n;
     int mi = 0;
@@ -222,8 +264,12 @@ __device__ __forceinline__ TileCoord tile_coord(const PrefillArgs& args, int til
         if (mt >= args.mod[i].mtile_begin) mi = i;
     c.mi = mi;
     c.m0 = (mt - args.mod[mi].mtile_begin) * kPairM;
-    c.n0 = nt * kBN;
-    c.nslab = (args.r > 0 && args.mod[mi].has_A) ? (args.r + kBK - 1) / kBK : 0;
+    c.n0 = nt * BN;
+    const int nkb_all = args.d / kBK;
+    c.part = part;
+    c.kb0 = nparts > 1 ? part * args.kbs : 0;
+    c.nkb = (part == nparts - 1) ? nkb_all - c.kb0 : args.kbs;
+    c.nslab = (part == nparts - 1 && args.r > 0 && args.mod[mi].has_A) ? (args.r + kBK - 1) / kBK : 0;
     return c;
 }
 
@@ -351,20 +397,20 @@ __device__ __forceinline__ uint32_t pf_e4m3_st_f16(uint32_t c, float st) {
 // FMT: GLOWQ_FMT_INT4 (w_hat = fp16((q - z) s)), GLOWQ_FMT_MXFP4 or
 // GLOWQ_FMT_NVFP4 (w_hat = fp16 of the E2M1 value times the block scale,
 // see the transform warps).
-template <int FMT>
+template <int FMT, int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const __grid_constant__ PrefillArgs args) {
+    using TC = PairTile<BN>;
     extern __shared__ __align__(1024) unsigned char gsm_raw[];
     // 1024-byte alignment of the stage buffers (swizzle atoms); the same offset in both CTAs
     unsigned char* gsm = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
-    unsigned char* epi = gsm + kGemmStages * kStageBytesG;            // kEpiBufs x kEpiBytes
+    unsigned char* epi = gsm + kGemmStages * TC::kStageBytes;            // kEpiBufs x kEpiBytes
     GemmBarriers* bars = reinterpret_cast<GemmBarriers*>(epi + kEpiBufs * kEpiBytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nkb = args.d / kBK;
     const uint32_t crank = cluster_ctarank();            // 0 = leader (issues the MMAs)
     const int first_tile = (int)cluster_id_x();
     const int tile_step = (int)cluster_count_x();
     const int row_off = (int)crank * kBM;                // this CTA's W rows within the pair tile
-    const int tok_off = (int)crank * kHalfN;             // this CTA's tokens within the pair tile
+    const int tok_off = (int)crank * TC::kHalf;             // this CTA's tokens within the pair tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
@@ -379,7 +425,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
         fence_mbar_init();
     }
     cluster_sync_all();                                  // barriers of both CTAs initialised
-    if (warp == 1) tmem_alloc_pair(&bars->tmem_base, kAccCols);
+    if (warp == 1) tmem_alloc_pair(&bars->tmem_base, TC::kAccCols);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -391,28 +437,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
         if (lane == 0) {
             bool ok = true, waited = false;
             int g = 0;   // ring position of this CTA
-            for (int tile = first_tile; tile < args.ntiles; tile += tile_step) {
-                const TileCoord c = tile_coord(args, tile);
-                const int nblocks = nkb + c.nslab;
+            for (int unit = first_tile; unit < args.nunits; unit += tile_step) {
+                const TileCoord c = tile_coord<BN>(args, unit);
+                const int nblocks = c.nkb + c.nslab;
                 for (int i = 0; i < nblocks; ++i, ++g) {
                     const int s = g % kGemmStages;
                     if (g >= kGemmStages && ok) ok = mbar_wait(&bars->empty[s], ((g / kGemmStages) - 1) & 1, args.status);
-                    unsigned char* st = gsm + s * kStageBytesG;
-                    const uint32_t xs = smem_u32(st), ws = smem_u32(st + kXBytes), qs = smem_u32(st + kXBytes + kWBytes);
-                    if (i < nkb) {
-                        mbar_arrive_expect_tx(&bars->full[s], kXBytes + kQBytes);
-                        tma_load_2d(xs, &args.tmX, &bars->full[s], i * kBK, c.n0 + tok_off);
+                    unsigned char* st = gsm + s * TC::kStageBytes;
+                    const uint32_t xs = smem_u32(st), ws = smem_u32(st + TC::kXBytes), qs = smem_u32(st + TC::kXBytes + kWBytes);
+                    if (i < c.nkb) {
+                        const int kb = c.kb0 + i;
+                        mbar_arrive_expect_tx(&bars->full[s], TC::kXBytes + kQBytes);
+                        tma_load_2d(xs, &args.tmX, &bars->full[s], kb * kBK, c.n0 + tok_off);
                         if constexpr (FMT == GLOWQ_FMT_INT4)
-                            tma_load_4d(qs, &args.tmQ[c.mi], &bars->full[s], 0, 0, i, (c.m0 + row_off) / 16);
+                            tma_load_4d(qs, &args.tmQ[c.mi], &bars->full[s], 0, 0, kb, (c.m0 + row_off) / 16);
                         else
-                            tma_load_2d(qs, &args.tmQ[c.mi], &bars->full[s], i * (kBK / 8), c.m0 + row_off);
+                            tma_load_2d(qs, &args.tmQ[c.mi], &bars->full[s], kb * (kBK / 8), c.m0 + row_off);
                     } else {
                         if (!waited && args.wait_dep) {   // R is complete
                             pdl_wait();
                             waited = true;
                         }
-                        const int j = i - nkb;
-                        mbar_arrive_expect_tx(&bars->full[s], kXBytes + kWBytes);
+                        const int j = i - c.nkb;
+                        mbar_arrive_expect_tx(&bars->full[s], TC::kXBytes + kWBytes);
                         tma_load_2d(xs, &args.tmR, &bars->full[s], j * kBK, c.n0 + tok_off);
                         tma_load_2d(ws, &args.tmA[c.mi], &bars->full[s], j * kBK, c.m0 + row_off);
                     }
@@ -425,10 +472,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
     } else if (warp == 1) {
         // ---------------- MMA issuer (leader CTA) ----------------
         if (crank == 0 && lane == 0) {
-            constexpr uint32_t idesc = f16_idesc(kPairM, kBN);
-            constexpr uint64_t kStageDesc = (uint64_t)(kStageBytesG >> 4);   // descriptor step per stage
+            constexpr uint32_t idesc = f16_idesc(kPairM, TC::kN);
+            constexpr uint64_t kStageDesc = (uint64_t)(TC::kStageBytes >> 4);   // descriptor step per stage
             // loop-invariant addresses: everything per stage is base + stage * step
-            const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(gsm + kXBytes));   // W of stage 0
+            const uint64_t adesc0 = sw128_kmajor_desc(smem_u32(gsm + TC::kXBytes));   // W of stage 0
             const uint64_t bdesc0 = sw128_kmajor_desc(smem_u32(gsm));             // X of stage 0
             const uint32_t empty_l0 = smem_u32(&bars->empty[0]);
             const uint32_t empty_p0 = cluster_addr(&bars->empty[0], 1);
@@ -441,13 +488,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
             // this position's MMAs are issued, so the shared-memory round trip of
             // the probe does not idle the tensor pipe.
             bool next_ready = false;
-            for (int tile = first_tile; tile < args.ntiles; tile += tile_step, ++tl) {
-                const TileCoord c = tile_coord(args, tile);
-                const int nblocks = nkb + c.nslab;
+            for (int unit = first_tile; unit < args.nunits; unit += tile_step, ++tl) {
+                const TileCoord c = tile_coord<BN>(args, unit);
+                const int nblocks = c.nkb + c.nslab;
                 const int buf = tl & 1;
                 if (tl >= 2 && ok) ok = mbar_wait_cluster(&bars->acc_empty[buf], ((tl >> 1) - 1) & 1, args.status);
                 tc_fence_after();
-                const uint32_t dacc = tmem + (uint32_t)(buf * kBN);
+                const uint32_t dacc = tmem + (uint32_t)(buf * TC::kN);
                 for (int i = 0; i < nblocks; ++i) {
                     // both CTAs' w_hat written and TMA landed (slab blocks: TMA only)
                     if (!next_ready && ok) ok = mbar_wait_cluster(&bars->dq[s], ph, args.status);
@@ -489,17 +536,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
         // scale/zero of the current and the next 3 groups (a shift register
         // refilled 4 groups ahead, across tile boundaries)
         int cur_tile = first_tile;
-        int f_tile = cur_tile, f_grp = 0;              // next group to fetch
-        TileCoord fc = tile_coord(args, cur_tile < args.ntiles ? cur_tile : 0);
+        int f_tile = cur_tile, f_grp = 0;              // next group to fetch (unit, group within it)
+        TileCoord fc = tile_coord<BN>(args, cur_tile < args.nunits ? cur_tile : 0);
         // per group: INT4 (s | z << 16) in .x; MXFP4 the four block scales as
         // fp16 in .x .y; NVFP4 the eight fp16_RN(e4m3 * s_t) in .x .. .w
         auto fetch = [&]() -> uint4 {
             uint4 v = make_uint4(0, 0, 0, 0);
-            if (f_tile < args.ntiles) {
+            if (f_tile < args.nunits) {
                 const int orow = fc.m0 + row_off + row;
                 const PrefillModule& FM = args.mod[fc.mi];
                 if (orow < FM.O) {
-                    const int64_t o = (int64_t)orow * ngroups + f_grp;
+                    const int64_t o = (int64_t)orow * ngroups + (fc.kb0 >> 1) + f_grp;
                     if constexpr (FMT == GLOWQ_FMT_INT4) {
                         v.x = (uint32_t)__half_as_ushort(static_cast<const __half*>(FM.s)[o]) |
                               ((uint32_t)FM.z[o] << 16);
@@ -516,27 +563,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                         v.w = pf_e4m3_st_f16(e8.y >> 16, st) | (pf_e4m3_st_f16(e8.y >> 24, st) << 16);
                     }
                 }
-                if (++f_grp == ngroups) {
+                if (++f_grp == (fc.nkb >> 1)) {
                     f_grp = 0;
                     f_tile += tile_step;
-                    if (f_tile < args.ntiles) fc = tile_coord(args, f_tile);
+                    if (f_tile < args.nunits) fc = tile_coord<BN>(args, f_tile);
                 }
             }
             return v;
         };
         uint4 sz0 = fetch(), sz1 = fetch(), sz2 = fetch(), sz3 = fetch();
-        for (; cur_tile < args.ntiles; cur_tile += tile_step) {
-            const TileCoord cc = tile_coord(args, cur_tile);
-            const int nblocks = nkb + cc.nslab;
-            // nkb is even, so block i of the tile (group i/2) is ours when (gbase + i) % 2 == par
+        for (; cur_tile < args.nunits; cur_tile += tile_step) {
+            const TileCoord cc = tile_coord<BN>(args, cur_tile);
+            const int nblocks = cc.nkb + cc.nslab;
+            // a unit's nkb is even, so block i of it (group i/2) is ours when (gbase + i) % 2 == par
             for (int i = (par ^ gbase) & 1; i < nblocks; i += 2) {
                 const int g = gbase + i;
                 const int s = g % kGemmStages;
                 if (ok) ok = mbar_wait(&bars->full[s], (g / kGemmStages) & 1, args.status);
-                if (i < nkb) {
-                    unsigned char* st = gsm + s * kStageBytesG;
+                if (i < cc.nkb) {
+                    unsigned char* st = gsm + s * TC::kStageBytes;
                     // 32-byte-swizzled INT4 rows: 16-byte half h of row r sits at r*32 + ((h ^ (r>>2)&1) << 4)
-                    const unsigned char* qrow = st + kXBytes + kWBytes + row * 32;
+                    const unsigned char* qrow = st + TC::kXBytes + kWBytes + row * 32;
                     const uint4 qa = *reinterpret_cast<const uint4*>(qrow + (hsw << 4));
                     const uint4 qb = *reinterpret_cast<const uint4*>(qrow + ((hsw ^ 1u) << 4));
                     const uint4 sz = sz0;                            // group i/2 (one block of it is ours)
@@ -546,7 +593,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
                     sz3 = fetch();
                     const uint32_t words[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
                     // row `row` of the W tile: 8 chunks of 16 B (8 fp16 in k order), chunk c at c ^ (row % 8)
-                    unsigned char* wrow = st + kXBytes + (row >> 3) * 1024 + (row & 7) * 128;
+                    unsigned char* wrow = st + TC::kXBytes + (row >> 3) * 1024 + (row & 7) * 128;
                     if constexpr (FMT != GLOWQ_FMT_INT4) {
                         // this k-block is half (i & 1) of its group: 2 MXFP4 / 4 NVFP4 blocks;
                         // word c holds k 8c .. 8c+7 (bytes = pairs in k order)
@@ -606,48 +653,113 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
         // shared memory ([32 tokens][128 rows] fp16) and written by one TMA
         // store, which clips rows >= O and tokens >= T.  A staging buffer is
         // rewritten only after the store issued from it has finished reading it.
+        // A part of a k-split tile instead stores its fp32 sums to its slot,
+        // frees the accumulator, and counts itself on the tile's ticket; the
+        // part that counts last adds the tile's slots in ascending part order
+        // (the same order whichever part is last, so y does not depend on
+        // timing) and stores y.  No CTA waits for another.
         const int quarter = warp & 3;                  // TMEM lanes 32*quarter .. +31
         const int row = quarter * 32 + lane;
         const bool leader = (warp == 10 && lane == 0);
         bool ok = true;
         int tl = 0, chunk = 0;
-        for (int tile = first_tile; tile < args.ntiles; tile += tile_step, ++tl) {
-            const TileCoord c = tile_coord(args, tile);
-            const int buf = tl & 1;
+        // fp16 of 32 tokens of this thread's row -> staging buffer -> TMA store
+        auto store_chunk = [&](const float (&f)[32], const TileCoord& c, int ch) {
+            unsigned char* sb = epi + (chunk % kEpiBufs) * kEpiBytes;
+            ++chunk;
+            if (leader) bulk_wait_read<kEpiBufs - 1>();   // the store from this buffer is done reading
+            named_barrier_sync(1, kEpiThreads);
+            __half* col = reinterpret_cast<__half*>(sb) + row;
+            const int tok0 = c.n0 + ch * kEpiChunk;
+            if (args.tok_scale) {   // W4A8: y = s_t (X' w_hat^T + R' A^T), one rounding
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const float ts = (tok0 + j < args.T) ? __ldg(args.tok_scale + tok0 + j) : 0.f;
+                    col[j * kBM] = __float2half_rn(f[j] * ts);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) col[j * kBM] = __float2half_rn(f[j]);
+            }
+            fence_proxy_async_smem();
+            named_barrier_sync(1, kEpiThreads);
             const int orow0 = c.m0 + row_off;
+            if (leader && orow0 < args.mod[c.mi].O && tok0 < args.T) {
+                tma_store_2d(&args.tmY[c.mi], smem_u32(sb), orow0, tok0);
+                bulk_commit();
+            }
+        };
+        for (int unit = first_tile; unit < args.nunits; unit += tile_step, ++tl) {
+            const TileCoord c = tile_coord<BN>(args, unit);
+            const int buf = tl & 1;
             if (ok) ok = mbar_wait(&bars->acc_full[buf], (tl >> 1) & 1, args.status);
             tc_fence_after();
-            const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * kBN);
+            const uint32_t tacc = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * TC::kN);
+            if (!c.split) {
 #pragma unroll 1
-            for (int ch = 0; ch < kBN / kEpiChunk; ++ch, ++chunk) {
+                for (int ch = 0; ch < TC::kN / kEpiChunk; ++ch) {
+                    uint32_t v[32];
+                    tmem_ld32(tacc + ch * kEpiChunk, v);
+                    float f[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) f[j] = __uint_as_float(v[j]);
+                    store_chunk(f, c, ch);
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(cluster_addr(&bars->acc_empty[buf], 0));   // buffer may be overwritten
+                continue;
+            }
+            // this part's sums: slot [128 rows][BN tokens] of this CTA
+            const size_t slot_floats = (size_t)kBM * BN;
+            float* mine = args.slots + ((size_t)(c.slot0 + c.part) * 2 + crank) * slot_floats + (size_t)row * BN;
+#pragma unroll 1
+            for (int ch = 0; ch < TC::kN / kEpiChunk; ++ch) {
                 uint32_t v[32];
                 tmem_ld32(tacc + ch * kEpiChunk, v);
-                unsigned char* sb = epi + (chunk % kEpiBufs) * kEpiBytes;
-                if (leader) bulk_wait_read<kEpiBufs - 1>();   // the store from this buffer is done reading
-                named_barrier_sync(1, kEpiThreads);
-                __half* col = reinterpret_cast<__half*>(sb) + row;
-                if (args.tok_scale) {   // W4A8: y = s_t (X' w_hat^T + R' A^T), one rounding
-                    const int t0 = c.n0 + ch * kEpiChunk;
+                float4* dst = reinterpret_cast<float4*>(mine + ch * kEpiChunk);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const float ts = (t0 + j < args.T) ? __ldg(args.tok_scale + t0 + j) : 0.f;
-                        col[j * kBM] = __float2half_rn(__uint_as_float(v[j]) * ts);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) col[j * kBM] = __float2half_rn(__uint_as_float(v[j]));
-                }
-                fence_proxy_async_smem();
-                named_barrier_sync(1, kEpiThreads);
-                const int tok0 = c.n0 + ch * kEpiChunk;
-                if (leader && orow0 < args.mod[c.mi].O && tok0 < args.T) {
-                    tma_store_2d(&args.tmY[c.mi], smem_u32(sb), orow0, tok0);
-                    bulk_commit();
-                }
+                for (int q = 0; q < 8; ++q)
+                    __stcg(dst + q, make_float4(__uint_as_float(v[4 * q]), __uint_as_float(v[4 * q + 1]),
+                                                __uint_as_float(v[4 * q + 2]), __uint_as_float(v[4 * q + 3])));
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(cluster_addr(&bars->acc_empty[buf], 0));   // buffer may be overwritten
+            if (lane == 0) mbar_arrive_remote(cluster_addr(&bars->acc_empty[buf], 0));   // sums are in the slot
+            __threadfence();                               // this thread's slot stores before the count
+            named_barrier_sync(1, kEpiThreads);
+            if (leader) {
+                unsigned int* tk = args.tickets + c.ticket * 2 + crank;
+                unsigned int prev;
+                asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(tk) : "memory");
+                const uint32_t last = (prev == (unsigned)(args.S - 1)) ? 1u : 0u;
+                if (last) atomicExch(tk, 0u);             // every part has counted: ready for the next call
+                *reinterpret_cast<volatile uint32_t*>(&bars->last_part) = last;
+            }
+            named_barrier_sync(1, kEpiThreads);
+            if (*reinterpret_cast<volatile uint32_t*>(&bars->last_part) == 0u) continue;
+            __threadfence();                               // the other parts' slots are visible
+            const float* part0 = args.slots + ((size_t)c.slot0 * 2 + crank) * slot_floats + (size_t)row * BN;
+#pragma unroll 1
+            for (int ch = 0; ch < TC::kN / kEpiChunk; ++ch) {
+                float f[32];
+#pragma unroll 1
+                for (int p = 0; p < args.S; ++p) {
+                    const float4* src = reinterpret_cast<const float4*>(part0 + (size_t)p * 2 * slot_floats + ch * kEpiChunk);
+                    float4 x[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) x[q] = __ldcg(src + q);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        if (p == 0) {
+                            f[4 * q] = x[q].x; f[4 * q + 1] = x[q].y; f[4 * q + 2] = x[q].z; f[4 * q + 3] = x[q].w;
+                        } else {
+                            f[4 * q] += x[q].x; f[4 * q + 1] += x[q].y; f[4 * q + 2] += x[q].z; f[4 * q + 3] += x[q].w;
+                        }
+                    }
+                }
+                store_chunk(f, c, ch);
+            }
         }
         if (leader) bulk_wait_all();
     }
@@ -656,7 +768,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
     tc_fence_before();
     __syncwarp();
     cluster_sync_all();                                  // no arrivals or MMA reads into either CTA remain
-    if (warp == 1) tmem_dealloc_pair(tmem, kAccCols);
+    if (warp == 1) tmem_dealloc_pair(tmem, TC::kAccCols);
 }
 
 // ---------------------------------------------------------------------------
@@ -896,19 +1008,23 @@ static bool make_map_q4(CUtensorMap* map, const void* q, int d, int64_t O) {
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static size_t gemm_smem_bytes() {
-    return (size_t)kGemmStages * kStageBytesG + kEpiBufs * kEpiBytes + sizeof(GemmBarriers) + 1024;
+static size_t gemm_smem_bytes(int bn) {
+    return (size_t)kGemmStages * (bn == 64 ? PairTile<64>::kStageBytes : PairTile<256>::kStageBytes) +
+           kEpiBufs * kEpiBytes + sizeof(GemmBarriers) + 1024;
 }
 // CTA pairs of the GEMM that can be resident at once (one CTA per SM).
-static int gemm_max_pairs(int num_sms) {
+int gemm_max_pairs(int num_sms) {
     static int cached_dev = -1, cached = 0;
     int dev = 0;
-    cudaGetDevice(&dev);
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return num_sms / 2;
+    }
     if (dev == cached_dev) return cached;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(num_sms / 2 * 2));
     cfg.blockDim = dim3(kGemmThreads);
-    cfg.dynamicSmemBytes = gemm_smem_bytes();
+    cfg.dynamicSmemBytes = gemm_smem_bytes(256);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -917,7 +1033,10 @@ static int gemm_max_pairs(int num_sms) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, (const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4>, &cfg) != cudaSuccess ||
+    if (cudaFuncSetAttribute((const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4, 256>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes(256)) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&clusters, (const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4, 256>, &cfg) !=
+            cudaSuccess ||
         clusters <= 0) {
         cudaGetLastError();
         clusters = num_sms / 2;
@@ -927,6 +1046,49 @@ static int gemm_max_pairs(int num_sms) {
     cached = clusters;
     return cached;
 }
+
+int prefill_tile_n(int64_t T) { return T <= kSmallBatchMaxTokens ? 64 : 256; }
+size_t prefill_slot_bytes(int bn) { return (size_t)2 * kBM * bn * sizeof(float); }
+
+// Work decomposition of the tcgen05 GEMM.  Small batches (tile width 64) are
+// weight-streaming: with few 256-row tiles (an o_proj or down_proj has 16-20)
+// most CTA pairs would idle, so each tile's k range is split into S parts
+// (whole 128-groups, at least kMinSplitBlocks k-blocks each) when that
+// shortens the busiest pair's work: the k-blocks it streams plus, in the same
+// units, the partial sums it writes (kSplitWriteCost per part) and reads back
+// when it reduces a tile (kSplitReduceCost per part).  Larger T keeps whole
+// tiles.
+SplitPlan plan_prefill_split(int64_t T, int d, int64_t mtiles, int pairs, int64_t max_slots) {
+    SplitPlan p;
+    p.bn = prefill_tile_n(T);
+    p.ntiles_n = (T + p.bn - 1) / p.bn;
+    p.ntiles = mtiles * p.ntiles_n;
+    const int nkb = d / kBK;
+    p.split_from = p.ntiles;
+    p.S = 1;
+    p.kbs = nkb;
+    p.slots = 0;
+    if (p.bn != 64 || pairs <= 0 || p.ntiles <= 0) return p;
+    int64_t best = (p.ntiles + pairs - 1) / pairs * (int64_t)nkb;
+    for (int S = 2; S <= kMaxSplit; ++S) {
+        const int kbs = ((nkb + S - 1) / S + 1) & ~1;
+        if (kbs < kMinSplitBlocks) break;
+        if ((int64_t)(S - 1) * kbs >= nkb) continue;      // the last part would be empty
+        const int64_t units = p.ntiles * S;
+        if (units > max_slots || p.ntiles * 2 > kMaxTickets) break;
+        const int64_t cost =
+            (units + pairs - 1) / pairs * (int64_t)(kbs + kSplitWriteCost) + (int64_t)S * kSplitReduceCost;
+        if (cost < best) {
+            best = cost;
+            p.S = S;
+            p.kbs = kbs;
+            p.split_from = 0;
+            p.slots = units;
+        }
+    }
+    return p;
+}
+
 static size_t rproj_smem_bytes(int rn) { return (size_t)kRStages * rproj_stage_bytes(rn) + sizeof(RprojBarriers) + 1024; }
 
 static cudaError_t launch_with(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
@@ -986,9 +1148,17 @@ cudaError_t launch_rproj_prefill(const uint16_t* X, const uint16_t* B, int64_t T
     return launch_with((const void*)rproj_sum_kernel, dim3((unsigned)((n4 + 255) / 256)), dim3(256), 0, st, true, a2);
 }
 
+template <int BN>
+static const void* gemm_kernel_for(int fmt) {
+    return fmt == GLOWQ_FMT_MXFP4   ? (const void*)corrected_gemm_kernel<GLOWQ_FMT_MXFP4, BN>
+           : fmt == GLOWQ_FMT_NVFP4 ? (const void*)corrected_gemm_kernel<GLOWQ_FMT_NVFP4, BN>
+                                    : (const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4, BN>;
+}
+
 glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const uint16_t* B, int r, const uint16_t* X,
                                    int64_t T, uint16_t* R, float* partial, int num_sms, cudaStream_t st, int fmt,
-                                   const float* tok_scale, uint16_t* R_scaled) {
+                                   const float* tok_scale, uint16_t* R_scaled, unsigned int* tickets, float* slots,
+                                   int64_t max_slots) {
     if (T > ((int64_t)1 << 30)) return GLOWQ_ERR_SHAPE;
     if (!encode_fn()) return GLOWQ_ERR_CUDA;
     const bool use_r = r > 0 && B != nullptr;
@@ -998,23 +1168,28 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     }
     static bool opted = false;
     if (!opted) {
-        if (cudaFuncSetAttribute((const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes()) != cudaSuccess ||
-            cudaFuncSetAttribute((const void*)corrected_gemm_kernel<GLOWQ_FMT_MXFP4>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes()) != cudaSuccess ||
-            cudaFuncSetAttribute((const void*)corrected_gemm_kernel<GLOWQ_FMT_NVFP4>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes()) != cudaSuccess)
-            return GLOWQ_ERR_CUDA;
+        const int f[3] = {GLOWQ_FMT_INT4, GLOWQ_FMT_MXFP4, GLOWQ_FMT_NVFP4};
+        for (int i = 0; i < 3; ++i)
+            if (cudaFuncSetAttribute(gemm_kernel_for<256>(f[i]), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gemm_smem_bytes(256)) != cudaSuccess ||
+                cudaFuncSetAttribute(gemm_kernel_for<64>(f[i]), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)gemm_smem_bytes(64)) != cudaSuccess)
+                return GLOWQ_ERR_CUDA;
         opted = true;
     }
+    int64_t mtiles = 0;
+    for (int i = 0; i < m; ++i) mtiles += (mods[i].O + kPairM - 1) / kPairM;
+    const int max_pairs = gemm_max_pairs(num_sms);
+    const SplitPlan plan = plan_prefill_split(T, d, mtiles, max_pairs, (tickets && slots) ? max_slots : 0);
+    const int bn = plan.bn;
     PrefillArgs* a = new PrefillArgs;
     std::memset(a, 0, sizeof(*a));
     bool ok = make_map(&a->tmX, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, X, (uint64_t)d, (uint64_t)T, (uint64_t)d * 2, kBK,
-                       kHalfN, CU_TENSOR_MAP_SWIZZLE_128B);
+                       (uint32_t)(bn / 2), CU_TENSOR_MAP_SWIZZLE_128B);
     if (use_r)
         ok = ok && make_map(&a->tmR, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, R, (uint64_t)r, (uint64_t)T, (uint64_t)r * 2, kBK,
-                            kHalfN, CU_TENSOR_MAP_SWIZZLE_128B);
-    int mtiles = 0;
+                            (uint32_t)(bn / 2), CU_TENSOR_MAP_SWIZZLE_128B);
+    int mt = 0;
     for (int i = 0; i < m && ok; ++i) {
         const ModuleView& mv = mods[i];
         ok = ok && ((fmt == GLOWQ_FMT_INT4)
@@ -1033,9 +1208,9 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
         a->mod[i].Y = reinterpret_cast<__half*>(mv.Y);
         a->mod[i].ldY = mv.ldY;
         a->mod[i].O = (int)mv.O;
-        a->mod[i].mtile_begin = mtiles;
+        a->mod[i].mtile_begin = mt;
         a->mod[i].has_A = has_A ? 1 : 0;
-        mtiles += (int)((mv.O + kPairM - 1) / kPairM);
+        mt += (int)((mv.O + kPairM - 1) / kPairM);
     }
     if (!ok) {
         delete a;
@@ -1045,21 +1220,26 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
     a->d = d;
     a->T = (int)T;
     a->r = use_r ? r : 0;
-    a->ntiles_n = (int)((T + kBN - 1) / kBN);
+    a->ntiles_n = (int)plan.ntiles_n;
+    a->ntiles = (int)plan.ntiles;
+    a->split_from = (int)plan.split_from;
+    a->S = plan.S;
+    a->kbs = plan.kbs;
+    a->nunits = (int)(plan.split_from + (plan.ntiles - plan.split_from) * plan.S);
+    a->slots = plan.S > 1 ? slots : nullptr;
+    a->tickets = plan.S > 1 ? tickets : nullptr;
     a->wait_dep = use_r ? 1 : 0;
     a->tok_scale = tok_scale;
     a->status = device_status_ptr();
-    const int64_t ntiles = (int64_t)mtiles * a->ntiles_n;
-    a->ntiles = (int)ntiles;
     void* args[] = {(void*)a};
-    // persistent grid: as many CTA pairs as fit at once (fewer if there are fewer tiles)
-    const int64_t pairs = ntiles < gemm_max_pairs(num_sms) ? ntiles : gemm_max_pairs(num_sms);
+    // persistent grid: as many CTA pairs as fit at once (fewer if there are fewer units)
+    const int64_t pairs = a->nunits < max_pairs ? a->nunits : max_pairs;
     cudaError_t e = cudaSuccess;
     if (pairs > 0) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(2 * pairs));
         cfg.blockDim = dim3(kGemmThreads);
-        cfg.dynamicSmemBytes = gemm_smem_bytes();
+        cfg.dynamicSmemBytes = gemm_smem_bytes(bn);
         cfg.stream = st;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1070,10 +1250,7 @@ glowq_status prefill_group_forward(const ModuleView* mods, int m, int d, const u
         attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
         cfg.numAttrs = use_r ? 2 : 1;
-        const void* kfn = fmt == GLOWQ_FMT_MXFP4   ? (const void*)corrected_gemm_kernel<GLOWQ_FMT_MXFP4>
-                          : fmt == GLOWQ_FMT_NVFP4 ? (const void*)corrected_gemm_kernel<GLOWQ_FMT_NVFP4>
-                                                   : (const void*)corrected_gemm_kernel<GLOWQ_FMT_INT4>;
-        e = cudaLaunchKernelExC(&cfg, kfn, args);
+        e = cudaLaunchKernelExC(&cfg, bn == 64 ? gemm_kernel_for<64>(fmt) : gemm_kernel_for<256>(fmt), args);
     }
     delete a;
     return e == cudaSuccess ? GLOWQ_OK : GLOWQ_ERR_CUDA;

@@ -68,6 +68,8 @@ def lib() -> C.CDLL:
         L.glowq_dequant_fp4.argtypes = [st, p, p, p, i64, i64, p, p]
         L.glowq_workspace_bytes.argtypes = [i64, i32]
         L.glowq_workspace_bytes.restype = C.c_size_t
+        L.glowq_workspace_bytes_for.argtypes = [i64, i32, i64, p, i32]
+        L.glowq_workspace_bytes_for.restype = C.c_size_t
         L.glowq_group_forward.argtypes = [C.POINTER(_Module), i32, i64, p, i32, p, i64, p, p, C.c_size_t, p]
         L.glowq_solo_forward.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p, C.c_size_t, p]
         L.glowq_solo_forward_noalloc.argtypes = [C.POINTER(_Module), i64, p, i32, p, i64, p]
@@ -262,12 +264,25 @@ def workspace_bytes(T: int, r: int) -> int:
     return int(lib().glowq_workspace_bytes(T, r))
 
 
-def alloc_workspace(T: int, r: int, device="cuda"):
-    # zero-filled: the first 256 bytes are the decode kernels' hand-off flags,
-    # which must start at zero (every call leaves them zero)
+def workspace_bytes_for(T: int, r: int, d: int, out_features: Sequence[int]) -> int:
+    """Workspace that also enables the k-split of a call of this shape."""
+    outs = (C.c_int64 * len(out_features))(*[int(o) for o in out_features])
+    return int(lib().glowq_workspace_bytes_for(T, r, d, outs, len(out_features)))
+
+
+def alloc_workspace(T: int, r: int, device="cuda", d: int = 0, out_features: Sequence[int] = ()):
+    # zero-filled: the first 4096 bytes (decode hand-off flags, k-split
+    # tickets) must start at zero (every call leaves them zero)
     import torch
-    n = max(workspace_bytes(T, r), 16)
-    return torch.zeros(n, dtype=torch.uint8, device=device)
+    n = workspace_bytes_for(T, r, d, out_features) if d and out_features else workspace_bytes(T, r)
+    return torch.zeros(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def _auto_workspace(T: int, r: int, d: int, out_features: Sequence[int], device):
+    """The workspace a call allocates for itself (None when it needs none)."""
+    if workspace_bytes_for(T, r, d, out_features) == 0:
+        return None
+    return alloc_workspace(T, r, device, d, out_features)
 
 
 def _module_structs(mods: Sequence[QModule], Ys, use_A: bool):
@@ -296,8 +311,8 @@ def group_forward(mods: Sequence[QModule], B, X, Ys=None, R_out=None, workspace=
             raise ValueError("outputs must have unit column stride")
     if r > 0 and R_out is None:
         R_out = torch.empty((T, r), dtype=torch.float16, device=X.device)
-    if workspace is None and r > 0:
-        workspace = alloc_workspace(T, r, X.device)
+    if workspace is None:
+        workspace = _auto_workspace(T, r, d, [m.out_features for m in mods], X.device)
     arr = _module_structs(mods, Ys, r > 0)
     ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().glowq_group_forward(arr, len(mods), d, _ptr(B), r, _ptr(X), T, _ptr(R_out), _ptr(workspace),
@@ -313,8 +328,8 @@ def solo_forward(mod: QModule, B, X, Y=None, workspace=None, stream=None):
     r = 0 if B is None else int(B.shape[0])
     if Y is None:
         Y = torch.empty((T, mod.out_features), dtype=torch.float16, device=X.device)
-    if workspace is None and r > 0:
-        workspace = alloc_workspace(T, r, X.device)
+    if workspace is None:
+        workspace = _auto_workspace(T, r, d, [mod.out_features], X.device)
     arr = _module_structs([mod], [Y], r > 0)
     ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().glowq_solo_forward(arr, d, _ptr(B), r, _ptr(X), T, _ptr(workspace), ws_n, _stream(stream)),
@@ -359,8 +374,8 @@ def group_forward_fp4(mods: Sequence[FP4Module], B, X, Ys=None, R_out=None, work
         Ys = [torch.empty((T, m.out_features), dtype=torch.float16, device=X.device) for m in mods]
     if r > 0 and R_out is None:
         R_out = torch.empty((T, r), dtype=torch.float16, device=X.device)
-    if workspace is None and r > 0:
-        workspace = alloc_workspace(T, r, X.device)
+    if workspace is None:
+        workspace = _auto_workspace(T, r, d, [m.out_features for m in mods], X.device)
     arr = _fp4_structs(mods, Ys, r > 0)
     ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().glowq_group_forward_fp4(fmt, arr, len(mods), d, _ptr(B), r, _ptr(X), T, _ptr(R_out),
@@ -375,8 +390,8 @@ def solo_forward_fp4(mod: FP4Module, B, X, Y=None, workspace=None, stream=None):
     r = 0 if B is None else int(B.shape[0])
     if Y is None:
         Y = torch.empty((T, mod.out_features), dtype=torch.float16, device=X.device)
-    if workspace is None and r > 0:
-        workspace = alloc_workspace(T, r, X.device)
+    if workspace is None:
+        workspace = _auto_workspace(T, r, d, [mod.out_features], X.device)
     arr = _fp4_structs([mod], [Y], r > 0)
     ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().glowq_solo_forward_fp4(mod.fmt, arr, d, _ptr(B), r, _ptr(X), T, _ptr(workspace), ws_n,
@@ -396,8 +411,8 @@ class ForwardPlan:
         _require_cuda(B, X)
         T, d = X.shape
         r = 0 if B is None else int(B.shape[0])
-        if r > 0 and workspace is None:
-            workspace = alloc_workspace(T, r, X.device)
+        if workspace is None:
+            workspace = _auto_workspace(T, r, d, [m.out_features for m in mods], X.device)
         if not solo and r > 0 and R_out is None:
             R_out = torch.empty((T, r), dtype=torch.float16, device=X.device)
         self._keep = (mods, B, X, Ys, R_out, workspace)

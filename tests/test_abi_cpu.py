@@ -42,12 +42,37 @@ def test_workspace_bytes(L):
     assert glowq.workspace_bytes(0, 64) == 0
     assert glowq.workspace_bytes(16, 0) == 0
     small = glowq.workspace_bytes(16, 64)
-    # hand-off flags + up to 16 d-slices of fp32 partial sums of R + solo R
-    assert small == 256 + 16 * 16 * 64 * 4 + 16 * 64 * 2
-    assert glowq.workspace_bytes(1, 64) == 256 + 16 * 64 * 4 + 256     # solo R rounded up to 256 B
+    # zero region (hand-off flags, k-split tickets) + up to 16 d-slices of fp32
+    # partial sums of R + solo R
+    assert small == 4096 + 16 * 16 * 64 * 4 + 16 * 64 * 2
+    assert glowq.workspace_bytes(1, 64) == 4096 + 16 * 64 * 4 + 256    # solo R rounded up to 256 B
     big = glowq.workspace_bytes(2048, 64)
-    assert big >= 256 + 8 * 2048 * 64 * 4 + 2048 * 64 * 2   # flags + split-d fp32 partials of R + solo R
+    assert big >= 4096 + 8 * 2048 * 64 * 4 + 2048 * 64 * 2  # zero region + split-d fp32 partials of R + solo R
     assert small % 256 == 0 and big % 256 == 0
+
+
+def test_workspace_bytes_for_the_k_split(L):
+    """Sizing of the small-batch k-split (host arithmetic only): slots of
+    2 x 128 rows x 64 tokens fp32 behind the other regions, S parts per tile."""
+    slot = 2 * 128 * 64 * 4
+    # no split outside 16 < T <= 64, or for bad arguments
+    for T in (1, 16, 65, 2048):
+        assert glowq.workspace_bytes_for(T, 64, 4096, [4096]) == glowq.workspace_bytes(T, 64)
+    assert glowq.workspace_bytes_for(40, 64, 200, [4096]) == glowq.workspace_bytes(40, 64)
+    assert glowq.workspace_bytes_for(40, 64, 4096, []) == glowq.workspace_bytes(40, 64)
+    # LLaMA-2-13B down_proj at T = 64: 20 tiles of 256 rows, far fewer than the CTA pairs
+    for T, r, d, outs in [(64, 64, 13824, [5120]), (17, 64, 4096, [1024]), (40, 32, 4096, [512, 256]),
+                          (48, 0, 8192, [512])]:
+        n = glowq.workspace_bytes_for(T, r, d, outs)
+        base = (glowq.workspace_bytes(T, r) if r else 4096)
+        assert n > base and (n - base) % slot == 0, (T, r, d, outs)
+        tiles = sum(-(-o // 256) for o in outs)
+        parts, rem = divmod((n - base) // slot, tiles)
+        assert rem == 0 and 2 <= parts <= 8, (T, d, outs, parts)
+        # every part holds at least 8 k-blocks of 64 (4 groups of 128)
+        assert -(-(d // 64) // parts) >= 8
+    # enough tiles to fill the GPU: whole tiles
+    assert glowq.workspace_bytes_for(64, 64, 4096, [4096] * 8) == glowq.workspace_bytes(64, 64)
 
 
 def _mods(n, O=128, q=0x1000, Y=0x2000, ldY=128, A=0x3000):
@@ -77,7 +102,7 @@ def test_host_validation_errors(L):
     assert _gf(L, _mods(1), R=None) == 1                # ... and R_out
     assert _gf(L, _mods(1), T=64, wsb=16) == 1          # workspace too small (T > 16 splits R)
     assert _gf(L, _mods(1), T=4, ws=None, wsb=0) == 1   # decode with r > 0 needs the hand-off flags
-    assert _gf(L, _mods(1), T=4, wsb=128) == 1          # ... all 256 bytes of them
+    assert _gf(L, _mods(1), T=4, wsb=128) == 1          # ... the whole zero region
     assert _gf(L, _mods(1), T=4, ws=0x7008) == 3        # misaligned workspace
     assert _gf(L, _mods(1), T=-1) == 1
     assert _gf(L, _mods(1), T=0) == 0                   # empty batch: no-op

@@ -75,7 +75,7 @@ def test_noalloc_size_boundary():
     import torch
     r, d, O = 64, 256, 64
     Tmax = _largest_T(r)
-    assert Tmax == 481                       # 256 + 8*T*r*4 + align256(T*r*2) <= 1 MiB
+    assert Tmax == 480                       # 4096 + 8*T*r*4 + align256(T*r*2) <= 1 MiB
     mods = make_modules(d, [O], seed=97)
     B = attach_random_factors(mods, d, r, seed=97)
     m = to_dev(mods)[0]
