@@ -832,14 +832,30 @@ def profile_case(case, device, steps=4):
     that the ncu summaries under profiles/ are captured from.  Launch order per
     step -- decode: corrected_gemv (Q/K/V group), corrected_gemv (o_proj);
     prefill: rproj_tc, rproj_sum, corrected_gemm
-    (gate/up), rproj_tc, rproj_sum, corrected_gemm (down_proj)."""
+    (gate/up), rproj_tc, rproj_sum, corrected_gemm (down_proj); small
+    (LLaMA-2-13B o_proj and down_proj solos at decode batch T = 64, k-split
+    64-token tiles): rproj_tc, rproj_sum, corrected_gemm (o_proj), rproj_tc,
+    rproj_sum, corrected_gemm (down_proj)."""
     import torch
-    from rank_error_correction_b200 import glowq
+    from rank_error_correction_b200 import glowq, synth
     if case == "decode":
         reps = build_replicas(8, 1, device)
         io = make_io(1, device)
         for i in range(steps):
             run_step(reps[i % len(reps)], io)
+    elif case == "small":
+        T = 64
+        units = []
+        for k, (outs, d) in enumerate((([5120], 5120), ([5120], 13824))):
+            mods, B = build_unit(outs, d, 0, 10 * k, device)
+            X = synth.device_activations(T, d, 0, sub=700 + k, device=device)
+            ws = torch.zeros(max(glowq.workspace_bytes_for(T, R_RANK, d, outs), 16), dtype=torch.uint8,
+                             device=device)
+            Y = torch.empty((T, outs[0]), dtype=torch.float16, device=device)
+            units.append((mods[0], B, X, Y, ws))
+        for i in range(steps):
+            for m, B, X, Y, ws in units:
+                glowq.solo_forward(m, B, X, Y=Y, workspace=ws)
     else:
         time_prefill(2048, 1, 0, device, n_rep=1, eager_steps=steps)
     torch.cuda.synchronize()
@@ -863,7 +879,7 @@ def main():
     ap.add_argument("--no-solve", action="store_true", help="skip the GPU offline solve line")
     ap.add_argument("--no-units", action="store_true",
                     help="skip the per-unit lines (LLaMA-3.1-8B layer, LLaMA-2-13B decode batches)")
-    ap.add_argument("--profile-case", choices=["decode", "prefill"],
+    ap.add_argument("--profile-case", choices=["decode", "prefill", "small"],
                     help="run a few untimed steps of one workload and exit (for ncu captures)")
     args = ap.parse_args()
 

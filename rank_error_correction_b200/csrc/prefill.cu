@@ -113,6 +113,10 @@ __device__ __forceinline__ void tma_store_2d(const void* map, uint32_t src, int 
                  : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Fetch a TMA descriptor (a kernel parameter) ahead of its first use.
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
 template <int N>
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -412,6 +416,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
     const int row_off = (int)crank * kBM;                // this CTA's W rows within the pair tile
     const int tok_off = (int)crank * TC::kHalf;             // this CTA's tokens within the pair tile
 
+    if (threadIdx.x == 32) {   // descriptors, fetched while thread 0 initialises the barriers
+        prefetch_tmap(&args.tmX);
+        if (args.r > 0) prefetch_tmap(&args.tmR);
+        for (int i = 0; i < args.m; ++i) {
+            prefetch_tmap(&args.tmQ[i]);
+            if (args.mod[i].has_A) prefetch_tmap(&args.tmA[i]);
+            prefetch_tmap(&args.tmY[i]);
+        }
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < kGemmStages; ++s) {
             mbar_init(&bars->full[s], 1);
@@ -742,19 +755,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) corrected_gemm_kernel(const _
             const float* part0 = args.slots + ((size_t)c.slot0 * 2 + crank) * slot_floats + (size_t)row * BN;
 #pragma unroll 1
             for (int ch = 0; ch < TC::kN / kEpiChunk; ++ch) {
+                // two parts' loads in flight per L2 round trip, added in ascending part order
                 float f[32];
+                const float4* src0 = reinterpret_cast<const float4*>(part0 + ch * kEpiChunk);
 #pragma unroll 1
-                for (int p = 0; p < args.S; ++p) {
-                    const float4* src = reinterpret_cast<const float4*>(part0 + (size_t)p * 2 * slot_floats + ch * kEpiChunk);
-                    float4 x[8];
+                for (int p = 0; p < args.S; p += 2) {
+                    const float4* src = src0 + (size_t)p * (2 * slot_floats / 4);
+                    const bool pair = p + 1 < args.S;
+                    float4 x[8], y[8];
 #pragma unroll
                     for (int q = 0; q < 8; ++q) x[q] = __ldcg(src + q);
+                    if (pair) {
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) y[q] = __ldcg(src + 2 * slot_floats / 4 + q);
+                    }
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         if (p == 0) {
                             f[4 * q] = x[q].x; f[4 * q + 1] = x[q].y; f[4 * q + 2] = x[q].z; f[4 * q + 3] = x[q].w;
                         } else {
                             f[4 * q] += x[q].x; f[4 * q + 1] += x[q].y; f[4 * q + 2] += x[q].z; f[4 * q + 3] += x[q].w;
+                        }
+                        if (pair) {
+                            f[4 * q] += y[q].x; f[4 * q + 1] += y[q].y; f[4 * q + 2] += y[q].z; f[4 * q + 3] += y[q].w;
                         }
                     }
                 }
@@ -928,16 +951,22 @@ __global__ void __launch_bounds__(256) rproj_sum_kernel(const float4* __restrict
     pdl_wait();                 // partial sums complete
     const int i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= n4) return;
-    // L2 loads: the partial sums were written while this grid was already resident
-    const uint4 a0 = ldcg_128(partial + i);
-    float4 acc = make_float4(__uint_as_float(a0.x), __uint_as_float(a0.y), __uint_as_float(a0.z), __uint_as_float(a0.w));
-    for (int y = 1; y < chunks; ++y) {
-        const uint4 u = ldcg_128(partial + (int64_t)y * n4 + i);
-        const float4 v = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+    // L2 loads (the partial sums were written while this grid was already
+    // resident), every slice's load in flight at once, added in ascending y
+    uint4 u[kRMaxChunks];
+#pragma unroll
+    for (int y = 0; y < kRMaxChunks; ++y)
+        if (y < chunks) u[y] = ldcg_128(partial + (int64_t)y * n4 + i);
+    float4 acc = make_float4(__uint_as_float(u[0].x), __uint_as_float(u[0].y), __uint_as_float(u[0].z),
+                             __uint_as_float(u[0].w));
+#pragma unroll
+    for (int y = 1; y < kRMaxChunks; ++y) {
+        if (y < chunks) {
+            acc.x += __uint_as_float(u[y].x);
+            acc.y += __uint_as_float(u[y].y);
+            acc.z += __uint_as_float(u[y].z);
+            acc.w += __uint_as_float(u[y].w);
+        }
     }
     uint2 o;
     o.x = h2_as_u32(__floats2half2_rn(acc.x, acc.y));
