@@ -13,7 +13,7 @@ around exactly K steps (all ranks, max over ranks); weights are rotated over
 enough replicas that every step streams its weights from HBM (inputs larger
 than L2).  `e2e` is the same metric through the public API with the token
 activations copied from pinned host memory and the outputs copied back each
-step.  `--impl reference` times the CPU oracle (float64 C) on a bounded sample
+step (one CUDA graph replay per step; the eagerly enqueued figure beside it).  `--impl reference` times the CPU oracle (float64 C) on a bounded sample
 of the same workload.  Multi-GPU runs are independent replicas (the layer has
 no cross-GPU exchange): weak scaling, no data-path collective.
 """
@@ -289,12 +289,15 @@ def time_decode(T, steps, warmup, device, n_rep, gpu_index, want_clocks=True, ra
                 clocks=sampler.summary() if sampler else None, reps=reps, io=io)
 
 
-def time_e2e(T, steps, device, reps, io, ranks=None):
+def time_e2e(T, steps, device, reps, io, ranks=None, graph=True):
     """Public-API steps with host<->device copies of the step's activations and
     outputs: one pinned H2D copy of both calls' inputs, the two calls as
     prepared plans (glowq.ForwardPlan: arguments marshalled once per replica),
     one D2H copy of both calls' outputs (Q/K/V and o_proj write column blocks
-    of one T x 16384 buffer through ldY)."""
+    of one T x 16384 buffer through ldY).  graph=True: each step is one replay
+    of a CUDA graph captured from exactly those four operations (one graph per
+    weight replica), the way a decode loop is driven; graph=False: the four
+    operations are enqueued eagerly from Python every step."""
     import torch
     from rank_error_correction_b200 import glowq
     Xall = torch.empty((2, T, D), dtype=torch.float16, device=device)
@@ -307,12 +310,13 @@ def time_e2e(T, steps, device, reps, io, ranks=None):
         views.append(Yall[:, c:c + O])
         c += O
     Yo = Yall[:, c:c + O_OUTS[0]]
+    stream = torch.cuda.Stream(device=device)
     plans = []
     for rep in reps:
         mods, B = rep["qkv"]
         mo, Bo = rep["o_proj"]
-        plans.append((glowq.ForwardPlan(mods, B, Xall[0], views, R_out=io["R"], workspace=io["ws"]),
-                      glowq.ForwardPlan([mo[0]], Bo, Xall[1], [Yo], workspace=io["ws"], solo=True)))
+        plans.append((glowq.ForwardPlan(mods, B, Xall[0], views, R_out=io["R"], workspace=io["ws"], stream=stream),
+                      glowq.ForwardPlan([mo[0]], Bo, Xall[1], [Yo], workspace=io["ws"], solo=True, stream=stream)))
     Xh = Xall.cpu().pin_memory()
     Yh = torch.empty((T, ncol), dtype=torch.float16).pin_memory()
     n = min(steps, 200)
@@ -324,19 +328,36 @@ def time_e2e(T, steps, device, reps, io, ranks=None):
         po()
         Yh.copy_(Yall, non_blocking=True)
 
-    for i in range(3):
-        one(i)
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            one(i)
+    stream.synchronize()
+    graphs = []
+    if graph:
+        for i in range(len(plans)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                one(i)
+            graphs.append(g)
+        with torch.cuda.stream(stream):
+            for g in graphs:
+                g.replay()
     torch.cuda.synchronize()
     if ranks is not None:
         ranks.barrier()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for i in range(n):
-        one(i)
-    t1.record()
+    with torch.cuda.stream(stream):
+        t0.record()
+        for i in range(n):
+            if graph:
+                graphs[i % len(graphs)].replay()
+            else:
+                one(i)
+        t1.record()
     torch.cuda.synchronize()
     ms = t0.elapsed_time(t1) / n
+    del graphs
     h2d = Xh.numel() * 2
     d2h = Yh.numel() * 2
     return ms, h2d, d2h, n
@@ -923,6 +944,8 @@ def main():
     launches_per_step = 1 + 1          # one corrected_gemv launch per call (R computed inside it)
     e2e_ms, h2d, d2h, _ = time_e2e(T, args.steps, device, res["reps"], res["io"], ranks=ranks)
     e2e_ms = ranks.max(e2e_ms)
+    e2e_eager_ms, _, _, _ = time_e2e(T, args.steps, device, res["reps"], res["io"], ranks=ranks, graph=False)
+    e2e_eager_ms = ranks.max(e2e_eager_ms)
 
     extra = []
     if not args.no_extra:
@@ -1006,7 +1029,11 @@ def main():
                          "us_per_launch_isolated": qkv_ms * 1e3},
             "o_proj_us": o_ms * 1e3,
             "e2e": {"value": ranks.rate(T, e2e_ms), "unit": "tok/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                    "driven_by": "one CUDA graph replay per step (pinned H2D copy, the two ForwardPlan calls, "
+                                 "D2H copy to pinned host memory)",
+                    "eager": {"value": ranks.rate(T, e2e_eager_ms), "ms_per_step": e2e_eager_ms,
+                              "driven_by": "the same four operations enqueued from Python every step"}},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": res["clocks"],
             "cpu_baseline": cpu,
