@@ -35,11 +35,14 @@ constexpr size_t kTicketOffsetBytes = 256;
 constexpr int kMaxTickets = (int)((kWorkspaceZeroBytes - kTicketOffsetBytes) / 4);
 constexpr int kMaxSplit = 8;          // parts per tile
 constexpr int kMinSplitBlocks = 8;    // k-blocks (of 64) per part, at least
-// Cost of a part's 64 KB of fp32 partial sums in k-blocks of streamed weights
-// (8 KB each at a 64-token tile; the sums stay in L2, ~2.5x HBM's bandwidth):
-// written once by every part, read once by the part that reduces.
-constexpr int kSplitWriteCost = 3;
-constexpr int kSplitReduceCost = 3;
+// Costs of the small-batch work decomposition in k-blocks of streamed weights
+// (fitted to a sweep of S = 1..8 over the LLaMA-2-7B / LLaMA-3.1-8B /
+// LLaMA-2-13B units at T = 32 and 64 on B200, ~0.37 us per k-block): a work
+// unit's fixed cost (ring fill, accumulator drain, stores), and a split tile's
+// partial-sum traffic and reduction, a base plus a share per part.
+constexpr int kUnitCost = 15;
+constexpr int kSplitBaseCost = 6;
+constexpr int kSplitPartCost = 3;
 
 // Argument checks of glowq_solo_forward, without the workspace (api.cu).
 glowq_status validate_solo_call(const glowq_module* mod, int64_t d, const uint16_t* B, int32_t r, const uint16_t* X,

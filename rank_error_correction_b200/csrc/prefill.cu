@@ -1083,9 +1083,9 @@ size_t prefill_slot_bytes(int bn) { return (size_t)2 * kBM * bn * sizeof(float);
 // weight-streaming: with few 256-row tiles (an o_proj or down_proj has 16-20)
 // most CTA pairs would idle, so each tile's k range is split into S parts
 // (whole 128-groups, at least kMinSplitBlocks k-blocks each) when that
-// shortens the busiest pair's work: the k-blocks it streams plus, in the same
-// units, the partial sums it writes (kSplitWriteCost per part) and reads back
-// when it reduces a tile (kSplitReduceCost per part).  Larger T keeps whole
+// shortens the busiest pair's work: per round of units the k-blocks of one
+// unit plus its fixed cost (kUnitCost), and for a split the partial sums and
+// their reduction (kSplitBaseCost + S kSplitPartCost).  Larger T keeps whole
 // tiles.
 SplitPlan plan_prefill_split(int64_t T, int d, int64_t mtiles, int pairs, int64_t max_slots) {
     SplitPlan p;
@@ -1098,15 +1098,32 @@ SplitPlan plan_prefill_split(int64_t T, int d, int64_t mtiles, int pairs, int64_
     p.kbs = nkb;
     p.slots = 0;
     if (p.bn != 64 || pairs <= 0 || p.ntiles <= 0) return p;
-    int64_t best = (p.ntiles + pairs - 1) / pairs * (int64_t)nkb;
+    // Tuning override: GLOWQ_SPLIT_S=S forces S parts per tile (1 <= S <= 8;
+    // ignored when the parts would be empty or the slots or tickets do not fit).
+    if (const char* env = std::getenv("GLOWQ_SPLIT_S")) {
+        const int S = std::atoi(env);
+        if (S == 1) return p;
+        if (S >= 2 && S <= kMaxSplit) {
+            const int kbs = ((nkb + S - 1) / S + 1) & ~1;
+            const int64_t units = p.ntiles * S;
+            if ((int64_t)(S - 1) * kbs < nkb && units <= max_slots && p.ntiles * 2 <= kMaxTickets) {
+                p.S = S;
+                p.kbs = kbs;
+                p.split_from = 0;
+                p.slots = units;
+                return p;
+            }
+        }
+    }
+    int64_t best = (p.ntiles + pairs - 1) / pairs * (int64_t)(nkb + kUnitCost);
     for (int S = 2; S <= kMaxSplit; ++S) {
         const int kbs = ((nkb + S - 1) / S + 1) & ~1;
         if (kbs < kMinSplitBlocks) break;
         if ((int64_t)(S - 1) * kbs >= nkb) continue;      // the last part would be empty
         const int64_t units = p.ntiles * S;
         if (units > max_slots || p.ntiles * 2 > kMaxTickets) break;
-        const int64_t cost =
-            (units + pairs - 1) / pairs * (int64_t)(kbs + kSplitWriteCost) + (int64_t)S * kSplitReduceCost;
+        const int64_t cost = (units + pairs - 1) / pairs * (int64_t)(kbs + kUnitCost) + kSplitBaseCost +
+                             (int64_t)S * kSplitPartCost;
         if (cost < best) {
             best = cost;
             p.S = S;
