@@ -49,12 +49,14 @@ def _margins_intact(buf, nbytes):
 @pytest.mark.parametrize("T", [1, 16, 40, 300])
 def test_group_and_solo_write_inside_their_buffers(T):
     import torch
-    d, outs, r = 1024, [256, 128], 32
+    d, outs, r = 2048, [256, 128], 32          # T = 40 takes the k-split at this d
     mods = make_modules(d, outs, seed=1200 + T)
     B = attach_random_factors(mods, d, r, seed=1200 + T)
     X = synth.activations(T, d, synth.ALPHA_QKV, seed=1200 + T)
     dm = to_dev(mods)
     Bd, Xd = torch.from_numpy(B).cuda(), torch.from_numpy(X).cuda()
+    if T == 40:
+        assert glowq.workspace_bytes_for(T, r, d, outs) > glowq.workspace_bytes(T, r)
 
     # workspace: zero region zero, the rest a pattern the kernels may overwrite
     wsn = max(glowq.workspace_bytes_for(T, r, d, outs), glowq.workspace_bytes_for(T, r, d, outs[1:]))
