@@ -1382,41 +1382,42 @@ static bool validated_shape(int rt, int kw, int kc, int stages, int T, int d, in
 // Work shapes measured on B200 for the LLaMA-2-7B, LLaMA-3.1-8B and LLaMA-2-13B
 // linear shapes at r = 64: every legal (rt, kw, kc, stages) timed as the
 // average call of a CUDA graph of back-to-back calls over weight replicas
-// larger than L2; an entry is kept where it beat the cost model's pick by 3 %
-// or more (o_proj 4096 x 4096 at T = 1: 10.3 -> 8.8 us; 13B gate/up at T = 4:
-// 51.6 -> 35.2 us; the model's pick stays for the other shapes).  The cost
-// model does not see two effects these shapes exploit: a launch that leaves
-// SMs free lets the next call's CTAs start there while it finishes, and a d
-// split across a small cluster shortens each warp's stream without adding
-// CTAs.  Key: row tiles (sum of O / 16), d, token class (T = 1; 2..8; 9..16).
+// larger than L2, at T = 1, 4, 8, 12 and 16; an entry is kept where it beat
+// the shape in force by 3 % or more (o_proj 4096 x 4096 at T = 1: 10.3 ->
+// 8.8 us; 13B gate/up at T = 4: 51.6 -> 35.2 us; 13B Q/K/V at T = 12: 41.0 ->
+// 34.0 us), and a token class without a better shape of its own keeps its
+// neighbour's entry, which the sweep found within 3 % there; the cost model's
+// pick stays for every other shape.  The model does not see two effects these
+// shapes exploit: a launch that leaves SMs free lets the next call's CTAs
+// start there while it finishes, and a split of d across a small cluster
+// shortens each warp's stream without adding CTAs.  Key: row tiles (sum of
+// O / 16), d, token class (T = 1; 2-5; 6-8; 9-12; 13-16, measured at 1, 4, 8,
+// 12, 16).
 struct TunedShape {
     int tiles, d, tclass, rt, kw, kc, stages;
 };
+static int token_class(int T) { return T == 1 ? 0 : T <= 5 ? 1 : T <= 8 ? 2 : T <= 12 ? 3 : 4; }
+// units: o_proj 4096 x 4096 (256, 4096); LLaMA-2-7B Q/K/V 3 x 4096 (768, 4096);
+// LLaMA-3.1-8B Q/K/V 4096 + 1024 + 1024 (384, 4096), gate/up 2 x 14336 (1792,
+// 4096), down_proj (256, 14336); LLaMA-2-7B down_proj (256, 11008); LLaMA-2-13B
+// o_proj (320, 5120), Q/K/V (960, 5120), gate/up 2 x 13824 (1728, 5120),
+// down_proj (320, 13824)
 static const TunedShape kTunedShapes[] = {
-    // T = 1
-    {256, 4096, 0, 7, 1, 2, 8},    // o_proj 4096 x 4096
-    {768, 4096, 0, 4, 1, 2, 4},    // LLaMA-2-7B Q/K/V 3 x 4096
-    {384, 4096, 0, 3, 1, 2, 8},    // LLaMA-3.1-8B Q/K/V 4096 + 1024 + 1024
-    {256, 11008, 0, 5, 1, 4, 4},   // LLaMA-2-7B down_proj
-    {256, 14336, 0, 4, 1, 4, 4},   // LLaMA-3.1-8B down_proj
-    {320, 5120, 0, 3, 4, 1, 4},    // LLaMA-2-13B o_proj
-    {320, 13824, 0, 5, 1, 4, 4},   // LLaMA-2-13B down_proj
-    // 2 <= T <= 8
-    {256, 4096, 1, 7, 1, 2, 8},
-    {384, 4096, 1, 7, 1, 2, 8},
-    {1792, 4096, 1, 15, 1, 2, 4},  // LLaMA-3.1-8B gate/up 2 x 14336
-    {256, 11008, 1, 10, 1, 4, 4},
-    {256, 14336, 1, 12, 1, 6, 4},
-    {320, 5120, 1, 15, 1, 3, 4},
-    {1728, 5120, 1, 12, 1, 2, 4},  // LLaMA-2-13B gate/up 2 x 13824
-    // 9 <= T <= 16
-    {256, 4096, 2, 15, 1, 4, 4},
-    {384, 4096, 2, 15, 1, 4, 4},
-    {1792, 4096, 2, 15, 1, 4, 4},
-    {256, 14336, 2, 10, 1, 8, 4},
-    {320, 5120, 2, 15, 1, 6, 4},
-    {960, 5120, 2, 15, 1, 6, 4},   // LLaMA-2-13B Q/K/V 3 x 5120
-    {320, 13824, 2, 8, 1, 6, 4},
+    {256, 4096, 0, 7, 1, 2, 8},    {768, 4096, 0, 4, 1, 2, 4},   {384, 4096, 0, 3, 1, 2, 8},
+    {256, 14336, 0, 4, 1, 4, 4},   {320, 5120, 0, 3, 4, 1, 4},   {320, 13824, 0, 5, 1, 4, 4},
+    {256, 11008, 0, 5, 1, 4, 4},
+    {256, 4096, 1, 7, 1, 2, 8},    {384, 4096, 1, 7, 1, 2, 8},   {256, 14336, 1, 12, 1, 6, 4},
+    {320, 5120, 1, 15, 1, 3, 4},   {256, 11008, 1, 10, 1, 4, 4}, {1792, 4096, 1, 15, 1, 2, 4},
+    {1728, 5120, 1, 12, 1, 2, 4},
+    {256, 4096, 2, 15, 1, 4, 4},   {384, 4096, 2, 7, 1, 2, 8},   {256, 14336, 2, 12, 1, 6, 4},
+    {320, 5120, 2, 15, 1, 6, 4},   {256, 11008, 2, 10, 1, 4, 4}, {1792, 4096, 2, 14, 1, 2, 4},
+    {1728, 5120, 2, 12, 1, 2, 4},
+    {256, 4096, 3, 15, 1, 4, 4},   {384, 4096, 3, 15, 1, 4, 4},  {256, 14336, 3, 8, 1, 4, 4},
+    {320, 5120, 3, 15, 1, 6, 4},   {320, 13824, 3, 12, 1, 8, 4}, {256, 11008, 3, 12, 1, 6, 4},
+    {1792, 4096, 3, 14, 1, 3, 4},  {960, 5120, 3, 15, 1, 4, 4},  {1728, 5120, 3, 14, 1, 4, 4},
+    {256, 4096, 4, 15, 1, 4, 4},   {384, 4096, 4, 15, 1, 4, 4},  {256, 14336, 4, 10, 1, 8, 4},
+    {320, 5120, 4, 15, 1, 6, 4},   {320, 13824, 4, 8, 1, 6, 4},  {1792, 4096, 4, 15, 1, 4, 4},
+    {960, 5120, 4, 15, 1, 6, 4},
 };
 
 cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int r, const uint16_t* X,
@@ -1458,7 +1459,7 @@ cudaError_t launch_gemv_decode(const ModuleView* mods, int m, int d, int T, int 
     }
     GemvShape sh = choose_shape(tiles, d, T, r, nt, num_sms, fmt);
     {   // measured shapes (at r = 64; also used without a correction, which only removes work)
-        const int tc = (T == 1) ? 0 : (T <= 8 ? 1 : 2);
+        const int tc = token_class(T);
         for (const TunedShape& e : kTunedShapes) {
             GemvShape t;
             if (e.tiles == tiles && e.d == d && e.tclass == tc &&

@@ -1,6 +1,7 @@
 """GPU parity of the decode kernel at every work shape of the library's measured
 shape table: the LLaMA-2-7B, LLaMA-3.1-8B and LLaMA-2-13B units (Q/K/V groups,
-o_proj, gate/up groups, down_proj) at T = 1, 4 and 16 with r = 64, each unit
+o_proj, gate/up groups, down_proj) at one token count of each of the table's
+token classes (T = 1, 4, 7, 11, 16) with r = 64, each unit
 checked on sampled outputs of every module against the oracle.  The table
 replaces the cost model's work shape for these sizes, so each of its entries
 must meet the same parity bar as the shapes the model picks.
@@ -33,9 +34,12 @@ UNITS = {
     "gu_13b": ([13824] * 2, 5120),
     "down_13b": ([5120], 13824),
 }
-# the table's entries: token count -> units
+# the table's entries, one token count per class (T = 1; 2-5; 6-8; 9-12; 13-16)
 CASES = [(1, u) for u in ("o_4096", "qkv_7b", "qkv_8b", "down_7b", "down_8b", "o_13b", "down_13b")] + \
         [(4, u) for u in ("o_4096", "qkv_8b", "gu_8b", "down_7b", "down_8b", "o_13b", "gu_13b")] + \
+        [(7, u) for u in ("o_4096", "qkv_8b", "gu_8b", "down_7b", "down_8b", "o_13b", "gu_13b")] + \
+        [(11, u) for u in ("o_4096", "qkv_8b", "gu_8b", "down_7b", "down_8b", "o_13b", "qkv_13b", "gu_13b",
+                           "down_13b")] + \
         [(16, u) for u in ("o_4096", "qkv_8b", "gu_8b", "down_8b", "o_13b", "qkv_13b", "down_13b")]
 
 _BUILT = {}
