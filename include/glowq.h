@@ -229,7 +229,11 @@ GLOWQ_API size_t glowq_workspace_bytes_for(int64_t T, int32_t r, int64_t d, cons
  *              (glowq_workspace_bytes_for: the size that enables the k-split;
  *              may be NULL when r == 0; 16-byte aligned when not NULL)
  * Small T (<= 16) runs the weight-streaming decode kernels; larger T runs the
- * tcgen05 tensor-core kernels (64-token tiles up to T = 64, 256 above).  Accumulation is fp32; R and Y are rounded to
+ * tcgen05 tensor-core kernels (64-token tiles up to T = 64, 256 above).
+ * Tuning overrides, read from the environment at every call (for measuring,
+ * e.g. with rank_error_correction_b200/tune.py; invalid values are ignored):
+ * GLOWQ_DECODE_SHAPE="rt,kw,kc,stages" sets the decode kernel's work shape,
+ * GLOWQ_SPLIT_S=S the number of parts per tile of the small-batch k-split.  Accumulation is fp32; R and Y are rounded to
  * fp16 (round-to-nearest-even).
  */
 GLOWQ_API glowq_status glowq_group_forward(const glowq_module* mods, int32_t m, int64_t d,
