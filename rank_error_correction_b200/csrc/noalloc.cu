@@ -1,7 +1,8 @@
 // noalloc.cu -- a solo-module forward that allocates nothing.
 //
 // glowq_solo_forward needs a scratch workspace (the projection R = X B^T, the
-// decode hand-off flags and, for T > 16, the split-d partial sums of R).
+// decode hand-off flags, for T > 16 the split-d partial sums of R, and for
+// small batches the k-split's tickets and partial tiles).
 // Normally the caller allocates it.  Some callers cannot allocate device
 // memory when they call us: a custom op or plugin running inside another
 // runtime's enqueue step, where that runtime owns every device allocation and

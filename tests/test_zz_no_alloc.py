@@ -110,8 +110,9 @@ def test_noalloc_rejects_oversized_requests():
 
 def test_noalloc_after_a_timed_out_wait():
     """A bounded wait that ran out (recorded in the device status word) leaves
-    the next allocation-free decode calls correct: each call clears the flag
-    bytes of the shared array before its kernels."""
+    the next allocation-free decode calls correct: each call clears the zero
+    region (hand-off flags, k-split tickets) of the shared array before its
+    kernels."""
     import torch
     glowq.selftest_wait_timeout(polls=64)
     assert glowq.device_status() == 5        # GLOWQ_ERR_TIMEOUT, read and cleared
@@ -123,6 +124,27 @@ def test_noalloc_after_a_timed_out_wait():
     h = mods[0]
     for T in (1, 16):
         X = synth.activations(T, d, synth.ALPHA_MLP, seed=98 + T)
+        rc, got = _noalloc(m, d, Bt, r, torch.from_numpy(X).cuda(), O)
+        assert rc == 0
+        ref = oracle.solo_forward(h.q, h.s, h.z, synth.bits(h.A), synth.bits(B), synth.bits(X))
+        check(got, ref)
+
+
+def test_noalloc_small_batch_split_twice():
+    """A small batch (T = 40) whose 256-row tiles are too few for the GPU takes
+    the k-split inside the fixed array (tickets in its zero region, partial
+    tiles behind R): two calls in a row match the oracle, so the tickets the
+    first call leaves are the zeros the second one needs."""
+    import torch
+    d, O, r, T = 4096, 1024, 64, 40
+    assert glowq.workspace_bytes_for(T, r, d, [O]) > glowq.workspace_bytes(T, r)
+    mods = make_modules(d, [O], seed=96)
+    B = attach_random_factors(mods, d, r, seed=96)
+    m = to_dev(mods)[0]
+    Bt = torch.from_numpy(B).cuda()
+    h = mods[0]
+    for k in range(2):
+        X = synth.activations(T, d, synth.ALPHA_MLP, seed=96 + k)
         rc, got = _noalloc(m, d, Bt, r, torch.from_numpy(X).cuda(), O)
         assert rc == 0
         ref = oracle.solo_forward(h.q, h.s, h.z, synth.bits(h.A), synth.bits(B), synth.bits(X))
