@@ -265,12 +265,12 @@ size_t glowq_workspace_bytes(int64_t T, int32_t r) {
 
 size_t glowq_workspace_bytes_for(int64_t T, int32_t r, int64_t d, const int64_t* out_features, int32_t m) {
     const size_t need = (r >= 0) ? glowq_workspace_bytes(T, r) : 0;
-    if (T <= kDecodeMaxTokens || r < 0 || d <= 0 || d % GLOWQ_GROUP_SIZE != 0 || !out_features || m < 1 ||
-        m > GLOWQ_MAX_MODULES)
+    if (T <= kDecodeMaxTokens || T > ((int64_t)1 << 30) || r < 0 || d <= 0 || d % GLOWQ_GROUP_SIZE != 0 ||
+        d > ((int64_t)1 << 20) || !out_features || m < 1 || m > GLOWQ_MAX_MODULES)
         return need;
     int64_t mtiles = 0;
     for (int i = 0; i < m; ++i) {
-        if (out_features[i] <= 0) return need;
+        if (out_features[i] <= 0 || out_features[i] > ((int64_t)1 << 30)) return need;
         mtiles += (out_features[i] + 255) / 256;
     }
     const SplitPlan p = plan_prefill_split(T, (int)d, mtiles, gemm_max_pairs(device_sm_count()), INT64_MAX);
