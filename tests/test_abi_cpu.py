@@ -60,6 +60,8 @@ def test_workspace_bytes_for_the_k_split(L):
         assert glowq.workspace_bytes_for(T, 64, 4096, [4096]) == glowq.workspace_bytes(T, 64)
     assert glowq.workspace_bytes_for(40, 64, 200, [4096]) == glowq.workspace_bytes(40, 64)
     assert glowq.workspace_bytes_for(40, 64, 4096, []) == glowq.workspace_bytes(40, 64)
+    assert glowq.workspace_bytes_for(40, 64, 1 << 21, [4096]) == glowq.workspace_bytes(40, 64)   # d > 2^20
+    assert glowq.workspace_bytes_for(40, 64, 4096, [0]) == glowq.workspace_bytes(40, 64)
     # LLaMA-2-13B down_proj at T = 64: 20 tiles of 256 rows, far fewer than the CTA pairs
     for T, r, d, outs in [(64, 64, 13824, [5120]), (17, 64, 4096, [1024]), (40, 32, 4096, [512, 256]),
                           (48, 0, 8192, [512])]:
