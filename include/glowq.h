@@ -204,10 +204,13 @@ GLOWQ_API size_t glowq_workspace_bytes(int64_t T, int32_t r);
  * counts last on the tile's ticket (zero region, bytes 256..4095) adds the S
  * slots in ascending part order and stores Y.  The order of the sum is fixed,
  * so Y does not depend on timing; no CTA waits for another.  A forward call
- * splits only when it is given a workspace (workspace_bytes) larger than
- * glowq_workspace_bytes(T, r) plus the solo R, and uses as many parts as fit;
- * with less it runs whole tiles.  Returns glowq_workspace_bytes(T, r) when the
- * call would not split (T <= 16, T > 64, enough tiles, invalid arguments).
+ * splits only when its workspace (workspace_bytes) reaches at least one slot
+ * past the zero region, the partial sums of R and the solo R (past the 4096
+ * zero bytes alone when r == 0), and uses as many parts as the rest holds;
+ * with less it runs whole tiles.  Any workspace passed, also with r == 0,
+ * follows the zero-region rule of glowq_workspace_bytes.  Returns
+ * glowq_workspace_bytes(T, r) when the call would not split (T <= 16, T > 64,
+ * enough tiles, invalid arguments).
  */
 GLOWQ_API size_t glowq_workspace_bytes_for(int64_t T, int32_t r, int64_t d, const int64_t* out_features,
                                            int32_t m);
